@@ -1,0 +1,343 @@
+"""Oracle for one dense single-stream DiT block, its stack, token reduction,
+the INT8 W8A8 variant and the flow-matching Euler loop with velocity reuse.
+
+TEST INFRASTRUCTURE ONLY (see the package docstring).
+
+Sources.  The MiniMax H3 / h3.c pages fix the block's context, not its
+internals:
+  * "MiniMax H3: video and audio generated together" (mobbang.com, model
+    section): H3 is a dense single-stream omni transformer; all frames and the
+    audio track are denoised at once, with attention across frames and
+    modalities.
+  * "h3.c MiniMax H3 inference engine for Mac" (jdon.com, 330B-parameter
+    section): token reduction pairs adjacent video tokens; fused kernels;
+    the QKV arena is reused for the attention heads, then the MLP input.
+  * "antirez/h3.c" (siami.tw, speed/quality control table): reuse 1/2/3 gives
+    20/11/8 fresh DiT evaluations at 20 steps; token reduction merges
+    horizontal video tokens in the middle blocks.
+  * same page, "data" section, and the 21cto.com page's M5 Max section: INT8
+    weight quantisation of the MLP, QKV and attention-output GEMMs;
+    jdon.com "speed vs quality" section: int8 FC2 with one activation scale
+    per row.
+The block form itself (pre-norm RMSNorm with eps 1e-6, QKV, 3D RoPE over
+(frame, row, col) and 1D RoPE for audio, full bidirectional attention,
+output projection + residual, RMSNorm, exact-erf GELU MLP + residual) is the
+one the workload specification states.  Where the pages and the specification
+are silent, the plainest reading is taken; each is named in ``READINGS``.
+
+Precision: fp64 everywhere, int64 for the integer GEMM, and fp32 for the
+quantisation rule (scale = max|row| / 127 in fp32, IEEE fp32 divide,
+round-half-even), which the method fixes in fp32.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+from scipy.special import erf as _erf
+
+__all__ = [
+    "READINGS", "PINS",
+    "rmsnorm", "gelu", "rope_sections", "token_positions", "rope_angles", "apply_rope",
+    "attention", "block_forward", "stack_forward", "token_merge", "token_unmerge",
+    "quantize_rows", "dequantize_rows", "int8_matmul", "dequant_weights", "block_forward_w8a8",
+    "sigmas", "is_fresh", "fresh_steps", "flow_step", "denoise",
+]
+
+# Readings taken where the pages (and the workload specification) leave a step open.
+READINGS = {
+    "block": "no biases, no QK-norm, no timestep modulation, no final norm (none is stated)",
+    "gelu": "exact erf form 0.5*x*(1+erf(x/sqrt2))",
+    "rope_pairs": "interleaved pairs (x[2j], x[2j+1]) within each head",
+    "rope_sections": "video head dims split [frame D/4 | row 3D/8 | col 3D/8]; audio: one 1D section over D",
+    "rope_freq": "pair j of a section of width n rotates by p * theta^(-2j/n), theta = 10000",
+    "rope_positions": "integer (f, r, c) from 0; audio a = 0..A-1 independent of video",
+    "merged_rope": "a merged token (f, r, c') sits at column position 2c'+0.5",
+    "merge": "mean of the horizontally adjacent pair (2c', 2c'+1); audio rows pass through",
+    "unmerge": "plain broadcast of the merged token to both columns",
+    "merge_blocks": "blocks 15..29, 0-indexed, inclusive",
+    "quant": "symmetric, s = max|row|/127 in fp32, q = rint(v/s) half-even, clamp [-127,127], zero row -> s=0,q=0",
+    "int8_coverage": "QKV, attention-output, FC1 and FC2 GEMMs; attention stays bf16",
+    "sigmas": "sigma_i = 1 - i/N, i = 0..N, computed in fp64 and stored fp32",
+    "fresh": "step i is fresh iff i % reuse == 0 or i == N-1",
+    "velocity": "the velocity is the stack output (no in/out projection is stated)",
+    "euler": "x <- x + (sigma_{i+1} - sigma_i) * v over all S tokens at width d",
+    "residual": "fp32 residual stream in every configuration",
+}
+
+# What pins each function to something other than itself (tests/test_oracle_*.py).
+PINS = {
+    "rmsnorm": "closed form on constant rows; unit RMS with g = 1",
+    "gelu": "math.erf closed form at scalar points; tanh approximation within 1e-3; limits",
+    "rope_angles/apply_rope": "hand-computed rotations per section; position 0 = identity; pair norms; "
+                              "relative-position invariance per section",
+    "attention": "pure-Python brute-force softmax attention on tiny inputs; rows sum to 1; "
+                 "uniform-attention closed form",
+    "block_forward": "pure-Python loop block on a tiny case; zero-weight identities; "
+                     "permutation equivariance without RoPE; row sampling = full rows",
+    "token_merge/unmerge": "explicit (f, r, c) loops; unmerge(merge(x)) = x on pair-constant x",
+    "quantize_rows": "hand-computed codes incl. half-even ties; zero row",
+    "int8_matmul": "pure-Python integer dot products",
+    "sigmas/fresh/denoise": "fresh counts 20/11/8 at 20 steps (control table); v = 0 identity; "
+                            "single-step closed form",
+}
+
+
+def _f64(a):
+    return np.asarray(a, dtype=np.float64)
+
+
+# ----------------------------------------------------------------------------- norm / activation
+def rmsnorm(x, g, eps):
+    """u = x * 1/sqrt(mean_j x_j^2 + eps) * g, per row (token)."""
+    x = _f64(x)
+    r = 1.0 / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps)
+    return x * r * _f64(g)
+
+
+def gelu(x):
+    """Exact GELU: 0.5 * x * (1 + erf(x / sqrt(2)))."""
+    x = _f64(x)
+    return 0.5 * x * (1.0 + _erf(x / math.sqrt(2.0)))
+
+
+# ----------------------------------------------------------------------------- RoPE
+def rope_sections(head_dim):
+    """Widths of the (frame, row, col) sections of one head: D/4, 3D/8, the rest."""
+    nf = head_dim // 4
+    nr = 3 * head_dim // 8
+    return nf, nr, head_dim - nf - nr
+
+
+def token_positions(dims, merged=False):
+    """(video positions [V', 3] as (f, r, c) floats, audio positions [A]).
+
+    Video tokens are ordered (f*H + r)*W + c.  After token reduction the grid
+    has W/2 columns and the merged token c' sits at column 2c' + 0.5."""
+    F, H, W, A = dims.frames, dims.rows, dims.cols, dims.n_audio
+    wc = W // 2 if merged else W
+    f, r, c = np.meshgrid(np.arange(F), np.arange(H), np.arange(wc), indexing="ij")
+    col = 2.0 * c + 0.5 if merged else c.astype(np.float64)
+    video = np.stack([f.ravel().astype(np.float64), r.ravel().astype(np.float64), col.ravel()], axis=1)
+    return video, np.arange(A, dtype=np.float64)
+
+
+def rope_angles(dims, merged=False):
+    """Rotation angle of every (token, pair) [S', D/2].
+
+    Video: pair j of the section of width n that carries position p (frame,
+    row or col) turns by p * theta^(-2j/n).  Audio: one section of width D
+    carrying the audio index a."""
+    D, theta = dims.head_dim, float(dims.rope_theta)
+    video, audio = token_positions(dims, merged)
+    cols = []
+    for axis, n in enumerate(rope_sections(D)):
+        j = np.arange(n // 2, dtype=np.float64)
+        omega = theta ** (-2.0 * j / n)
+        cols.append(video[:, axis:axis + 1] * omega[None, :])
+    ang_v = np.concatenate(cols, axis=1)
+    j = np.arange(D // 2, dtype=np.float64)
+    ang_a = audio[:, None] * (theta ** (-2.0 * j / D))[None, :]
+    return np.concatenate([ang_v, ang_a], axis=0)
+
+
+def apply_rope(t, angles, n_heads):
+    """Rotate each interleaved pair (t[2j], t[2j+1]) of every head by angles[:, j]."""
+    t = _f64(t)
+    S = t.shape[0]
+    D = t.shape[1] // n_heads
+    th = t.reshape(S, n_heads, D // 2, 2)
+    c = np.cos(angles)[:, None, :]
+    s = np.sin(angles)[:, None, :]
+    x0, x1 = th[..., 0], th[..., 1]
+    out = np.empty_like(th)
+    out[..., 0] = x0 * c - x1 * s
+    out[..., 1] = x0 * s + x1 * c
+    return out.reshape(S, n_heads * D)
+
+
+# ----------------------------------------------------------------------------- attention
+def attention(q, k, v, n_heads, chunk=2048):
+    """o = softmax(q k^T / sqrt(D)) v per head, every query against every key
+    (bidirectional, no mask).  Query rows are independent; they are taken in
+    chunks only to bound memory."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    Sq = q.shape[0]
+    D = q.shape[1] // n_heads
+    out = np.empty((Sq, n_heads * D))
+    scale = 1.0 / math.sqrt(D)
+    for h in range(n_heads):
+        sl = slice(h * D, (h + 1) * D)
+        kh, vh = k[:, sl], v[:, sl]
+        for r0 in range(0, Sq, chunk):
+            sc = (q[r0:r0 + chunk, sl] @ kh.T) * scale
+            sc -= sc.max(axis=1, keepdims=True)
+            p = np.exp(sc)
+            p /= p.sum(axis=1, keepdims=True)
+            out[r0:r0 + chunk, sl] = p @ vh
+    return out
+
+
+# ----------------------------------------------------------------------------- block / stack
+def block_forward(x, w, dims, merged=False, rows=None, rope=True):
+    """One DiT block on the residual stream x [S', d]:
+
+        u  = RMSNorm(x; g_attn)
+        q, k, v = u W_qkv^T split in thirds; q, k <- RoPE(q), RoPE(k) per head
+        x1 = x + softmax(q k^T / sqrt(D)) v  W_o^T
+        x2 = x1 + GELU(RMSNorm(x1; g_mlp) W_fc1^T) W_fc2^T
+
+    ``rows`` (optional index array) returns x2 only at those tokens; keys and
+    values still cover every token, so the sampled rows equal the full
+    result's rows.  ``rope=False`` leaves q and k unrotated (invariance tests).
+    """
+    x = _f64(x)
+    S, d = x.shape
+    H = dims.n_heads
+    rows = np.arange(S) if rows is None else np.asarray(rows)
+    wqkv = _f64(w["w_qkv"])
+    u = rmsnorm(x, w["g_attn"], dims.eps)
+    k = u @ wqkv[d:2 * d].T
+    v = u @ wqkv[2 * d:3 * d].T
+    q = u[rows] @ wqkv[:d].T
+    if rope:
+        ang = rope_angles(dims, merged)
+        q = apply_rope(q, ang[rows], H)
+        k = apply_rope(k, ang, H)
+    o = attention(q, k, v, H)
+    x1 = x[rows] + o @ _f64(w["w_o"]).T
+    hmid = gelu(rmsnorm(x1, w["g_mlp"], dims.eps) @ _f64(w["w_fc1"]).T)
+    return x1 + hmid @ _f64(w["w_fc2"]).T
+
+
+def token_merge(x, dims):
+    """Token reduction: the merged video token (f, r, c') is the mean of the
+    horizontally adjacent pair (f, r, 2c') and (f, r, 2c'+1); audio rows are
+    carried unchanged after the merged video rows."""
+    x = _f64(x)
+    F, H, W, A = dims.frames, dims.rows, dims.cols, dims.n_audio
+    V = F * H * W
+    vid = x[:V].reshape(F, H, W, -1)
+    m = (vid[:, :, 0::2, :] + vid[:, :, 1::2, :]) * 0.5
+    return np.concatenate([m.reshape(V // 2, -1), x[V:V + A]], axis=0)
+
+
+def token_unmerge(xm, dims):
+    """Inverse of the reduction: each merged token is broadcast back to both
+    columns it came from; audio rows are carried unchanged."""
+    xm = _f64(xm)
+    F, H, W, A = dims.frames, dims.rows, dims.cols, dims.n_audio
+    V = F * H * W
+    vid = xm[:V // 2].reshape(F, H, W // 2, -1)
+    full = np.repeat(vid, 2, axis=2)
+    return np.concatenate([full.reshape(V, -1), xm[V // 2:V // 2 + A]], axis=0)
+
+
+def stack_forward(x, blocks, dims, merge_first=-1, merge_last=-1, block_fn=None):
+    """Blocks 0..L-1 in order; with token reduction on, merge before block
+    ``merge_first`` and unmerge after block ``merge_last`` (inclusive)."""
+    fn = block_forward if block_fn is None else block_fn
+    on = merge_first >= 0
+    x = _f64(x)
+    for layer, w in enumerate(blocks):
+        if on and layer == merge_first:
+            x = token_merge(x, dims)
+        x = fn(x, w, dims, merged=on and merge_first <= layer <= merge_last)
+        if on and layer == merge_last:
+            x = token_unmerge(x, dims)
+    return x
+
+
+# ----------------------------------------------------------------------------- INT8 W8A8
+def quantize_rows(a):
+    """Per-row symmetric int8: s = max|row|/127 (fp32), q = rint(row/s) with an
+    IEEE fp32 divide, half-even, clamped to [-127, 127]; an all-zero row gives
+    s = 0 and q = 0.  Used for weights (per output channel) and for
+    activations (per token)."""
+    a32 = np.asarray(a, dtype=np.float32)
+    s = (np.max(np.abs(a32), axis=1) / np.float32(127.0)).astype(np.float32)
+    q = np.zeros(a32.shape, dtype=np.float32)
+    nz = s > 0
+    q[nz] = np.rint(a32[nz] / s[nz, None])
+    return np.clip(q, -127, 127).astype(np.int8), s
+
+
+def dequantize_rows(q, s):
+    return q.astype(np.float64) * _f64(s)[:, None]
+
+
+def int8_matmul(qa, qw):
+    """Exact integer GEMM: acc[m, n] = sum_k qa[m, k] * qw[n, k] in int64."""
+    return qa.astype(np.int64) @ qw.astype(np.int64).T
+
+
+def dequant_weights(w):
+    """Block weights with each GEMM matrix replaced by its int8 round trip
+    q * s_w (the reference the W8A8 block is held to)."""
+    out = dict(w)
+    for key in ("w_qkv", "w_o", "w_fc1", "w_fc2"):
+        q, s = quantize_rows(w[key])
+        out[key] = dequantize_rows(q, s)
+    return out
+
+
+def _w8a8_linear(a, wq, ws):
+    qa, sa = quantize_rows(a)
+    # integer sums are exact in fp64 here (|acc| < 2^53)
+    acc = qa.astype(np.float64) @ wq.astype(np.float64).T
+    return acc * _f64(sa)[:, None] * _f64(ws)[None, :]
+
+
+def block_forward_w8a8(x, w, dims, merged=False, rope=True):
+    """Diagnostic block with every GEMM input fake-quantised per token as well
+    as the weights per output channel (the full W8A8 arithmetic in fp64)."""
+    x = _f64(x)
+    d, H = x.shape[1], dims.n_heads
+    qw = {k: quantize_rows(w[k]) for k in ("w_qkv", "w_o", "w_fc1", "w_fc2")}
+    u = rmsnorm(x, w["g_attn"], dims.eps)
+    qkv = _w8a8_linear(u, *qw["w_qkv"])
+    q, k, v = qkv[:, :d], qkv[:, d:2 * d], qkv[:, 2 * d:]
+    if rope:
+        ang = rope_angles(dims, merged)
+        q, k = apply_rope(q, ang, H), apply_rope(k, ang, H)
+    o = attention(q, k, v, H)
+    x1 = x + _w8a8_linear(o, *qw["w_o"])
+    g = gelu(_w8a8_linear(rmsnorm(x1, w["g_mlp"], dims.eps), *qw["w_fc1"]))
+    return x1 + _w8a8_linear(g, *qw["w_fc2"])
+
+
+# ----------------------------------------------------------------------------- flow-matching loop
+def sigmas(n_steps):
+    """Linear grid 1 -> 0: sigma_i = 1 - i/N for i = 0..N (fp64, stored fp32)."""
+    return (1.0 - np.arange(n_steps + 1, dtype=np.float64) / n_steps).astype(np.float32)
+
+
+def is_fresh(i, n_steps, reuse):
+    """Whole-velocity reuse: step i runs a fresh DiT evaluation iff
+    i % reuse == 0 or it is the last step."""
+    return i % reuse == 0 or i == n_steps - 1
+
+
+def fresh_steps(n_steps, reuse):
+    return [i for i in range(n_steps) if is_fresh(i, n_steps, reuse)]
+
+
+def flow_step(x, v, sigma_cur, sigma_next):
+    """Euler step of the flow ODE: x + (sigma_next - sigma_cur) * v."""
+    return _f64(x) + (float(sigma_next) - float(sigma_cur)) * _f64(v)
+
+
+def denoise(x0, blocks, dims, n_steps, reuse, merge_first=-1, merge_last=-1, block_fn=None):
+    """N Euler steps over the sigma grid; the velocity is the stack output on
+    fresh steps and the last fresh velocity otherwise.  Returns (x_N, number
+    of fresh evaluations)."""
+    sig = sigmas(n_steps)
+    x = _f64(x0)
+    v = None
+    n_fresh = 0
+    for i in range(n_steps):
+        if is_fresh(i, n_steps, reuse):
+            v = stack_forward(x, blocks, dims, merge_first, merge_last, block_fn)
+            n_fresh += 1
+        x = flow_step(x, v, sig[i], sig[i + 1])
+    return x, n_fresh

@@ -1,0 +1,423 @@
+"""Pins for the CPU oracle: each check ties an oracle function to something
+other than itself (closed forms, pure-Python brute force on tiny inputs,
+invariants, the fresh-evaluation counts printed on the pages)."""
+import json
+import math
+import os
+import random
+import types
+
+import numpy as np
+import pytest
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def dims_of(F, H, W, A, d, h, ffn, eps=1e-6, theta=10000.0):
+    return types.SimpleNamespace(frames=F, rows=H, cols=W, n_audio=A, d=d, n_heads=h,
+                                 head_dim=d // h, ffn=ffn, eps=eps, rope_theta=theta)
+
+
+# ----------------------------------------------------------------------------- RMSNorm / GELU
+def test_rmsnorm_constant_rows_closed_form():
+    eps = 1e-6
+    for c in (0.0, 1e-4, 0.3, -2.5, 1e3):
+        x = np.full((1, 16), c)
+        u = oracle.rmsnorm(x, np.ones(16), eps)
+        assert np.allclose(u, c / math.sqrt(c * c + eps), rtol=1e-15, atol=0)
+
+
+def test_rmsnorm_unit_rms_and_gain():
+    rng = np.random.default_rng(0)
+    x = rng.normal(size=(5, 64)) * 3.0
+    u = oracle.rmsnorm(x, np.ones(64), 0.0)
+    assert np.allclose(np.sqrt(np.mean(u * u, axis=1)), 1.0, rtol=1e-14)
+    g = rng.uniform(0.5, 2.0, size=64)
+    ug = oracle.rmsnorm(x, g, 0.0)
+    assert np.allclose(ug, u * g, rtol=1e-14)
+
+
+def test_gelu_closed_form_and_limits():
+    for v in (-6.0, -1.7, -0.3, 0.0, 0.25, 1.0, 3.3):
+        ref = 0.5 * v * (1.0 + math.erf(v / math.sqrt(2.0)))
+        assert abs(float(oracle.gelu(np.array([v]))[0]) - ref) < 1e-15
+    assert oracle.gelu(np.array([40.0]))[0] == 40.0
+    assert abs(oracle.gelu(np.array([-40.0]))[0]) < 1e-300
+    xs = np.linspace(-5, 5, 1001)
+    tanh_form = 0.5 * xs * (1 + np.tanh(math.sqrt(2 / math.pi) * (xs + 0.044715 * xs ** 3)))
+    assert np.max(np.abs(oracle.gelu(xs) - tanh_form)) < 1e-3
+
+
+# ----------------------------------------------------------------------------- RoPE
+def test_rope_sections():
+    assert oracle.rope_sections(64) == (16, 24, 24)
+    assert oracle.rope_sections(128) == (32, 48, 48)
+
+
+def test_rope_angles_hand_computed():
+    dm = dims_of(3, 4, 5, 3, 128, 2, 512)  # D = 64
+    th = 10000.0
+    ang = oracle.rope_angles(dm)
+    assert ang.shape == (3 * 4 * 5 + 3, 32)
+    t = (2 * 4 + 3) * 5 + 4  # video token (f=2, r=3, c=4)
+    assert ang[t, 0] == pytest.approx(2.0)                       # frame section, pair 0
+    assert ang[t, 1] == pytest.approx(2.0 * th ** (-2 / 16))     # frame section, pair 1
+    assert ang[t, 8] == pytest.approx(3.0)                       # row section starts at pair D/8
+    assert ang[t, 9] == pytest.approx(3.0 * th ** (-2 / 24))
+    assert ang[t, 20] == pytest.approx(4.0)                      # col section starts at pair D/8+3D/16
+    assert ang[t, 31] == pytest.approx(4.0 * th ** (-22 / 24))
+    a = 60 + 2  # audio token 2
+    for j in (0, 5, 31):
+        assert ang[a, j] == pytest.approx(2.0 * th ** (-2 * j / 64))
+    # merged geometry: token (f=1, r=2, c'=1) sits at column 2*1+0.5
+    angm = oracle.rope_angles(dm, merged=True)
+    assert angm.shape == (3 * 4 * 2 + 3, 32)
+    tm = (1 * 4 + 2) * 2 + 1
+    assert angm[tm, 20] == pytest.approx(2.5)
+    assert angm[tm, 0] == pytest.approx(1.0) and angm[tm, 8] == pytest.approx(2.0)
+
+
+def test_apply_rope_rotates_interleaved_pairs():
+    rng = np.random.default_rng(1)
+    S, H, D = 3, 2, 16
+    ang = rng.uniform(-3, 3, size=(S, D // 2))
+    for s in range(S):
+        for j in range(D // 2):
+            e = np.zeros((S, H * D))
+            e[s, D + 2 * j] = 1.0          # head 1, even element of pair j
+            e[s, D + 2 * j + 1] = 0.5      # odd element
+            out = oracle.apply_rope(e, ang, H)
+            c, sn = math.cos(ang[s, j]), math.sin(ang[s, j])
+            assert out[s, D + 2 * j] == pytest.approx(1.0 * c - 0.5 * sn, abs=1e-15)
+            assert out[s, D + 2 * j + 1] == pytest.approx(1.0 * sn + 0.5 * c, abs=1e-15)
+            others = np.delete(out[s], [D + 2 * j, D + 2 * j + 1])
+            assert np.all(others == 0)
+
+
+def test_rope_position_zero_identity_and_norms():
+    dm = dims_of(2, 3, 4, 5, 128, 2, 512)
+    ang = oracle.rope_angles(dm)
+    rng = np.random.default_rng(2)
+    t = rng.normal(size=(ang.shape[0], 128))
+    out = oracle.apply_rope(t, ang, 2)
+    assert np.array_equal(out[0], t[0])                 # video (0,0,0)
+    assert np.array_equal(out[24], t[24])               # audio a = 0
+    pn_in = t.reshape(-1, 64, 2)
+    pn_out = out.reshape(-1, 64, 2)
+    assert np.allclose(np.hypot(pn_in[..., 0], pn_in[..., 1]), np.hypot(pn_out[..., 0], pn_out[..., 1]), rtol=1e-13)
+
+
+def test_rope_relative_position_property():
+    """<R_p q, R_p' k> depends on p - p' only, section by section."""
+    dm = dims_of(4, 6, 6, 8, 64, 1, 256)
+    ang = oracle.rope_angles(dm)
+    rng = np.random.default_rng(3)
+    q, k = rng.normal(size=64), rng.normal(size=64)
+
+    def idx(f, r, c):
+        return (f * 6 + r) * 6 + c
+
+    def dot(i, j):
+        Q = oracle.apply_rope(q[None], ang[i:i + 1], 1)[0]
+        K = oracle.apply_rope(k[None], ang[j:j + 1], 1)[0]
+        return Q @ K
+
+    base = dot(idx(1, 2, 3), idx(0, 4, 1))
+    assert dot(idx(3, 3, 5), idx(2, 5, 3)) == pytest.approx(base, rel=1e-12)
+    assert dot(idx(1, 2, 3), idx(0, 4, 2)) != pytest.approx(base, rel=1e-6)
+    V = 4 * 6 * 6
+    assert dot(V + 1, V + 5) == pytest.approx(dot(V + 3, V + 7), rel=1e-12)
+
+
+# ----------------------------------------------------------------------------- attention
+def brute_attention(q, k, v, H):
+    Sq, HD = len(q), len(q[0])
+    D = HD // H
+    out = [[0.0] * HD for _ in range(Sq)]
+    for h in range(H):
+        for i in range(Sq):
+            sc = [sum(q[i][h * D + e] * k[j][h * D + e] for e in range(D)) / math.sqrt(D) for j in range(len(k))]
+            m = max(sc)
+            w = [math.exp(s - m) for s in sc]
+            z = sum(w)
+            for e in range(D):
+                out[i][h * D + e] = sum(w[j] * v[j][h * D + e] for j in range(len(k))) / z
+    return np.array(out)
+
+
+def test_attention_vs_bruteforce():
+    rng = np.random.default_rng(4)
+    for S, H, D in ((1, 1, 4), (7, 2, 4), (13, 3, 8)):
+        q, k, v = (rng.normal(size=(S, H * D)) * 2 for _ in range(3))
+        ref = brute_attention(q.tolist(), k.tolist(), v.tolist(), H)
+        assert np.allclose(oracle.attention(q, k, v, H, chunk=4), ref, rtol=1e-12, atol=1e-13)
+
+
+def test_attention_uniform_and_convex():
+    rng = np.random.default_rng(5)
+    S, H, D = 9, 2, 8
+    k, v = rng.normal(size=(S, H * D)), rng.normal(size=(S, H * D))
+    o = oracle.attention(np.zeros((S, H * D)), k, v, H)
+    assert np.allclose(o, v.mean(axis=0, keepdims=True), rtol=1e-14)
+    o1 = oracle.attention(rng.normal(size=(S, H * D)), k, np.ones((S, H * D)), H)
+    assert np.allclose(o1, 1.0, rtol=1e-14)
+
+
+# ----------------------------------------------------------------------------- block
+def brute_block(x, w, dm, merged=False):
+    """Pure-Python loops: RMSNorm, QKV, RoPE by explicit (f,r,c)/audio
+    positions, softmax attention, output projection, RMSNorm, GELU MLP."""
+    S, d, H, D, f = len(x), dm.d, dm.n_heads, dm.head_dim, dm.ffn
+    wqkv, wo, w1, w2 = (w[k].tolist() for k in ("w_qkv", "w_o", "w_fc1", "w_fc2"))
+
+    def norm(row, g):
+        r = 1.0 / math.sqrt(sum(a * a for a in row) / d + dm.eps)
+        return [a * r * gg for a, gg in zip(row, g)]
+
+    def mv(W, a):
+        return [sum(wr[i] * a[i] for i in range(len(a))) for wr in W]
+
+    F, Hr, Wc, A = dm.frames, dm.rows, dm.cols, dm.n_audio
+    wc = Wc // 2 if merged else Wc
+    nf, nr = D // 4, 3 * D // 8
+    pos = []
+    for fi in range(F):
+        for ri in range(Hr):
+            for ci in range(wc):
+                pos.append(("v", fi, ri, 2 * ci + 0.5 if merged else ci))
+    for a in range(A):
+        pos.append(("a", a))
+
+    def rot(vec, p):
+        out = list(vec)
+        for h in range(H):
+            for j in range(D // 2):
+                if p[0] == "a":
+                    ang = p[1] * dm.rope_theta ** (-2 * j / D)
+                elif j < nf // 2:
+                    ang = p[1] * dm.rope_theta ** (-2 * j / nf)
+                elif j < (nf + nr) // 2:
+                    ang = p[2] * dm.rope_theta ** (-2 * (j - nf // 2) / nr)
+                else:
+                    nc = D - nf - nr
+                    ang = p[3] * dm.rope_theta ** (-2 * (j - (nf + nr) // 2) / nc)
+                a0, a1 = vec[h * D + 2 * j], vec[h * D + 2 * j + 1]
+                out[h * D + 2 * j] = a0 * math.cos(ang) - a1 * math.sin(ang)
+                out[h * D + 2 * j + 1] = a0 * math.sin(ang) + a1 * math.cos(ang)
+        return out
+
+    u = [norm(row, w["g_attn"].tolist()) for row in x]
+    qkv = [mv(wqkv, row) for row in u]
+    q = [rot(r[:d], pos[i]) for i, r in enumerate(qkv)]
+    k = [rot(r[d:2 * d], pos[i]) for i, r in enumerate(qkv)]
+    v = [r[2 * d:] for r in qkv]
+    o = brute_attention(q, k, v, H).tolist()
+    x1 = [[a + b for a, b in zip(x[i], mv(wo, o[i]))] for i in range(S)]
+    out = []
+    for i in range(S):
+        hvec = mv(w1, norm(x1[i], w["g_mlp"].tolist()))
+        g = [0.5 * a * (1 + math.erf(a / math.sqrt(2))) for a in hvec]
+        out.append([a + b for a, b in zip(x1[i], mv(w2, g))])
+    return np.array(out)
+
+
+def rand_block(rng, d, f, scale=0.2):
+    return {"w_qkv": rng.normal(size=(3 * d, d)) * scale, "w_o": rng.normal(size=(d, d)) * scale,
+            "w_fc1": rng.normal(size=(f, d)) * scale, "w_fc2": rng.normal(size=(d, f)) * scale,
+            "g_attn": rng.uniform(0.5, 1.5, size=d), "g_mlp": rng.uniform(0.5, 1.5, size=d)}
+
+
+@pytest.mark.parametrize("merged", [False, True])
+def test_block_vs_bruteforce(merged):
+    dm = dims_of(1, 2, 4, 2, 32, 2, 64)   # D = 16 -> sections 4/6/6
+    rng = np.random.default_rng(6)
+    S = (4 if merged else 8) + 2
+    x = rng.normal(size=(S, 32))
+    w = rand_block(rng, 32, 64)
+    ref = brute_block(x.tolist(), w, dm, merged)
+    assert np.allclose(oracle.block_forward(x, w, dm, merged=merged), ref, rtol=1e-11, atol=1e-12)
+
+
+def test_block_zero_weight_identities():
+    dm = dims_of(2, 2, 2, 3, 64, 4, 128)
+    rng = np.random.default_rng(7)
+    x = rng.normal(size=(11, 64))
+    w = rand_block(rng, 64, 128)
+    w0 = dict(w, w_o=np.zeros((64, 64)), w_fc2=np.zeros((64, 128)))
+    assert np.array_equal(oracle.block_forward(x, w0, dm), x)
+    # zero QKV -> attention output is 0, block reduces to the MLP branch alone
+    wq = dict(w, w_qkv=np.zeros((192, 64)))
+    mlp = x + oracle.gelu(oracle.rmsnorm(x, w["g_mlp"], 1e-6) @ w["w_fc1"].T) @ w["w_fc2"].T
+    assert np.allclose(oracle.block_forward(x, wq, dm), mlp, rtol=1e-14)
+
+
+def test_block_permutation_equivariant_without_rope():
+    dm = dims_of(2, 2, 2, 3, 64, 4, 128)
+    rng = np.random.default_rng(8)
+    x = rng.normal(size=(11, 64))
+    w = rand_block(rng, 64, 128)
+    perm = rng.permutation(11)
+    a = oracle.block_forward(x, w, dm, rope=False)[perm]
+    b = oracle.block_forward(x[perm], w, dm, rope=False)
+    assert np.allclose(a, b, rtol=1e-12, atol=1e-13)
+    # with RoPE the positions break the symmetry
+    c = oracle.block_forward(x[perm], w, dm)
+    assert not np.allclose(oracle.block_forward(x, w, dm)[perm], c, rtol=1e-6)
+
+
+def test_block_row_sampling_matches_full():
+    dm = dims_of(2, 4, 4, 5, 64, 2, 128)
+    rng = np.random.default_rng(9)
+    x = rng.normal(size=(37, 64))
+    w = rand_block(rng, 64, 128)
+    rows = np.array([0, 5, 31, 32, 36])
+    full = oracle.block_forward(x, w, dm)
+    assert np.allclose(oracle.block_forward(x, w, dm, rows=rows), full[rows], rtol=1e-13, atol=1e-14)
+
+
+# ----------------------------------------------------------------------------- token reduction
+def test_merge_unmerge_explicit_indices():
+    F, H, W, A, d = 2, 3, 4, 3, 5
+    dm = dims_of(F, H, W, A, 8, 1, 8)
+    rng = np.random.default_rng(10)
+    x = rng.normal(size=(F * H * W + A, d))
+    m = oracle.token_merge(x, dm)
+    assert m.shape == (F * H * W // 2 + A, d)
+    for f in range(F):
+        for r in range(H):
+            for c in range(W // 2):
+                i = (f * H + r) * (W // 2) + c
+                assert np.array_equal(m[i], (x[(f * H + r) * W + 2 * c] + x[(f * H + r) * W + 2 * c + 1]) * 0.5)
+    assert np.array_equal(m[F * H * W // 2:], x[F * H * W:])
+    u = oracle.token_unmerge(m, dm)
+    for f in range(F):
+        for r in range(H):
+            for c in range(W):
+                assert np.array_equal(u[(f * H + r) * W + c], m[(f * H + r) * (W // 2) + c // 2])
+    assert np.array_equal(u[F * H * W:], x[F * H * W:])
+
+
+def test_merge_unmerge_identity_on_pair_constant():
+    dm = dims_of(3, 2, 6, 4, 8, 1, 8)
+    rng = np.random.default_rng(11)
+    m = rng.normal(size=(3 * 2 * 3 + 4, 7))
+    x = oracle.token_unmerge(m, dm)           # pair-constant by construction
+    assert np.array_equal(oracle.token_unmerge(oracle.token_merge(x, dm), dm), x)
+    assert np.array_equal(oracle.token_merge(x, dm), m)
+
+
+def test_merge_fp32_single_rounding():
+    """The fp64 mean of two fp32 values, rounded once to fp32, equals the fp32
+    (a + b) * 0.5 -- the property the bit-exact merge check relies on."""
+    rng = np.random.default_rng(12)
+    a = (rng.normal(size=100000) * 10.0 ** rng.integers(-30, 30, size=100000)).astype(np.float32)
+    b = (rng.normal(size=100000) * 10.0 ** rng.integers(-30, 30, size=100000)).astype(np.float32)
+    via64 = ((a.astype(np.float64) + b.astype(np.float64)) * 0.5).astype(np.float32)
+    via32 = (a + b) * np.float32(0.5)
+    assert np.array_equal(via64, via32)
+
+
+# ----------------------------------------------------------------------------- INT8
+def test_quantize_rows_hand_computed():
+    q, s = oracle.quantize_rows(np.array([[127.0, 0.5, 1.5, 2.5, -0.5, -127.0],
+                                          [0.0, 0.0, 0.0, 0.0, 0.0, 0.0],
+                                          [2.0, -1.0, 0.25, 0.0, 1.0, -2.0]]))
+    assert s[0] == 1.0 and s[1] == 0.0
+    assert q[0].tolist() == [127, 0, 2, 2, 0, -127]          # half-even ties
+    assert q[1].tolist() == [0] * 6
+    s2 = np.float32(2.0) / np.float32(127.0)
+    assert s[2] == s2
+    assert q[2].tolist() == [127, int(np.rint(np.float32(-1.0) / s2)), int(np.rint(np.float32(0.25) / s2)), 0,
+                             int(np.rint(np.float32(1.0) / s2)), -127]
+    assert q[2].tolist() == [127, -64, 16, 0, 64, -127]
+
+
+def test_quantize_rows_bounds_and_roundtrip():
+    rng = np.random.default_rng(13)
+    a = rng.normal(size=(50, 300)).astype(np.float32)
+    q, s = oracle.quantize_rows(a)
+    assert q.dtype == np.int8 and s.dtype == np.float32
+    assert np.all(np.abs(q.astype(int)) <= 127)
+    assert np.all(np.max(np.abs(q.astype(int)), axis=1) == 127)
+    assert np.all(np.abs(oracle.dequantize_rows(q, s) - a) <= s[:, None] * 0.5 * (1 + 1e-6))
+
+
+def test_int8_matmul_vs_python():
+    rng = np.random.default_rng(14)
+    qa = rng.integers(-127, 128, size=(5, 37)).astype(np.int8)
+    qw = rng.integers(-127, 128, size=(6, 37)).astype(np.int8)
+    acc = oracle.int8_matmul(qa, qw)
+    for m in range(5):
+        for n in range(6):
+            assert acc[m, n] == sum(int(qa[m, k]) * int(qw[n, k]) for k in range(37))
+    big_a = np.full((1, 4096), 127, np.int8)
+    assert oracle.int8_matmul(big_a, -big_a)[0, 0] == -127 * 127 * 4096
+
+
+def test_w8a8_block_close_to_dequant_reference():
+    dm = dims_of(2, 4, 4, 4, 128, 2, 512)
+    rng = np.random.default_rng(15)
+    x = rng.normal(size=(36, 128))
+    w = rand_block(rng, 128, 512, scale=0.05)
+    ref = oracle.block_forward(x, oracle.dequant_weights(w), dm)
+    diag = oracle.block_forward_w8a8(x, w, dm)
+    rel = np.linalg.norm(diag - ref) / np.linalg.norm(ref)
+    assert 0 < rel < 2e-2
+
+
+# ----------------------------------------------------------------------------- flow-matching loop
+def test_fresh_counts_golden():
+    g = json.load(open(os.path.join(GOLDEN, "fresh_counts.json")))
+    for r, n in g["fresh_evaluations"].items():
+        assert len(oracle.fresh_steps(g["n_steps"], int(r))) == n
+
+
+def test_sigmas_grid():
+    s = oracle.sigmas(20)
+    assert s.dtype == np.float32 and len(s) == 21
+    assert s[0] == 1.0 and s[-1] == 0.0 and np.all(np.diff(s) < 0)
+    assert s[5] == np.float32(0.75)
+
+
+def test_flow_step_zero_velocity_and_closed_form():
+    rng = np.random.default_rng(16)
+    x = rng.normal(size=(4, 8))
+    assert np.array_equal(oracle.flow_step(x, np.zeros_like(x), 0.7, 0.65), x)
+    v = rng.normal(size=(4, 8))
+    dt = float(np.float32(0.7)) - 0.75          # the fp32 sigma, exactly
+    assert np.allclose(oracle.flow_step(x, v, np.float32(0.75), np.float32(0.7)),
+                       x + dt * v, rtol=1e-15, atol=0)
+
+
+def test_denoise_constant_velocity_and_reuse_pattern():
+    dm = dims_of(1, 1, 2, 1, 4, 1, 4)
+    x0 = np.arange(12.0).reshape(3, 4)
+    c = np.full((3, 4), 2.0)
+    for r in (1, 2, 3):
+        xN, nf = oracle.denoise(x0, [None], dm, 20, r, block_fn=lambda x, w, d, merged: c)
+        assert nf == {1: 20, 2: 11, 3: 8}[r]
+        assert np.allclose(xN, x0 - c, atol=1e-12)
+    # v = x on fresh steps only: hand-computed N = 3, reuse 2 -> fresh at 0 and 2
+    s = oracle.sigmas(3).astype(np.float64)
+    xN, nf = oracle.denoise(x0, [None], dm, 3, 2, block_fn=lambda x, w, d, merged: x)
+    v0 = x0
+    x1 = x0 + (s[1] - s[0]) * v0
+    x2 = x1 + (s[2] - s[1]) * v0
+    x3 = x2 + (s[3] - s[2]) * x2
+    assert nf == 2 and np.allclose(xN, x3, rtol=1e-14)
+
+
+def test_stack_merge_window():
+    dm = dims_of(2, 2, 4, 3, 8, 1, 8)
+    seen = []
+
+    def fn(x, w, d, merged):
+        seen.append((len(x), merged))
+        return x * 1.0
+
+    x = np.random.default_rng(17).normal(size=(19, 8))
+    out = oracle.stack_forward(x, [None] * 6, dm, 2, 3, block_fn=fn)
+    assert seen == [(19, False), (19, False), (11, True), (11, True), (19, False), (19, False)]
+    assert np.allclose(out, oracle.token_unmerge(oracle.token_merge(x, dm), dm))
