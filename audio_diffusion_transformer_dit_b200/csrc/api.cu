@@ -1,0 +1,594 @@
+// h3b C ABI: argument validation, workspace planning (aliased activation
+// arenas), the block / stack / denoise orchestration, tracing and the
+// tensor-map encoder.  Every entry point only enqueues work on the caller's
+// stream; nothing here allocates device memory or synchronises (except the
+// explicitly synchronising h3b_device_error / h3b_trace_stop).
+#include <math.h>
+#include <string.h>
+
+#include <mutex>
+#include <vector>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace h3b {
+
+__device__ int g_device_error;  // device error word (one per device)
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  bool ready = false;
+  int num_sms = 0;
+  int* err = nullptr;
+};
+
+std::mutex g_mu;
+DeviceInfo g_dev[kMaxDevices];
+
+int device_ctx(cudaStream_t stream, Ctx* c) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return H3B_ERR_DEVICE;
+  DeviceInfo& di = g_dev[dev];
+  if (!di.ready) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!di.ready) {
+      int major = 0, sms = 0;
+      if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return H3B_ERR_DEVICE;
+      if (major != 10) return H3B_ERR_DEVICE;
+      if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return H3B_ERR_DEVICE;
+      void* p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return H3B_ERR_CUDA;
+      di.num_sms = sms;
+      di.err = static_cast<int*>(p);
+      di.ready = true;
+    }
+  }
+  c->stream = stream;
+  c->err = di.err;
+  c->num_sms = di.num_sms;
+  return H3B_OK;
+}
+
+// ------------------------------------------------------------------ tracing
+struct TraceRec {
+  int kid;
+  cudaEvent_t a, b;
+};
+struct Trace {
+  bool on = false;
+  int cap = 0, n = 0;
+  std::vector<TraceRec> recs;
+  std::vector<float> ms;
+} g_trace;
+
+const char* kKernelNames[KID_COUNT] = {"flow_step", "token_merge", "token_unmerge", "rope_table", "rmsnorm",
+                                       "quant_rows", "quant_absmax", "gemm_qkv_rope", "gemm_o_resid",
+                                       "gemm_fc1_gelu", "gemm_fc2_resid", "gemm", "attention", "memset"};
+
+struct TraceScope {
+  TraceRec* rec = nullptr;
+  cudaStream_t s;
+  TraceScope(int kid, cudaStream_t st) : s(st) {
+    if (g_trace.on && g_trace.n < g_trace.cap) {
+      rec = &g_trace.recs[g_trace.n++];
+      rec->kid = kid;
+      cudaEventRecord(rec->a, s);
+    }
+  }
+  ~TraceScope() {
+    if (rec) cudaEventRecord(rec->b, s);
+  }
+};
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+// ------------------------------------------------------------------ validation
+int check_dims(const h3b_dims* dm) {
+  if (!dm) return H3B_ERR_NULL;
+  if (dm->frames < 0 || dm->rows < 0 || dm->cols < 0 || dm->n_audio < 0) return H3B_ERR_DIMS;
+  if (dm->head_dim != 64 && dm->head_dim != 128) return H3B_ERR_DIMS;
+  if (dm->n_heads <= 0 || dm->d != dm->n_heads * dm->head_dim) return H3B_ERR_DIMS;
+  if (dm->d % 128 != 0 || dm->d > 8192) return H3B_ERR_DIMS;
+  if (dm->ffn <= 0 || dm->ffn % 128 != 0 || dm->ffn > 32768) return H3B_ERR_DIMS;
+  if (!(dm->eps >= 0.f) || !(dm->rope_theta > 0.f)) return H3B_ERR_DIMS;
+  const long long s = 1LL * dm->frames * dm->rows * dm->cols + dm->n_audio;
+  if (s <= 0 || s > (1LL << 24)) return H3B_ERR_DIMS;
+  return H3B_OK;
+}
+
+int seq_len(const h3b_dims& dm, int merged) {
+  return dm.frames * dm.rows * (merged ? dm.cols / 2 : dm.cols) + dm.n_audio;
+}
+
+size_t al256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Workspace layout.  The block's activation arenas alias across its lifetime:
+//   [qkv 3d bf16 | o d bf16 | u1 (norm-1 out)] during the attention half;
+//   the MLP input u2 reuses the QKV arena (offset 0) and the FC1 hidden
+//   overlays the rest (qkv, o and u1 are dead by then).
+struct Plan {
+  size_t qkv, o, u1, oq, u2, g, gq;   // byte offsets inside the arena
+  size_t arena, naive;                // arena bytes, bytes without aliasing
+  size_t s_act, s_g, amax;            // fp32 [S] scale / max vectors (INT8)
+  size_t rope, rope_m, xm;            // RoPE tables, merged-sequence buffer
+  size_t total;
+};
+
+Plan plan(const h3b_dims& dm, int dtype, int reduction) {
+  Plan p{};
+  const size_t S = seq_len(dm, 0), d = dm.d, f = dm.ffn;
+  if (dtype == H3B_INT8) {
+    p.qkv = 0;
+    p.o = al256(6 * d * S);
+    p.u1 = p.o + al256(2 * d * S);
+    p.oq = p.u1 + al256(d * S);
+    const size_t attn_end = p.oq + al256(d * S);
+    p.u2 = 0;
+    p.g = al256(d * S);
+    p.gq = p.g + al256(2 * f * S);
+    const size_t mlp_end = p.gq + al256(f * S);
+    p.arena = attn_end > mlp_end ? attn_end : mlp_end;
+    p.naive = al256(6 * d * S) + al256(2 * d * S) + 3 * al256(d * S) + al256(2 * f * S) + al256(f * S);
+  } else {
+    p.qkv = 0;
+    p.o = al256(6 * d * S);
+    p.u1 = p.o + al256(2 * d * S);
+    const size_t attn_end = p.u1 + al256(2 * d * S);
+    p.u2 = 0;
+    p.g = al256(2 * d * S);
+    const size_t mlp_end = p.g + al256(2 * f * S);
+    p.arena = attn_end > mlp_end ? attn_end : mlp_end;
+    p.oq = p.gq = 0;
+    p.naive = al256(6 * d * S) + 3 * al256(2 * d * S) + al256(2 * f * S);
+  }
+  size_t off = al256(p.arena);
+  p.s_act = off;
+  off += al256(S * 4);
+  p.s_g = off;
+  off += al256(S * 4);
+  p.amax = off;
+  off += al256(S * 4);
+  p.rope = off;
+  off += al256(S * (dm.head_dim / 2) * 8);
+  if (reduction) {
+    const size_t Sm = seq_len(dm, 1);
+    p.rope_m = off;
+    off += al256(Sm * (dm.head_dim / 2) * 8);
+    p.xm = off;
+    off += al256(Sm * d * 4);
+  } else {
+    p.rope_m = p.xm = 0;
+  }
+  p.total = off;
+  return p;
+}
+
+int check_weights(const h3b_block_weights* w, int dtype) {
+  if (!w) return H3B_ERR_NULL;
+  if (w->dtype != dtype) return H3B_ERR_DTYPE;
+  if (!w->w_qkv || !w->w_o || !w->w_fc1 || !w->w_fc2 || !w->g_attn || !w->g_mlp) return H3B_ERR_NULL;
+  if (!aligned16(w->w_qkv) || !aligned16(w->w_o) || !aligned16(w->w_fc1) || !aligned16(w->w_fc2) ||
+      !aligned16(w->g_attn) || !aligned16(w->g_mlp))
+    return H3B_ERR_ALIGN;
+  if (dtype == H3B_INT8) {
+    if (!w->s_qkv || !w->s_o || !w->s_fc1 || !w->s_fc2) return H3B_ERR_NULL;
+    if (!aligned16(w->s_qkv) || !aligned16(w->s_o) || !aligned16(w->s_fc1) || !aligned16(w->s_fc2))
+      return H3B_ERR_ALIGN;
+  }
+  return H3B_OK;
+}
+
+#define H3B_TRY(expr)                 \
+  do {                                \
+    const int _st = (expr);           \
+    if (_st != H3B_OK) return _st;    \
+  } while (0)
+#define H3B_CU(kid, expr)                                    \
+  do {                                                       \
+    TraceScope _ts((kid), c.stream);                         \
+    if ((expr) != cudaSuccess) return H3B_ERR_CUDA;          \
+  } while (0)
+
+GemmArgs gemm_args(int M, int N, int K, void* C, const float* sa, const float* sb, const float* rope,
+                   const h3b_dims& dm, float* amax, int* err) {
+  GemmArgs a;
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.C = C;
+  a.sa = sa;
+  a.sb = sb;
+  a.rope = reinterpret_cast<const float2*>(rope);
+  a.d = dm.d;
+  a.head_dim = dm.head_dim;
+  a.row_absmax = amax;
+  a.err = err;
+  return a;
+}
+
+// One block on x [S_eff, d]; rope = table of this geometry (already filled).
+int block_impl(const Ctx& c, const h3b_dims& dm, const h3b_block_weights& w, float* x, int merged, uint8_t* ws,
+               const Plan& p, const float* rope) {
+  const int S = seq_len(dm, merged), d = dm.d, f = dm.ffn;
+  uint8_t* A = ws;
+  void* qkv = A + p.qkv;
+  void* o = A + p.o;
+  void* u1 = A + p.u1;
+  void* u2 = A + p.u2;
+  void* g = A + p.g;
+  float* s_act = reinterpret_cast<float*>(ws + p.s_act);
+  if (w.dtype == H3B_BF16) {
+    H3B_CU(KID_RMSNORM, launch_rmsnorm(c, x, w.g_attn, S, d, dm.eps, u1, nullptr, 0));
+    H3B_CU(KID_GEMM_QKV, launch_gemm(c, u1, w.w_qkv, 0, H3B_EPI_QKV_ROPE,
+                                     gemm_args(S, 3 * d, d, qkv, nullptr, nullptr, rope, dm, nullptr, c.err)));
+    H3B_CU(KID_ATTN, launch_attention(c, qkv, S, dm.n_heads, dm.head_dim, o));
+    H3B_CU(KID_GEMM_O, launch_gemm(c, o, w.w_o, 0, H3B_EPI_RESID,
+                                   gemm_args(S, d, d, x, nullptr, nullptr, nullptr, dm, nullptr, c.err)));
+    H3B_CU(KID_RMSNORM, launch_rmsnorm(c, x, w.g_mlp, S, d, dm.eps, u2, nullptr, 0));
+    H3B_CU(KID_GEMM_FC1, launch_gemm(c, u2, w.w_fc1, 0, H3B_EPI_GELU,
+                                     gemm_args(S, f, d, g, nullptr, nullptr, nullptr, dm, nullptr, c.err)));
+    H3B_CU(KID_GEMM_FC2, launch_gemm(c, g, w.w_fc2, 0, H3B_EPI_RESID,
+                                     gemm_args(S, d, f, x, nullptr, nullptr, nullptr, dm, nullptr, c.err)));
+  } else {
+    int8_t* oq = reinterpret_cast<int8_t*>(A + p.oq);
+    int8_t* gq = reinterpret_cast<int8_t*>(A + p.gq);
+    float* s_g = reinterpret_cast<float*>(ws + p.s_g);
+    float* amax = reinterpret_cast<float*>(ws + p.amax);
+    H3B_CU(KID_RMSNORM, launch_rmsnorm(c, x, w.g_attn, S, d, dm.eps, u1, s_act, 1));
+    H3B_CU(KID_GEMM_QKV, launch_gemm(c, u1, w.w_qkv, 1, H3B_EPI_QKV_ROPE,
+                                     gemm_args(S, 3 * d, d, qkv, s_act, w.s_qkv, rope, dm, nullptr, c.err)));
+    H3B_CU(KID_ATTN, launch_attention(c, qkv, S, dm.n_heads, dm.head_dim, o));
+    H3B_CU(KID_QUANT_ROWS, launch_quant_rows(c, o, S, d, oq, s_act));
+    H3B_CU(KID_GEMM_O, launch_gemm(c, oq, w.w_o, 1, H3B_EPI_RESID,
+                                   gemm_args(S, d, d, x, s_act, w.s_o, nullptr, dm, nullptr, c.err)));
+    H3B_CU(KID_RMSNORM, launch_rmsnorm(c, x, w.g_mlp, S, d, dm.eps, u2, s_act, 1));
+    H3B_CU(KID_MEMSET, cudaMemsetAsync(amax, 0, sizeof(float) * S, c.stream));
+    H3B_CU(KID_GEMM_FC1, launch_gemm(c, u2, w.w_fc1, 1, H3B_EPI_GELU,
+                                     gemm_args(S, f, d, g, s_act, w.s_fc1, nullptr, dm, amax, c.err)));
+    H3B_CU(KID_QUANT_ABSMAX, launch_quant_absmax(c, g, amax, S, f, gq, s_g));
+    H3B_CU(KID_GEMM_FC2, launch_gemm(c, gq, w.w_fc2, 1, H3B_EPI_RESID,
+                                     gemm_args(S, d, f, x, s_g, w.s_fc2, nullptr, dm, nullptr, c.err)));
+  }
+  return H3B_OK;
+}
+
+int stack_impl(const Ctx& c, const h3b_dims& dm, const h3b_block_weights* blocks, int n_blocks, int mf, int ml,
+               float* x, uint8_t* ws, const Plan& p) {
+  const int on = mf >= 0;
+  float* rope = reinterpret_cast<float*>(ws + p.rope);
+  float* rope_m = on ? reinterpret_cast<float*>(ws + p.rope_m) : nullptr;
+  float* xm = on ? reinterpret_cast<float*>(ws + p.xm) : nullptr;
+  H3B_CU(KID_ROPE_TABLE, launch_rope_table(c, dm, 0, rope));
+  if (on) H3B_CU(KID_ROPE_TABLE, launch_rope_table(c, dm, 1, rope_m));
+  const int V = dm.frames * dm.rows * dm.cols;
+  for (int l = 0; l < n_blocks; ++l) {
+    if (on && l == mf) H3B_CU(KID_MERGE, launch_merge(c, x, xm, V, dm.n_audio, dm.d));
+    const bool merged = on && l >= mf && l <= ml;
+    H3B_TRY(block_impl(c, dm, blocks[l], merged ? xm : x, merged, ws, p, merged ? rope_m : rope));
+    if (on && l == ml) H3B_CU(KID_UNMERGE, launch_unmerge(c, xm, x, V, dm.n_audio, dm.d));
+  }
+  return H3B_OK;
+}
+
+int check_stack_args(const h3b_dims* dims, const h3b_block_weights* blocks, int n_blocks, int mf, int ml, float* x,
+                     void* ws, size_t ws_bytes, Plan* out) {
+  H3B_TRY(check_dims(dims));
+  if (!blocks || !x || !ws) return H3B_ERR_NULL;
+  if (!aligned16(x) || !aligned16(ws)) return H3B_ERR_ALIGN;
+  if (n_blocks < 0) return H3B_ERR_DIMS;
+  if (mf >= 0) {
+    if (ml < mf || ml >= n_blocks || (dims->cols & 1)) return H3B_ERR_DIMS;
+  }
+  const int dtype = n_blocks > 0 ? blocks[0].dtype : H3B_BF16;
+  if (dtype != H3B_BF16 && dtype != H3B_INT8) return H3B_ERR_DTYPE;
+  for (int l = 0; l < n_blocks; ++l) H3B_TRY(check_weights(&blocks[l], dtype));
+  *out = plan(*dims, dtype, mf >= 0);
+  if (ws_bytes < out->total) return H3B_ERR_WORKSPACE;
+  return H3B_OK;
+}
+
+}  // namespace
+
+// ------------------------------------------------------------------ tensor maps
+bool encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, int elem_bytes, const void* base, uint64_t inner,
+                    uint64_t outer, uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer) {
+  typedef CUresult (*EncodeFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                               const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                               CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+  static EncodeFn fn = nullptr;
+  if (!fn) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!fn) {
+      void* p = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+          q != cudaDriverEntryPointSuccess || !p)
+        return false;
+      fn = reinterpret_cast<EncodeFn>(p);
+    }
+  }
+  (void)elem_bytes;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_stride_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace h3b
+
+using namespace h3b;
+
+// ====================================================================== C ABI
+extern "C" {
+
+const char* h3b_status_string(int s) {
+  switch (s) {
+    case H3B_OK: return "ok";
+    case H3B_ERR_NULL: return "a required pointer is NULL";
+    case H3B_ERR_ALIGN: return "a pointer is not 16-byte aligned";
+    case H3B_ERR_DIMS: return "unsupported or inconsistent sizes";
+    case H3B_ERR_DTYPE: return "unknown dtype or epilogue";
+    case H3B_ERR_WORKSPACE: return "workspace smaller than required";
+    case H3B_ERR_CUDA: return "a CUDA call failed";
+    case H3B_ERR_DEVICE: return "no usable sm_100 device";
+    case H3B_ERR_TIMEOUT: return "a bounded device-side wait gave up";
+    default: return "unknown status";
+  }
+}
+
+int h3b_seq_len(const h3b_dims* dims, int merged) {
+  if (check_dims(dims) != H3B_OK) return -1;
+  if (merged && (dims->cols & 1)) return -1;
+  return seq_len(*dims, merged);
+}
+
+size_t h3b_workspace_bytes(const h3b_dims* dims, int dtype, int token_reduction) {
+  if (check_dims(dims) != H3B_OK || (dtype != H3B_BF16 && dtype != H3B_INT8)) return 0;
+  if (token_reduction && (dims->cols & 1)) return 0;
+  return plan(*dims, dtype, token_reduction != 0).total;
+}
+
+size_t h3b_workspace_saved_bytes(const h3b_dims* dims, int dtype) {
+  if (check_dims(dims) != H3B_OK || (dtype != H3B_BF16 && dtype != H3B_INT8)) return 0;
+  const Plan p = plan(*dims, dtype, 0);
+  return p.naive - p.arena;
+}
+
+int h3b_block_forward(const h3b_dims* dims, const h3b_block_weights* w, float* x, int merged, void* ws,
+                      size_t ws_bytes, void* stream) {
+  H3B_TRY(check_dims(dims));
+  if (!w || !x || !ws) return H3B_ERR_NULL;
+  if (!aligned16(x) || !aligned16(ws)) return H3B_ERR_ALIGN;
+  if (merged && (dims->cols & 1)) return H3B_ERR_DIMS;
+  if (w->dtype != H3B_BF16 && w->dtype != H3B_INT8) return H3B_ERR_DTYPE;
+  H3B_TRY(check_weights(w, w->dtype));
+  const Plan p = plan(*dims, w->dtype, 0);
+  if (ws_bytes < p.total) return H3B_ERR_WORKSPACE;
+  Ctx c;
+  H3B_TRY(device_ctx(static_cast<cudaStream_t>(stream), &c));
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  float* rope = reinterpret_cast<float*>(wsb + p.rope);
+  H3B_CU(KID_ROPE_TABLE, launch_rope_table(c, *dims, merged, rope));
+  return block_impl(c, *dims, *w, x, merged, wsb, p, rope);
+}
+
+int h3b_stack_forward(const h3b_dims* dims, const h3b_block_weights* blocks, int n_blocks, int merge_first,
+                      int merge_last, float* x, void* ws, size_t ws_bytes, void* stream) {
+  Plan p;
+  H3B_TRY(check_stack_args(dims, blocks, n_blocks, merge_first, merge_last, x, ws, ws_bytes, &p));
+  Ctx c;
+  H3B_TRY(device_ctx(static_cast<cudaStream_t>(stream), &c));
+  return stack_impl(c, *dims, blocks, n_blocks, merge_first, merge_last, x, static_cast<uint8_t*>(ws), p);
+}
+
+int h3b_denoise(const h3b_dims* dims, const h3b_block_weights* blocks, int n_blocks, int merge_first,
+                int merge_last, int n_steps, int reuse, float* x, float* v, void* ws, size_t ws_bytes, int* n_fresh,
+                void* stream) {
+  Plan p;
+  H3B_TRY(check_stack_args(dims, blocks, n_blocks, merge_first, merge_last, x, ws, ws_bytes, &p));
+  if (!v) return H3B_ERR_NULL;
+  if (!aligned16(v)) return H3B_ERR_ALIGN;
+  if (n_steps <= 0 || reuse <= 0) return H3B_ERR_DIMS;
+  Ctx c;
+  H3B_TRY(device_ctx(static_cast<cudaStream_t>(stream), &c));
+  const size_t n = static_cast<size_t>(seq_len(*dims, 0)) * dims->d;
+  auto fresh = [&](int i) { return i % reuse == 0 || i == n_steps - 1; };
+  int count = 0;
+  H3B_CU(KID_MEMSET, cudaMemcpyAsync(v, x, n * sizeof(float), cudaMemcpyDeviceToDevice, c.stream));
+  for (int i = 0; i < n_steps; ++i) {
+    if (fresh(i)) {
+      H3B_TRY(stack_impl(c, *dims, blocks, n_blocks, merge_first, merge_last, v, static_cast<uint8_t*>(ws), p));
+      ++count;
+    }
+    const float s0 = static_cast<float>(1.0 - static_cast<double>(i) / n_steps);
+    const float s1 = static_cast<float>(1.0 - static_cast<double>(i + 1) / n_steps);
+    const bool next_fresh = i + 1 < n_steps && fresh(i + 1);
+    H3B_CU(KID_FLOW, launch_flow_step(c, x, v, s1 - s0, n, next_fresh ? v : nullptr));
+  }
+  if (n_fresh) *n_fresh = count;
+  return H3B_OK;
+}
+
+int h3b_quantize_weights(const void* w, int rows, int k, int8_t* q, float* scale, void* stream) {
+  if (!w || !q || !scale) return H3B_ERR_NULL;
+  if (!aligned16(w) || !aligned16(q) || !aligned16(scale)) return H3B_ERR_ALIGN;
+  if (rows < 0 || k <= 0 || k % 8 != 0 || k > 32768) return H3B_ERR_DIMS;
+  Ctx c;
+  H3B_TRY(device_ctx(static_cast<cudaStream_t>(stream), &c));
+  H3B_CU(KID_QUANT_ROWS, launch_quant_rows(c, w, rows, k, q, scale));
+  return H3B_OK;
+}
+
+int h3b_quantize_rows_absmax(const void* a, const float* absmax, int rows, int k, int8_t* q, float* scale,
+                             void* stream) {
+  if (!a || !absmax || !q || !scale) return H3B_ERR_NULL;
+  if (!aligned16(a) || !aligned16(q) || !aligned16(scale) || !aligned16(absmax)) return H3B_ERR_ALIGN;
+  if (rows < 0 || k <= 0 || k % 8 != 0) return H3B_ERR_DIMS;
+  Ctx c;
+  H3B_TRY(device_ctx(static_cast<cudaStream_t>(stream), &c));
+  H3B_CU(KID_QUANT_ABSMAX, launch_quant_absmax(c, a, absmax, rows, k, q, scale));
+  return H3B_OK;
+}
+
+int h3b_token_merge(const h3b_dims* dims, const float* x, float* xm, void* stream) {
+  H3B_TRY(check_dims(dims));
+  if (!x || !xm) return H3B_ERR_NULL;
+  if (!aligned16(x) || !aligned16(xm)) return H3B_ERR_ALIGN;
+  if (dims->cols & 1) return H3B_ERR_DIMS;
+  Ctx c;
+  H3B_TRY(device_ctx(static_cast<cudaStream_t>(stream), &c));
+  H3B_CU(KID_MERGE, launch_merge(c, x, xm, dims->frames * dims->rows * dims->cols, dims->n_audio, dims->d));
+  return H3B_OK;
+}
+
+int h3b_token_unmerge(const h3b_dims* dims, const float* xm, float* x, void* stream) {
+  H3B_TRY(check_dims(dims));
+  if (!x || !xm) return H3B_ERR_NULL;
+  if (!aligned16(x) || !aligned16(xm)) return H3B_ERR_ALIGN;
+  if (dims->cols & 1) return H3B_ERR_DIMS;
+  Ctx c;
+  H3B_TRY(device_ctx(static_cast<cudaStream_t>(stream), &c));
+  H3B_CU(KID_UNMERGE, launch_unmerge(c, xm, x, dims->frames * dims->rows * dims->cols, dims->n_audio, dims->d));
+  return H3B_OK;
+}
+
+int h3b_flow_step(float* x, const float* v, float sigma_cur, float sigma_next, size_t n, float* x_copy,
+                  void* stream) {
+  if (n == 0) return H3B_OK;  // nothing to update; empty buffers may be NULL
+  if (!x || !v) return H3B_ERR_NULL;
+  if (!aligned16(x) || !aligned16(v) || (x_copy && !aligned16(x_copy))) return H3B_ERR_ALIGN;
+  Ctx c;
+  H3B_TRY(device_ctx(static_cast<cudaStream_t>(stream), &c));
+  H3B_CU(KID_FLOW, launch_flow_step(c, x, v, sigma_next - sigma_cur, n, x_copy));
+  return H3B_OK;
+}
+
+int h3b_rope_table(const h3b_dims* dims, int merged, float* table, void* stream) {
+  H3B_TRY(check_dims(dims));
+  if (!table) return H3B_ERR_NULL;
+  if (!aligned16(table)) return H3B_ERR_ALIGN;
+  if (merged && (dims->cols & 1)) return H3B_ERR_DIMS;
+  Ctx c;
+  H3B_TRY(device_ctx(static_cast<cudaStream_t>(stream), &c));
+  H3B_CU(KID_ROPE_TABLE, launch_rope_table(c, *dims, merged, table));
+  return H3B_OK;
+}
+
+int h3b_rmsnorm(const float* x, const float* g, int rows, int d, float eps, void* out, float* out_scale,
+                int out_dtype, void* stream) {
+  if (!x || !g || !out || (out_dtype == H3B_INT8 && !out_scale)) return H3B_ERR_NULL;
+  if (!aligned16(x) || !aligned16(g) || !aligned16(out)) return H3B_ERR_ALIGN;
+  if (out_dtype != H3B_BF16 && out_dtype != H3B_INT8) return H3B_ERR_DTYPE;
+  if (rows < 0 || d <= 0 || d % 4 != 0 || d > 8192 || !(eps >= 0.f)) return H3B_ERR_DIMS;
+  Ctx c;
+  H3B_TRY(device_ctx(static_cast<cudaStream_t>(stream), &c));
+  H3B_CU(KID_RMSNORM, launch_rmsnorm(c, x, g, rows, d, eps, out, out_scale, out_dtype == H3B_INT8));
+  return H3B_OK;
+}
+
+int h3b_gemm(const void* A, const void* B, int M, int N, int K, int ab_dtype, int epilogue, void* C,
+             const float* scale_a, const float* scale_b, const float* rope_table, const h3b_dims* dims,
+             float* row_absmax, void* stream) {
+  if (!A || !B || !C) return H3B_ERR_NULL;
+  if (!aligned16(A) || !aligned16(B) || !aligned16(C)) return H3B_ERR_ALIGN;
+  if (ab_dtype != H3B_BF16 && ab_dtype != H3B_INT8) return H3B_ERR_DTYPE;
+  if (epilogue < H3B_EPI_F32 || epilogue > H3B_EPI_I32) return H3B_ERR_DTYPE;
+  if (epilogue == H3B_EPI_I32 && ab_dtype != H3B_INT8) return H3B_ERR_DTYPE;
+  if (M < 0 || N <= 0 || K <= 0 || N % 32 != 0 || K % (ab_dtype == H3B_INT8 ? 128 : 64) != 0) return H3B_ERR_DIMS;
+  if (ab_dtype == H3B_INT8 && epilogue != H3B_EPI_I32) {
+    if (!scale_a || !scale_b) return H3B_ERR_NULL;
+    if (!aligned16(scale_b)) return H3B_ERR_ALIGN;
+  }
+  h3b_dims dm{};
+  if (epilogue == H3B_EPI_QKV_ROPE) {
+    H3B_TRY(check_dims(dims));
+    if (!rope_table) return H3B_ERR_NULL;
+    if (!aligned16(rope_table)) return H3B_ERR_ALIGN;
+    if (N != 3 * dims->d) return H3B_ERR_DIMS;
+    dm = *dims;
+  }
+  if (epilogue == H3B_EPI_GELU && ab_dtype == H3B_INT8 && !row_absmax) return H3B_ERR_NULL;
+  Ctx c;
+  H3B_TRY(device_ctx(static_cast<cudaStream_t>(stream), &c));
+  H3B_CU(KID_GEMM, launch_gemm(c, A, B, ab_dtype == H3B_INT8, epilogue,
+                               gemm_args(M, N, K, C, scale_a, scale_b, rope_table, dm, row_absmax, c.err)));
+  return H3B_OK;
+}
+
+int h3b_attention(const void* qkv, int S, int n_heads, int head_dim, void* o, void* stream) {
+  if (!qkv || !o) return H3B_ERR_NULL;
+  if (!aligned16(qkv) || !aligned16(o)) return H3B_ERR_ALIGN;
+  if (S < 0 || n_heads <= 0 || (head_dim != 64 && head_dim != 128)) return H3B_ERR_DIMS;
+  Ctx c;
+  H3B_TRY(device_ctx(static_cast<cudaStream_t>(stream), &c));
+  H3B_CU(KID_ATTN, launch_attention(c, qkv, S, n_heads, head_dim, o));
+  return H3B_OK;
+}
+
+int h3b_device_error(void* stream) {
+  Ctx c;
+  H3B_TRY(device_ctx(static_cast<cudaStream_t>(stream), &c));
+  int v = 0;
+  if (cudaMemcpyAsync(&v, c.err, sizeof(int), cudaMemcpyDeviceToHost, c.stream) != cudaSuccess) return H3B_ERR_CUDA;
+  if (cudaStreamSynchronize(c.stream) != cudaSuccess) return H3B_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyAsync(c.err, &zero, sizeof(int), cudaMemcpyHostToDevice, c.stream) != cudaSuccess ||
+        cudaStreamSynchronize(c.stream) != cudaSuccess)
+      return H3B_ERR_CUDA;
+  }
+  return v;
+}
+
+int h3b_trace_start(int capacity) {
+  if (capacity < 0) return H3B_ERR_DIMS;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (static_cast<int>(g_trace.recs.size()) < capacity) {
+    const size_t old = g_trace.recs.size();
+    g_trace.recs.resize(capacity);
+    for (size_t i = old; i < g_trace.recs.size(); ++i) {
+      if (cudaEventCreate(&g_trace.recs[i].a) != cudaSuccess || cudaEventCreate(&g_trace.recs[i].b) != cudaSuccess) {
+        g_trace.recs.resize(i);
+        return H3B_ERR_CUDA;
+      }
+    }
+  }
+  g_trace.cap = capacity;
+  g_trace.n = 0;
+  g_trace.on = true;
+  return H3B_OK;
+}
+
+int h3b_trace_stop(int* n_records) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_trace.on = false;
+  g_trace.ms.assign(g_trace.n, 0.f);
+  for (int i = 0; i < g_trace.n; ++i) {
+    if (cudaEventSynchronize(g_trace.recs[i].b) != cudaSuccess) return H3B_ERR_CUDA;
+    if (cudaEventElapsedTime(&g_trace.ms[i], g_trace.recs[i].a, g_trace.recs[i].b) != cudaSuccess)
+      return H3B_ERR_CUDA;
+  }
+  if (n_records) *n_records = g_trace.n;
+  return H3B_OK;
+}
+
+int h3b_trace_read(int* kernel_ids, float* ms, int max_records) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  const int n = g_trace.n < max_records ? g_trace.n : max_records;
+  for (int i = 0; i < n && i < static_cast<int>(g_trace.ms.size()); ++i) {
+    if (kernel_ids) kernel_ids[i] = g_trace.recs[i].kid;
+    if (ms) ms[i] = g_trace.ms[i];
+  }
+  return n;
+}
+
+const char* h3b_kernel_name(int kid) { return (kid >= 0 && kid < KID_COUNT) ? kKernelNames[kid] : "unknown"; }
+
+}  // extern "C"

@@ -1,0 +1,320 @@
+// Tensor-core GEMM C = A B^T for the DiT block's four linear layers, on the
+// sm_100a tcgen05 path: TMA (128-byte swizzle) -> shared-memory ring ->
+// tcgen05.mma (bf16 -> fp32, or int8 -> int32) with the accumulator in TMEM ->
+// epilogue warps read TMEM and apply the fused epilogue.
+//
+// Structure (one CTA per SM, persistent over output tiles):
+//   warp 0      TMA producer (one elected thread): A tile [128 x 128 B] and
+//               B tile [256 x 128 B] per stage, 4 stages.
+//   warp 1      MMA issuer (one thread): 4 MMAs of 128x256xK16 (bf16) or
+//               128x256xK32 (int8) per stage; commits free the stage.
+//   warps 2..5  epilogue: warp w reads TMEM lanes 32*(w%4).. (one output row
+//               per thread), 32 columns at a time.
+// Two 256-column accumulators (all 512 TMEM columns) let the epilogue of
+// tile i overlap the MMAs of tile i+1.
+//
+// Epilogues fused into the store (h3b.h H3B_EPI_*): plain fp32 / bf16, QKV
+// with RoPE applied to the Q and K columns, fp32 residual add (x += acc),
+// GELU (+ per-row max |GELU| for the next int8 quantisation), raw int32.
+// INT8 inputs are dequantised as float(acc) * s_a[m] * s_w[n] first.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace h3b {
+
+namespace {
+
+constexpr int BM = 128, BN = 256, KBYTES = 128, STAGES = 4;
+constexpr int A_STAGE = BM * KBYTES;  // 16 KB
+constexpr int B_STAGE = BN * KBYTES;  // 32 KB
+constexpr int TMEM_COLS = 2 * BN;     // two fp32 / int32 accumulators
+constexpr int THREADS = 192;
+constexpr int NUM_BARS = 2 * STAGES + 5;
+constexpr int SMEM_BYTES = 1024 + STAGES * (A_STAGE + B_STAGE) + NUM_BARS * 8 + 16;
+constexpr int GROUP_N = 8;  // N tiles per raster group (L2 reuse of A rows)
+
+// Tile t -> (m block, n block): groups of GROUP_N n-blocks, m-major inside a
+// group, so the tiles in flight share a band of B and sweep A.
+__device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int& mb, int& nb) {
+  const int per_group = num_m * GROUP_N;
+  const int g = t / per_group;
+  const int first_n = g * GROUP_N;
+  const int gs = min(GROUP_N, num_n - first_n);
+  const int local = t - g * per_group;
+  mb = local / gs;
+  nb = first_n + local % gs;
+}
+
+template <bool INT8, int EPI>
+__device__ __forceinline__ void epilogue_chunk(const GemmArgs& p, int m, int n, const uint32_t (&r)[32],
+                                               float& row_amax) {
+  const size_t off = static_cast<size_t>(m) * p.N + n;
+  if (EPI == H3B_EPI_I32) {
+    int4* c = reinterpret_cast<int4*>(static_cast<int*>(p.C) + off);
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      c[i] = make_int4(static_cast<int>(r[4 * i]), static_cast<int>(r[4 * i + 1]), static_cast<int>(r[4 * i + 2]),
+                       static_cast<int>(r[4 * i + 3]));
+    return;
+  }
+  float v[32];
+  if (INT8) {
+    const float sa = p.sa[m];
+    const float4* sb4 = reinterpret_cast<const float4*>(p.sb + n);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float4 sb = __ldg(sb4 + i);
+      v[4 * i + 0] = static_cast<float>(static_cast<int>(r[4 * i + 0])) * sa * sb.x;
+      v[4 * i + 1] = static_cast<float>(static_cast<int>(r[4 * i + 1])) * sa * sb.y;
+      v[4 * i + 2] = static_cast<float>(static_cast<int>(r[4 * i + 2])) * sa * sb.z;
+      v[4 * i + 3] = static_cast<float>(static_cast<int>(r[4 * i + 3])) * sa * sb.w;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+  }
+
+  if (EPI == H3B_EPI_F32) {
+    float4* c = reinterpret_cast<float4*>(static_cast<float*>(p.C) + off);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) c[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+    return;
+  }
+  if (EPI == H3B_EPI_RESID) {
+    float4* c = reinterpret_cast<float4*>(static_cast<float*>(p.C) + off);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      float4 a = c[i];
+      a.x += v[4 * i];
+      a.y += v[4 * i + 1];
+      a.z += v[4 * i + 2];
+      a.w += v[4 * i + 3];
+      c[i] = a;
+    }
+    return;
+  }
+  if (EPI == H3B_EPI_QKV_ROPE) {
+    if (n < 2 * p.d) {  // Q or K column block: rotate its 16 interleaved pairs
+      const int j0 = (n % p.head_dim) >> 1;
+      const float4* t4 = reinterpret_cast<const float4*>(p.rope + static_cast<size_t>(m) * (p.head_dim >> 1) + j0);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float4 cs = __ldg(t4 + i);  // (cos, sin) of pairs 2i and 2i+1
+        const float a0 = v[4 * i], a1 = v[4 * i + 1], b0 = v[4 * i + 2], b1 = v[4 * i + 3];
+        v[4 * i] = a0 * cs.x - a1 * cs.y;
+        v[4 * i + 1] = a0 * cs.y + a1 * cs.x;
+        v[4 * i + 2] = b0 * cs.z - b1 * cs.w;
+        v[4 * i + 3] = b0 * cs.w + b1 * cs.z;
+      }
+    }
+  }
+  if (EPI == H3B_EPI_GELU) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = gelu_erf(v[i]);
+  }
+  // bf16 store (BF16, QKV_ROPE, GELU)
+  uint32_t w[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) w[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+  if (EPI == H3B_EPI_GELU && INT8) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const float lo = __uint_as_float(w[i] << 16), hi = __uint_as_float(w[i] & 0xffff0000u);
+      row_amax = fmaxf(row_amax, fmaxf(fabsf(lo), fabsf(hi)));
+    }
+  }
+  uint4* c = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.C) + off);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) c[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+}
+
+template <bool INT8, int EPI>
+__global__ void __launch_bounds__(THREADS, 1)
+    k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const GemmArgs p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * A_STAGE;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * B_STAGE);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NUM_BARS);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t bar0 = smem_u32(bars);
+  // barrier map: full[s], empty[s], tmem_full[2], tmem_empty[2], mma_done
+  const uint32_t full0 = bar0, empty0 = bar0 + 8 * STAGES, tfull0 = bar0 + 16 * STAGES,
+                 tempty0 = tfull0 + 16, mma_done = tempty0 + 16;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull0 + 8 * a, 1);
+      mbar_init(tempty0 + 8 * a, 4);  // one arrival per epilogue warp
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int num_m = (p.M + BM - 1) / BM, num_n = (p.N + BN - 1) / BN, num_tiles = num_m * num_n;
+  constexpr int KE = INT8 ? 128 : 64;  // K elements per stage
+  const int num_kb = p.K / KE;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0, issued = 0, issued_par = 0;
+      for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+        int mb, nb;
+        tile_coords(t, num_m, num_n, mb, nb);
+        bool ok = true;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(empty0 + 8 * stage, phase ^ 1, abort_flag, p.err, (EK_GEMM << 8) | 1)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = full0 + 8 * stage;
+          mbar_arrive_expect_tx(fb, A_STAGE + B_STAGE);
+          tma_load_2d(smem_u32(sA + stage * A_STAGE), &tmA, fb, kb * KE, mb * BM);
+          tma_load_2d(smem_u32(sB + stage * B_STAGE), &tmB, fb, kb * KE, nb * BN);
+          issued |= 1u << stage;
+          issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+      }
+      // every copy this thread issued lands before the CTA may exit
+      for (int s = 0; s < STAGES; ++s)
+        if ((issued >> s) & 1) mbar_drain(full0 + 8 * s, (issued_par >> s) & 1);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = INT8 ? idesc_i8(BM, BN) : idesc_bf16(BM, BN, false);
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+        if (!mbar_wait(tempty0 + 8 * acc, acc_phase ^ 1, abort_flag, p.err, (EK_GEMM << 8) | 2)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        bool ok = true;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(full0 + 8 * stage, phase, abort_flag, p.err, (EK_GEMM << 8) | 3)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + stage * A_STAGE), b0 = smem_u32(sB + stage * B_STAGE);
+#pragma unroll
+          for (int k = 0; k < KBYTES / 32; ++k) {
+            const uint64_t ad = desc_sw128_k(a0 + 32 * k), bd = desc_sw128_k(b0 + 32 * k);
+            if (INT8)
+              mma_i8_ss(d_tmem, ad, bd, idesc, (kb | k) != 0);
+            else
+              mma_bf16_ss(d_tmem, ad, bd, idesc, (kb | k) != 0);
+          }
+          tc_commit(empty0 + 8 * stage);  // frees the stage once these MMAs have read it
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        tc_commit(tfull0 + 8 * acc);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1;
+      }
+      // all issued MMAs complete before TMEM can be released
+      tc_commit(mma_done);
+      mbar_drain(mma_done, 0);
+    }
+  } else {
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+      int mb, nb;
+      tile_coords(t, num_m, num_n, mb, nb);
+      const bool ok = mbar_wait(tfull0 + 8 * acc, acc_phase, abort_flag, p.err, (EK_GEMM << 8) | 4);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      const int m = mb * BM + q * 32 + lane;
+      float row_amax = 0.f;
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        const int n = nb * BN + c * 32;
+        if (n >= p.N) break;
+        uint32_t r[32];
+        tmem_ld32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN + c * 32, r);
+        tmem_ld_wait();
+        if (m < p.M) epilogue_chunk<INT8, EPI>(p, m, n, r, row_amax);
+      }
+      if (INT8 && EPI == H3B_EPI_GELU && m < p.M)
+        atomicMax(reinterpret_cast<int*>(p.row_absmax) + m, __float_as_int(row_amax));
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty0 + 8 * acc);
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1;
+    }
+  }
+
+  __syncthreads();
+  if (warp == 0) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+using GemmKernel = void (*)(const CUtensorMap, const CUtensorMap, const GemmArgs);
+
+template <bool INT8>
+GemmKernel pick(int epi) {
+  switch (epi) {
+    case H3B_EPI_F32: return k_gemm<INT8, H3B_EPI_F32>;
+    case H3B_EPI_BF16: return k_gemm<INT8, H3B_EPI_BF16>;
+    case H3B_EPI_QKV_ROPE: return k_gemm<INT8, H3B_EPI_QKV_ROPE>;
+    case H3B_EPI_RESID: return k_gemm<INT8, H3B_EPI_RESID>;
+    case H3B_EPI_GELU: return k_gemm<INT8, H3B_EPI_GELU>;
+    case H3B_EPI_I32: return INT8 ? k_gemm<INT8, H3B_EPI_I32> : nullptr;
+    default: return nullptr;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_gemm(const Ctx& c, const void* A, const void* B, int ab_int8, int epi, const GemmArgs& args) {
+  GemmKernel kern = ab_int8 ? pick<true>(epi) : pick<false>(epi);
+  if (!kern) return cudaErrorInvalidValue;
+  const int eb = ab_int8 ? 1 : 2;
+  const CUtensorMapDataType dt = ab_int8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  CUtensorMap ta, tb;
+  if (!encode_tmap_2d(&ta, dt, eb, A, args.K, args.M, static_cast<uint64_t>(args.K) * eb, KBYTES / eb, BM) ||
+      !encode_tmap_2d(&tb, dt, eb, B, args.K, args.N, static_cast<uint64_t>(args.K) * eb, KBYTES / eb, BN))
+    return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  const int tiles = ((args.M + BM - 1) / BM) * ((args.N + BN - 1) / BN);
+  const int grid = tiles < c.num_sms ? tiles : c.num_sms;
+  if (grid == 0) return cudaSuccess;
+  kern<<<grid, THREADS, SMEM_BYTES, c.stream>>>(ta, tb, args);
+  return cudaGetLastError();
+}
+
+}  // namespace h3b

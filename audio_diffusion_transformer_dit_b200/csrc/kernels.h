@@ -1,0 +1,69 @@
+// Internal launcher declarations shared by the h3b translation units.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "h3b.h"
+
+namespace h3b {
+
+// kernel ids for tracing (names in h3b_kernel_name)
+enum KernelId {
+  KID_FLOW = 0,
+  KID_MERGE,
+  KID_UNMERGE,
+  KID_ROPE_TABLE,
+  KID_RMSNORM,
+  KID_QUANT_ROWS,
+  KID_QUANT_ABSMAX,
+  KID_GEMM_QKV,
+  KID_GEMM_O,
+  KID_GEMM_FC1,
+  KID_GEMM_FC2,
+  KID_GEMM,
+  KID_ATTN,
+  KID_MEMSET,
+  KID_COUNT
+};
+
+struct Ctx {
+  cudaStream_t stream;
+  int* err;
+  int num_sms;
+};
+
+// returns cudaError_t of the launch
+cudaError_t launch_flow_step(const Ctx& c, float* x, const float* v, float dt, size_t n, float* x_copy);
+cudaError_t launch_merge(const Ctx& c, const float* x, float* xm, int n_video, int n_audio, int d);
+cudaError_t launch_unmerge(const Ctx& c, const float* xm, float* x, int n_video, int n_audio, int d);
+cudaError_t launch_rope_table(const Ctx& c, const h3b_dims& dm, int merged, float* table);
+cudaError_t launch_rmsnorm(const Ctx& c, const float* x, const float* g, int rows, int d, float eps, void* out,
+                           float* out_scale, int out_int8);
+cudaError_t launch_quant_rows(const Ctx& c, const void* a, int rows, int k, int8_t* q, float* s);
+cudaError_t launch_quant_absmax(const Ctx& c, const void* a, const float* absmax, int rows, int k, int8_t* q,
+                                float* s);
+
+struct GemmArgs {
+  int M, N, K;
+  void* C;
+  const float* sa;
+  const float* sb;
+  const float2* rope;
+  int d, head_dim;
+  float* row_absmax;
+  int* err;
+};
+
+// A [M,K], B [N,K] K-major (bf16 or int8); C per epilogue.
+cudaError_t launch_gemm(const Ctx& c, const void* A, const void* B, int ab_int8, int epi, const GemmArgs& args);
+
+cudaError_t launch_attention(const Ctx& c, const void* qkv, int S, int n_heads, int head_dim, void* o);
+
+// tensor-map encoding through the driver entry point (no libcuda link)
+bool encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, int elem_bytes, const void* base, uint64_t inner,
+                    uint64_t outer, uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer);
+
+}  // namespace h3b

@@ -1,0 +1,363 @@
+// Memory-bound kernels of the DiT block path: flow-matching Euler update,
+// token merge / unmerge, RoPE table, RMSNorm (to bf16, or fused with per-token
+// int8 quantisation) and per-row int8 quantisation.
+//
+// All of them stream HBM with 16-byte vector accesses, consecutive threads on
+// consecutive 16-byte words, and grids sized in multiples of the SM count.
+#include <math.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace h3b {
+
+namespace {
+
+constexpr int kThreads = 256;
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// Block-wide reduction (sum or max) for up to 32 warps; all threads get the result.
+template <bool MAX>
+__device__ __forceinline__ float block_reduce(float v, float* red) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = (blockDim.x + 31) >> 5;
+  v = MAX ? warp_max(v) : warp_sum(v);
+  __syncthreads();  // protect `red` from the previous use
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  float r = lane < nw ? red[lane] : (MAX ? 0.f : 0.f);
+  r = MAX ? warp_max(r) : warp_sum(r);
+  return r;
+}
+
+__device__ __forceinline__ int8_t quant1(float v, float s) {
+  float q = s > 0.f ? rintf(v / s) : 0.f;  // IEEE divide, round half to even
+  q = fminf(fmaxf(q, -127.f), 127.f);
+  return static_cast<int8_t>(static_cast<int>(q));
+}
+
+// ------------------------------------------------------------------ Euler step
+__global__ void k_flow(float* __restrict__ x, const float* __restrict__ v, float dt, size_t n,
+                       float* __restrict__ xc) {
+  const size_t n4 = n >> 2;
+  const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
+  float4* x4 = reinterpret_cast<float4*>(x);
+  const float4* v4 = reinterpret_cast<const float4*>(v);
+  float4* c4 = reinterpret_cast<float4*>(xc);
+  for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4; i += stride) {
+    float4 a = x4[i];
+    const float4 b = __ldcs(v4 + i);
+    a.x = fmaf(dt, b.x, a.x);
+    a.y = fmaf(dt, b.y, a.y);
+    a.z = fmaf(dt, b.z, a.z);
+    a.w = fmaf(dt, b.w, a.w);
+    x4[i] = a;
+    if (xc) c4[i] = a;
+  }
+  for (size_t i = (n4 << 2) + static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += stride) {
+    const float a = fmaf(dt, v[i], x[i]);
+    x[i] = a;
+    if (xc) xc[i] = a;
+  }
+}
+
+// ------------------------------------------------------------------ token reduction
+// Video token (f, r, 2c'+k) is row 2*((f*H + r)*(W/2) + c') + k of the full
+// sequence, so merged row i averages full rows 2i and 2i+1; audio rows follow.
+__global__ void k_merge(const float4* __restrict__ x, float4* __restrict__ xm, int half_video, int n_audio, int d4) {
+  const size_t total = static_cast<size_t>(half_video + n_audio) * d4;
+  const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
+  for (size_t e = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < total; e += stride) {
+    const size_t row = e / d4, col = e - row * d4;
+    float4 o;
+    if (row < static_cast<size_t>(half_video)) {
+      const float4 a = __ldcs(x + (2 * row) * d4 + col);
+      const float4 b = __ldcs(x + (2 * row + 1) * d4 + col);
+      o.x = __fmul_rn(__fadd_rn(a.x, b.x), 0.5f);
+      o.y = __fmul_rn(__fadd_rn(a.y, b.y), 0.5f);
+      o.z = __fmul_rn(__fadd_rn(a.z, b.z), 0.5f);
+      o.w = __fmul_rn(__fadd_rn(a.w, b.w), 0.5f);
+    } else {
+      o = __ldcs(x + (row + half_video) * d4 + col);  // audio: full row = V + a = merged row + V/2
+    }
+    xm[e] = o;
+  }
+}
+
+__global__ void k_unmerge(const float4* __restrict__ xm, float4* __restrict__ x, int n_video, int n_audio, int d4) {
+  const size_t total = static_cast<size_t>(n_video + n_audio) * d4;
+  const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
+  const int half = n_video / 2;
+  for (size_t e = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < total; e += stride) {
+    const size_t row = e / d4, col = e - row * d4;
+    const size_t src = row < static_cast<size_t>(n_video) ? row / 2 : row - half;
+    x[e] = xm[src * d4 + col];
+  }
+}
+
+// ------------------------------------------------------------------ RoPE table
+// table[s][j] = (cos, sin) of pos * theta^(-2 jl / n) for pair j of token s,
+// jl the pair's index inside its section of width n (fp64 angle, fp32 store).
+__global__ void k_rope_table(float2* __restrict__ table, int F, int H, int Wc, int A, int D, float theta,
+                             int merged) {
+  const int half = D / 2;
+  const int n_video = F * H * Wc;
+  const size_t total = static_cast<size_t>(n_video + A) * half;
+  const int nf = D / 4, nr = 3 * D / 8, nc = D - nf - nr;
+  for (size_t e = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < total;
+       e += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const int s = static_cast<int>(e / half), j = static_cast<int>(e % half);
+    double pos;
+    int jl, n;
+    if (s < n_video) {
+      const int f = s / (H * Wc), rem = s % (H * Wc), r = rem / Wc, c = rem % Wc;
+      if (j < nf / 2) {
+        pos = f; jl = j; n = nf;
+      } else if (j < (nf + nr) / 2) {
+        pos = r; jl = j - nf / 2; n = nr;
+      } else {
+        pos = merged ? 2.0 * c + 0.5 : static_cast<double>(c); jl = j - (nf + nr) / 2; n = nc;
+      }
+    } else {
+      pos = s - n_video; jl = j; n = D;
+    }
+    const double ang = pos * pow(static_cast<double>(theta), -2.0 * jl / n);
+    double sn, cs;
+    sincos(ang, &sn, &cs);
+    table[e] = make_float2(static_cast<float>(cs), static_cast<float>(sn));
+  }
+}
+
+// ------------------------------------------------------------------ RMSNorm (+ quant)
+// One CTA per token row; the row stays in registers between the statistics and
+// the output pass (x is read from HBM exactly once).
+template <int VPT, bool INT8>
+__global__ void __launch_bounds__(kThreads) k_rmsnorm(const float* __restrict__ x, const float* __restrict__ g, int d,
+                                                      float eps, void* __restrict__ out, float* __restrict__ out_scale) {
+  __shared__ float red[32];
+  const int row = blockIdx.x, d4 = d >> 2;
+  const float4* xr = reinterpret_cast<const float4*>(x + static_cast<size_t>(row) * d);
+  const float4* g4 = reinterpret_cast<const float4*>(g);
+  float4 v[VPT];
+  float ss = 0.f;
+#pragma unroll
+  for (int i = 0; i < VPT; ++i) {
+    const int c = threadIdx.x + i * blockDim.x;
+    if (c < d4) {
+      v[i] = xr[c];
+      ss += v[i].x * v[i].x + v[i].y * v[i].y + v[i].z * v[i].z + v[i].w * v[i].w;
+    } else {
+      v[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  }
+  ss = block_reduce<false>(ss, red);
+  const float r = 1.0f / sqrtf(ss / static_cast<float>(d) + eps);
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < VPT; ++i) {
+    const int c = threadIdx.x + i * blockDim.x;
+    if (c < d4) {
+      const float4 gg = g4[c];
+      v[i].x = v[i].x * r * gg.x;
+      v[i].y = v[i].y * r * gg.y;
+      v[i].z = v[i].z * r * gg.z;
+      v[i].w = v[i].w * r * gg.w;
+      if (INT8) amax = fmaxf(amax, fmaxf(fmaxf(fabsf(v[i].x), fabsf(v[i].y)), fmaxf(fabsf(v[i].z), fabsf(v[i].w))));
+      else {
+        uint2 p;
+        p.x = pack_bf16x2(v[i].x, v[i].y);
+        p.y = pack_bf16x2(v[i].z, v[i].w);
+        reinterpret_cast<uint2*>(out)[static_cast<size_t>(row) * d4 + c] = p;
+      }
+    }
+  }
+  if (INT8) {
+    amax = block_reduce<true>(amax, red);
+    const float s = amax / 127.0f;
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+      const int c = threadIdx.x + i * blockDim.x;
+      if (c < d4) {
+        char4 q;
+        q.x = quant1(v[i].x, s);
+        q.y = quant1(v[i].y, s);
+        q.z = quant1(v[i].z, s);
+        q.w = quant1(v[i].w, s);
+        reinterpret_cast<char4*>(out)[static_cast<size_t>(row) * d4 + c] = q;
+      }
+    }
+    if (threadIdx.x == 0) out_scale[row] = s;
+  }
+}
+
+// ------------------------------------------------------------------ row quantisation
+__device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float (&f)[8]) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
+}
+
+__device__ __forceinline__ uint2 quant8(const float (&f)[8], float s) {
+  uint32_t lo = 0, hi = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    lo |= (static_cast<uint32_t>(static_cast<uint8_t>(quant1(f[i], s)))) << (8 * i);
+    hi |= (static_cast<uint32_t>(static_cast<uint8_t>(quant1(f[4 + i], s)))) << (8 * i);
+  }
+  return make_uint2(lo, hi);
+}
+
+// One CTA per row: max |row| then codes, row held in registers.
+template <int VPT>
+__global__ void __launch_bounds__(kThreads) k_quant_rows(const uint4* __restrict__ a, int k8, int8_t* __restrict__ q,
+                                                         float* __restrict__ scale) {
+  __shared__ float red[32];
+  const int row = blockIdx.x;
+  const uint4* ar = a + static_cast<size_t>(row) * k8;
+  uint4 v[VPT];
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < VPT; ++i) {
+    const int c = threadIdx.x + i * blockDim.x;
+    v[i] = c < k8 ? ar[c] : make_uint4(0, 0, 0, 0);
+    float f[8];
+    bf16x8_to_f32(v[i], f);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(f[j]));
+  }
+  amax = block_reduce<true>(amax, red);
+  const float s = amax / 127.0f;
+  uint2* qr = reinterpret_cast<uint2*>(q + static_cast<size_t>(row) * k8 * 8);
+#pragma unroll
+  for (int i = 0; i < VPT; ++i) {
+    const int c = threadIdx.x + i * blockDim.x;
+    if (c < k8) {
+      float f[8];
+      bf16x8_to_f32(v[i], f);
+      qr[c] = quant8(f, s);
+    }
+  }
+  if (threadIdx.x == 0) scale[row] = s;
+}
+
+// Known row maxima: purely elementwise.
+__global__ void k_quant_absmax(const uint4* __restrict__ a, const float* __restrict__ absmax, int rows, int k8,
+                               int8_t* __restrict__ q, float* __restrict__ scale) {
+  const size_t total = static_cast<size_t>(rows) * k8;
+  const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
+  uint2* q2 = reinterpret_cast<uint2*>(q);
+  for (size_t e = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < total; e += stride) {
+    const size_t row = e / k8;
+    const float s = absmax[row] / 127.0f;
+    float f[8];
+    bf16x8_to_f32(__ldcs(a + e), f);
+    q2[e] = quant8(f, s);
+    if (e - row * k8 == 0) scale[row] = s;
+  }
+}
+
+int grid_for(size_t work_items, int num_sms, int per_sm = 8) {
+  const size_t want = (work_items + kThreads - 1) / kThreads;
+  const size_t cap = static_cast<size_t>(num_sms) * per_sm;
+  return static_cast<int>(want < cap ? (want > 0 ? want : 1) : cap);
+}
+
+}  // namespace
+
+cudaError_t launch_flow_step(const Ctx& c, float* x, const float* v, float dt, size_t n, float* x_copy) {
+  if (n == 0) return cudaSuccess;
+  k_flow<<<grid_for((n + 3) / 4, c.num_sms), kThreads, 0, c.stream>>>(x, v, dt, n, x_copy);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_merge(const Ctx& c, const float* x, float* xm, int n_video, int n_audio, int d) {
+  const int d4 = d / 4;
+  const size_t total = static_cast<size_t>(n_video / 2 + n_audio) * d4;
+  if (total == 0) return cudaSuccess;
+  k_merge<<<grid_for(total, c.num_sms), kThreads, 0, c.stream>>>(reinterpret_cast<const float4*>(x),
+                                                                  reinterpret_cast<float4*>(xm), n_video / 2,
+                                                                  n_audio, d4);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_unmerge(const Ctx& c, const float* xm, float* x, int n_video, int n_audio, int d) {
+  const int d4 = d / 4;
+  const size_t total = static_cast<size_t>(n_video + n_audio) * d4;
+  if (total == 0) return cudaSuccess;
+  k_unmerge<<<grid_for(total, c.num_sms), kThreads, 0, c.stream>>>(reinterpret_cast<const float4*>(xm),
+                                                                    reinterpret_cast<float4*>(x), n_video, n_audio,
+                                                                    d4);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rope_table(const Ctx& c, const h3b_dims& dm, int merged, float* table) {
+  const int wc = merged ? dm.cols / 2 : dm.cols;
+  const size_t total = static_cast<size_t>(dm.frames * dm.rows * wc + dm.n_audio) * (dm.head_dim / 2);
+  if (total == 0) return cudaSuccess;
+  k_rope_table<<<grid_for(total, c.num_sms, 4), kThreads, 0, c.stream>>>(
+      reinterpret_cast<float2*>(table), dm.frames, dm.rows, wc, dm.n_audio, dm.head_dim, dm.rope_theta, merged);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rmsnorm(const Ctx& c, const float* x, const float* g, int rows, int d, float eps, void* out,
+                           float* out_scale, int out_int8) {
+  if (rows == 0) return cudaSuccess;
+  const int d4 = d / 4;
+  int threads = d4 >= kThreads ? kThreads : ((d4 + 31) / 32) * 32;
+  const int vpt = (d4 + threads - 1) / threads;
+#define H3B_NORM_CASE(V)                                                                                  \
+  case V:                                                                                                 \
+    if (out_int8)                                                                                         \
+      k_rmsnorm<V, true><<<rows, threads, 0, c.stream>>>(x, g, d, eps, out, out_scale);                   \
+    else                                                                                                  \
+      k_rmsnorm<V, false><<<rows, threads, 0, c.stream>>>(x, g, d, eps, out, out_scale);                  \
+    break;
+  switch (vpt) {
+    H3B_NORM_CASE(1) H3B_NORM_CASE(2) H3B_NORM_CASE(3) H3B_NORM_CASE(4)
+    H3B_NORM_CASE(5) H3B_NORM_CASE(6) H3B_NORM_CASE(7) H3B_NORM_CASE(8)
+    default: return cudaErrorInvalidValue;
+  }
+#undef H3B_NORM_CASE
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quant_rows(const Ctx& c, const void* a, int rows, int k, int8_t* q, float* s) {
+  if (rows == 0) return cudaSuccess;
+  const int k8 = k / 8;
+  const int threads = k8 >= kThreads ? kThreads : ((k8 + 31) / 32) * 32;
+  const int vpt = (k8 + threads - 1) / threads;
+  const uint4* a4 = reinterpret_cast<const uint4*>(a);
+#define H3B_Q_CASE(V) \
+  case V: k_quant_rows<V><<<rows, threads, 0, c.stream>>>(a4, k8, q, s); break;
+  switch (vpt) {
+    H3B_Q_CASE(1) H3B_Q_CASE(2) H3B_Q_CASE(3) H3B_Q_CASE(4) H3B_Q_CASE(5) H3B_Q_CASE(6)
+    H3B_Q_CASE(7) H3B_Q_CASE(8) H3B_Q_CASE(9) H3B_Q_CASE(10) H3B_Q_CASE(11) H3B_Q_CASE(12)
+    H3B_Q_CASE(13) H3B_Q_CASE(14) H3B_Q_CASE(15) H3B_Q_CASE(16)
+    default: return cudaErrorInvalidValue;
+  }
+#undef H3B_Q_CASE
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quant_absmax(const Ctx& c, const void* a, const float* absmax, int rows, int k, int8_t* q,
+                                float* s) {
+  const size_t total = static_cast<size_t>(rows) * (k / 8);
+  if (total == 0) return cudaSuccess;
+  k_quant_absmax<<<grid_for(total, c.num_sms), kThreads, 0, c.stream>>>(reinterpret_cast<const uint4*>(a), absmax,
+                                                                         rows, k / 8, q, s);
+  return cudaGetLastError();
+}
+
+}  // namespace h3b

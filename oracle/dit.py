@@ -38,7 +38,7 @@ from scipy.special import erf as _erf
 
 __all__ = [
     "READINGS", "PINS",
-    "rmsnorm", "gelu", "rope_sections", "token_positions", "rope_angles", "apply_rope",
+    "linear", "rmsnorm", "gelu", "rope_sections", "token_positions", "rope_angles", "apply_rope",
     "attention", "block_forward", "stack_forward", "token_merge", "token_unmerge",
     "quantize_rows", "dequantize_rows", "int8_matmul", "dequant_weights", "block_forward_w8a8",
     "sigmas", "is_fresh", "fresh_steps", "flow_step", "denoise",
@@ -87,7 +87,12 @@ def _f64(a):
     return np.asarray(a, dtype=np.float64)
 
 
-# ----------------------------------------------------------------------------- norm / activation
+# ----------------------------------------------------------------------------- linear / norm / activation
+def linear(a, w):
+    """y = a W^T for W stored [out, in] (a library matmul in fp64)."""
+    return _f64(a) @ _f64(w).T
+
+
 def rmsnorm(x, g, eps):
     """u = x * 1/sqrt(mean_j x_j^2 + eps) * g, per row (token)."""
     x = _f64(x)

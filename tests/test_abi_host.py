@@ -1,0 +1,103 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every function include/h3b.h declares, and rejects bad arguments before it
+touches the device."""
+import ctypes
+
+import pytest
+
+import workloads as wlmod
+
+h3b = pytest.importorskip("audio_diffusion_transformer_dit_b200.h3b")
+
+
+def test_every_header_function_is_exported():
+    names = h3b.header_functions()
+    assert len(names) >= 20
+    for n in names:
+        assert hasattr(h3b.lib, n), n
+
+
+def test_status_strings():
+    for code in range(0, -9, -1):
+        assert h3b.lib.h3b_status_string(code).decode() != "unknown status"
+    assert h3b.lib.h3b_status_string(-99).decode() == "unknown status"
+
+
+def test_seq_len_and_workspace_plan():
+    wl = wlmod.WORKLOADS["stack8_d5120_s6528"]
+    dm = h3b.dims_of(wl)
+    assert h3b.seq_len(dm) == 6528 and h3b.seq_len(dm, True) == 3456
+    S, d, f = 6528, 5120, 20480
+    ws = h3b.workspace_bytes(dm)
+    # aliased arenas: max(qkv+o+u1, u2+g) = max(10dS, 2dS+2fS) bytes, plus scales and the RoPE table
+    arena = max(10 * d * S, 2 * d * S + 2 * f * S)
+    extra = ws - arena
+    assert 0 < extra < 3 * 4 * S + S * 64 * 8 + 8 * 256
+    assert h3b.workspace_saved_bytes(dm) == (6 + 2 + 2 + 2) * d * S + 2 * f * S - arena
+    wsr = h3b.workspace_bytes(dm, h3b.BF16, True)
+    assert wsr - ws >= 3456 * d * 4 + 3456 * 64 * 8
+    assert h3b.workspace_bytes(dm, h3b.INT8) > 0
+
+
+def test_invalid_dims_rejected():
+    base = dict(frames=2, rows=2, cols=2, n_audio=1, d=256, n_heads=2, head_dim=128, ffn=1024, eps=1e-6,
+                rope_theta=1e4)
+    assert h3b.lib.h3b_seq_len(ctypes.byref(h3b.Dims(**base)), 0) == 9
+    for bad in (dict(head_dim=96, n_heads=3, d=288), dict(d=384), dict(ffn=1000), dict(eps=-1.0),
+                dict(frames=-1), dict(frames=0, n_audio=0)):
+        dm = h3b.Dims(**{**base, **bad})
+        assert h3b.lib.h3b_seq_len(ctypes.byref(dm), 0) == -1
+        assert h3b.lib.h3b_workspace_bytes(ctypes.byref(dm), 0, 0) == 0
+    odd = h3b.Dims(**{**base, "cols": 3})
+    assert h3b.lib.h3b_seq_len(ctypes.byref(odd), 1) == -1
+    assert h3b.lib.h3b_workspace_bytes(ctypes.byref(odd), 0, 1) == 0
+
+
+def _weights(ptr, dtype=0):
+    return h3b.BlockWeights(dtype, ptr, ptr, ptr, ptr, ptr, ptr, ptr, ptr, ptr, ptr)
+
+
+# Every call below fails validation on the host; none may reach a launch (the
+# pointers are fake), so each case breaks at least one rule.
+def test_block_forward_argument_errors_before_device():
+    dm = h3b.dims_of(wlmod.WORKLOADS["block_d256_s288"])
+    need = h3b.workspace_bytes(dm)
+    fake = 1 << 20  # never dereferenced: validation fails first
+    w = _weights(fake)
+    f = h3b.lib.h3b_block_forward
+    assert f(ctypes.byref(dm), ctypes.byref(w), None, 0, fake, need, None) == -1
+    assert f(ctypes.byref(dm), ctypes.byref(w), fake + 4, 0, fake, need, None) == -2
+    assert f(ctypes.byref(dm), ctypes.byref(w), fake, 0, fake, need - 1, None) == -5
+    assert f(ctypes.byref(dm), ctypes.byref(_weights(fake, 7)), fake, 0, fake, need, None) == -4
+    assert f(ctypes.byref(dm), ctypes.byref(_weights(fake, 1)), fake, 0, fake, need, None) == -5  # int8 needs more
+    bad = h3b.Dims(dm.frames, dm.rows, dm.cols, dm.n_audio, 200, 2, 100, 800, 1e-6, 1e4)
+    assert f(ctypes.byref(bad), ctypes.byref(w), fake, 0, fake, need, None) == -3
+
+
+def test_stack_and_denoise_argument_errors():
+    dm = h3b.dims_of(wlmod.WORKLOADS["block_d256_s288"])
+    fake = 1 << 20
+    arr = (h3b.BlockWeights * 3)(_weights(fake), _weights(fake), _weights(fake))
+    need = h3b.workspace_bytes(dm, 0, 1)
+    st = h3b.lib.h3b_stack_forward
+    assert st(ctypes.byref(dm), arr, 3, 2, 1, fake, fake, need, None) == -3      # last < first
+    assert st(ctypes.byref(dm), arr, 3, 1, 3, fake, fake, need, None) == -3      # last beyond stack
+    assert st(ctypes.byref(dm), arr, 3, 0, 2, fake, fake, need - 256, None) == -5
+    mixed = (h3b.BlockWeights * 2)(_weights(fake, 0), _weights(fake, 1))
+    assert st(ctypes.byref(dm), mixed, 2, -1, -1, fake, fake, need, None) == -4
+    dn = h3b.lib.h3b_denoise
+    assert dn(ctypes.byref(dm), arr, 3, -1, -1, 0, 2, fake, fake, fake, need, None, None) == -3
+    assert dn(ctypes.byref(dm), arr, 3, -1, -1, 20, 0, fake, fake, fake, need, None, None) == -3
+    assert dn(ctypes.byref(dm), arr, 3, -1, -1, 20, 2, fake, None, fake, need, None, None) == -1
+
+
+def test_gemm_argument_errors():
+    g = h3b.lib.h3b_gemm
+    fake = 1 << 20
+    assert g(fake, fake, 128, 100, 128, 0, 0, fake, None, None, None, None, None, None) == -3   # N % 32
+    assert g(fake, fake, 128, 128, 96, 0, 0, fake, None, None, None, None, None, None) == -3    # K % 64
+    assert g(fake, fake, 128, 128, 64, 1, 0, fake, None, None, None, None, None, None) == -3    # int8 K % 128
+    assert g(fake, fake, 128, 128, 128, 0, 5, fake, None, None, None, None, None, None) == -4   # I32 needs int8
+    assert g(fake, fake, 128, 128, 128, 1, 0, fake, None, None, None, None, None, None) == -1   # scales
+    assert g(fake, fake, 128, 128, 128, 0, 9, fake, None, None, None, None, None, None) == -4
+    assert g(fake, fake + 8, 128, 128, 128, 0, 0, fake, None, None, None, None, None, None) == -2

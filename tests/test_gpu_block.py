@@ -1,0 +1,214 @@
+"""Block, stack and denoising-loop parity through the C ABI against the oracle.
+
+Tolerances (per the block's stated bar): block output relative L2 <= 1e-2 and
+max-abs <= 5e-2 for BF16; relative L2 <= 2e-2 for INT8 against the oracle
+block run on the int8 round-trip of the weights.  The block update x2 - x is
+also checked on its own (a stricter view: the residual dominates x2), with a
+bound derived from the bf16 roundings on the path (u, qkv, P, o, u2, GELU out:
+six roundings of 2^-9 relative each, attenuated through the GEMMs) -> 2e-2
+for BF16; for INT8 the per-token activation codes add ~1% per GEMM -> 6e-2.
+At full sizes the oracle computes a sample of output rows (all keys/values).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as wlmod
+from tests._util import np64, rel_l2, max_abs, host_weights
+
+pytestmark = pytest.mark.gpu
+
+h3b = pytest.importorskip("audio_diffusion_transformer_dit_b200.h3b")
+
+TINY = wlmod.WORKLOADS["block_d256_s288"]
+
+
+def make_block(wl, layer, dev, int8):
+    w = wlmod.block_weights(wl, layer, dev)
+    return w, (h3b.Block.quantized(w) if int8 else h3b.Block.from_dict(w))
+
+
+def run_block(wl, layer, dev, int8=False, merged=False):
+    w, blk = make_block(wl, layer, dev, int8)
+    dm = h3b.dims_of(wl)
+    S = h3b.seq_len(dm, merged)
+    x0 = wlmod.initial_tokens(wl, dev, seq=S)
+    x = x0.clone()
+    ws = h3b.workspace(dm, h3b.INT8 if int8 else h3b.BF16)
+    h3b.block_forward(dm, blk, x, ws, merged)
+    torch.cuda.synchronize()
+    assert h3b.device_error() == 0
+    return np64(x0), np64(x), host_weights(w)
+
+
+def check_bf16(x0, got, ref):
+    assert np.isfinite(got).all()
+    assert rel_l2(got, ref) <= 1e-2
+    assert max_abs(got, ref) <= 5e-2
+    assert rel_l2(got - x0, ref - x0) <= 2e-2
+
+
+def check_int8(x0, got, ref):
+    assert np.isfinite(got).all()
+    assert rel_l2(got, ref) <= 2e-2
+    assert rel_l2(got - x0, ref - x0) <= 6e-2
+
+
+@pytest.mark.parametrize("merged", [False, True])
+def test_block_tiny_bf16(cuda_dev, merged):
+    x0, got, w = run_block(TINY, 0, cuda_dev, merged=merged)
+    check_bf16(x0, got, oracle.block_forward(x0, w, TINY, merged=merged))
+
+
+def test_block_tiny_int8(cuda_dev):
+    x0, got, w = run_block(TINY, 0, cuda_dev, int8=True)
+    check_int8(x0, got, oracle.block_forward(x0, oracle.dequant_weights(w), TINY))
+
+
+@pytest.mark.parametrize("int8", [False, True])
+def test_block_medium(cuda_dev, int8):
+    wl = wlmod.Workload("m", 3, 10, 12, 77, 1024, 8, 128, 4096, 1, 1 if int8 else 0, 11, False)
+    x0, got, w = run_block(wl, 0, cuda_dev, int8=int8)
+    if int8:
+        check_int8(x0, got, oracle.block_forward(x0, oracle.dequant_weights(w), wl))
+    else:
+        check_bf16(x0, got, oracle.block_forward(x0, w, wl))
+
+
+def test_block_head_dim_64(cuda_dev):
+    wl = wlmod.Workload("h64", 2, 6, 8, 21, 512, 8, 64, 2048, 1, 0, 12, False)
+    x0, got, w = run_block(wl, 0, cuda_dev)
+    check_bf16(x0, got, oracle.block_forward(x0, w, wl))
+
+
+def sample_rows(S, n_video, k=48, seed=0):
+    rng = np.random.default_rng(seed)
+    fixed = [0, 1, 127, 128, n_video - 1, n_video, S - 1]
+    return np.unique(np.concatenate([fixed, rng.choice(S, size=k, replace=False)]))
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name,layer,merged", [("block_d3072_s6400", 0, False),
+                                               ("stack8_d5120_s6528", 0, False),
+                                               ("stack8_d5120_s6528", 7, False),
+                                               ("loop45_d5120_s6528", 20, True)])
+def test_block_full_size_sampled(cuda_dev, name, layer, merged):
+    wl = wlmod.WORKLOADS[name]
+    x0, got, w = run_block(wl, layer, cuda_dev, merged=merged)
+    S = x0.shape[0]
+    nv = wl.n_video // 2 if merged else wl.n_video
+    rows = sample_rows(S, nv)
+    ref = oracle.block_forward(x0, w, wl, merged=merged, rows=rows)
+    check_bf16(x0[rows], got[rows], ref)
+
+
+@pytest.mark.slow
+def test_block_int8_full_size_sampled(cuda_dev):
+    wl = wlmod.WORKLOADS["block_int8_d5120_s20640"]
+    x0, got, w = run_block(wl, 0, cuda_dev, int8=True)
+    rows = sample_rows(x0.shape[0], wl.n_video, k=32)
+    ref = oracle.block_forward(x0, oracle.dequant_weights(w), wl, rows=rows)
+    check_int8(x0[rows], got[rows], ref)
+
+
+# ----------------------------------------------------------------------------- stack
+def run_stack(wl, dev, mf=-1, ml=-1):
+    ws_ = [wlmod.block_weights(wl, l, dev) for l in range(wl.n_blocks)]
+    blocks = [h3b.Block.from_dict(w) for w in ws_]
+    dm = h3b.dims_of(wl)
+    x0 = wlmod.initial_tokens(wl, dev)
+    x = x0.clone()
+    ws = h3b.workspace(dm, h3b.BF16, mf >= 0)
+    h3b.stack_forward(dm, blocks, x, ws, mf, ml)
+    torch.cuda.synchronize()
+    return x0, x, ws_, blocks, ws
+
+
+@pytest.mark.parametrize("mf,ml", [(-1, -1), (2, 4)])
+def test_stack_small_vs_oracle(cuda_dev, mf, ml):
+    wl = TINY.with_(n_blocks=6, depth_scaled_init=True, seed=5)
+    x0, x, ws_, _, _ = run_stack(wl, cuda_dev, mf, ml)
+    ref = oracle.stack_forward(np64(x0), [host_weights(w) for w in ws_], wl, mf, ml)
+    check_bf16(np64(x0), np64(x), ref)
+
+
+def test_stack_equals_block_sequence(cuda_dev):
+    """h3b_stack_forward = merge + the same block calls + unmerge, bit for bit."""
+    wl = TINY.with_(n_blocks=5, depth_scaled_init=True, seed=6)
+    x0, x, _, blocks, ws = run_stack(wl, cuda_dev, 1, 3)
+    dm = h3b.dims_of(wl)
+    y = x0.clone()
+    for l in (0,):
+        h3b.block_forward(dm, blocks[l], y, ws)
+    ym = torch.empty((h3b.seq_len(dm, True), wl.d), device=cuda_dev)
+    h3b.token_merge(dm, y, ym)
+    for l in (1, 2, 3):
+        h3b.block_forward(dm, blocks[l], ym, ws, merged=True)
+    h3b.token_unmerge(dm, ym, y)
+    h3b.block_forward(dm, blocks[4], y, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(x, y)
+
+
+@pytest.mark.slow
+def test_stack8_full_size_equals_blocks(cuda_dev):
+    wl = wlmod.WORKLOADS["stack8_d5120_s6528"]
+    x0, x, _, blocks, ws = run_stack(wl, cuda_dev)
+    dm = h3b.dims_of(wl)
+    y = x0.clone()
+    for b in blocks:
+        h3b.block_forward(dm, b, y, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(x, y)
+    assert torch.isfinite(x).all()
+
+
+# ----------------------------------------------------------------------------- denoising loop
+@pytest.mark.parametrize("steps,reuse,mf,ml", [(5, 2, 1, 2), (4, 1, -1, -1), (20, 3, -1, -1)])
+def test_denoise_small_vs_oracle(cuda_dev, steps, reuse, mf, ml):
+    wl = TINY.with_(n_blocks=4, depth_scaled_init=True, seed=7)
+    ws_ = [wlmod.block_weights(wl, l, cuda_dev) for l in range(wl.n_blocks)]
+    blocks = [h3b.Block.from_dict(w) for w in ws_]
+    dm = h3b.dims_of(wl)
+    x0 = wlmod.initial_tokens(wl, cuda_dev)
+    x = x0.clone()
+    v = torch.empty_like(x)
+    ws = h3b.workspace(dm, h3b.BF16, mf >= 0)
+    nf = h3b.denoise(dm, blocks, x, v, ws, steps, reuse, mf, ml)
+    torch.cuda.synchronize()
+    ref, nf_ref = oracle.denoise(np64(x0), [host_weights(w) for w in ws_], wl, steps, reuse, mf, ml)
+    assert nf == nf_ref == len(oracle.fresh_steps(steps, reuse))
+    assert rel_l2(x, ref) <= 1e-2
+    assert max_abs(x, ref) <= 5e-2
+
+
+def test_denoise_fresh_counts(cuda_dev):
+    wl = TINY.with_(n_blocks=1)
+    blocks = [h3b.Block.from_dict(wlmod.block_weights(wl, 0, cuda_dev))]
+    dm = h3b.dims_of(wl)
+    x = wlmod.initial_tokens(wl, cuda_dev)
+    v = torch.empty_like(x)
+    ws = h3b.workspace(dm)
+    assert [h3b.denoise(dm, blocks, x, v, ws, 20, r) for r in (1, 2, 3)] == [20, 11, 8]
+
+
+# ----------------------------------------------------------------------------- host-side errors on a GPU machine
+def test_workspace_too_small_is_rejected(cuda_dev):
+    dm = h3b.dims_of(TINY)
+    _, blk = make_block(TINY, 0, cuda_dev, False)
+    x = wlmod.initial_tokens(TINY, cuda_dev)
+    ws = torch.empty(h3b.workspace_bytes(dm) - 256, dtype=torch.uint8, device=cuda_dev)
+    with pytest.raises(h3b.H3bError) as e:
+        h3b.block_forward(dm, blk, x, ws)
+    assert e.value.status == -5
+
+
+def test_misaligned_pointer_is_rejected(cuda_dev):
+    dm = h3b.dims_of(TINY)
+    _, blk = make_block(TINY, 0, cuda_dev, False)
+    buf = torch.zeros(TINY.seq * TINY.d + 1, device=cuda_dev)
+    ws = h3b.workspace(dm)
+    st = h3b.lib.h3b_block_forward(h3b.ctypes.byref(dm), h3b.ctypes.byref(blk.c), buf.data_ptr() + 4, 0,
+                                   ws.data_ptr(), ws.numel(), h3b._stream())
+    assert st == -2

@@ -1,0 +1,284 @@
+"""Kernel-level parity: each h3b kernel, called through the C ABI, against the
+CPU oracle on the same seeded inputs (ragged tails and several tiles)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as wlmod
+from tests._util import np64, rel_l2, max_abs, ulp_diff_f32
+
+pytestmark = pytest.mark.gpu
+
+h3b = pytest.importorskip("audio_diffusion_transformer_dit_b200.h3b")
+
+
+def small_dims(F=2, H=4, W=6, A=5, d=256, heads=4, ffn=1024):
+    return wlmod.Workload("t", F, H, W, A, d, heads, d // heads, ffn, 1, 0, 0, False)
+
+
+# ----------------------------------------------------------------------------- Euler step
+@pytest.mark.parametrize("n", [0, 1, 7, 4096, 1_000_003])
+def test_flow_step(cuda_dev, n):
+    x = wlmod.normal_tensor((n,), 1, cuda_dev)
+    v = wlmod.normal_tensor((n,), 2, cuda_dev)
+    x0 = x.clone()
+    cp = torch.full_like(x, 7.0)
+    s0, s1 = np.float32(0.65), np.float32(0.6)
+    h3b.flow_step(x, v, float(s0), float(s1), x_copy=cp)
+    torch.cuda.synchronize()
+    ref = oracle.flow_step(np64(x0), np64(v), s0, s1).astype(np.float32)
+    got = x.cpu().numpy()
+    assert np.all(ulp_diff_f32(got, ref) <= 1)
+    assert np.array_equal(cp.cpu().numpy(), got)
+
+
+def test_flow_step_zero_velocity_identity(cuda_dev):
+    x = wlmod.normal_tensor((12345,), 3, cuda_dev)
+    x0 = x.clone()
+    h3b.flow_step(x, torch.zeros_like(x), 0.9, 0.85)
+    assert torch.equal(x, x0)
+
+
+# ----------------------------------------------------------------------------- token reduction
+@pytest.mark.parametrize("geom", [(2, 3, 4, 5, 128), (6, 32, 32, 384, 256), (1, 1, 2, 0, 128), (5, 48, 84, 480, 5120)])
+def test_merge_unmerge_bitexact(cuda_dev, geom):
+    F, H, W, A, d = geom
+    wl = wlmod.Workload("g", F, H, W, A, d, d // 128, 128, 4 * d, 1, 0, 0, False)
+    dm = h3b.dims_of(wl)
+    x = wlmod.normal_tensor((F * H * W + A, d), 4, cuda_dev) * 3.0
+    xm = torch.empty((F * H * W // 2 + A, d), dtype=torch.float32, device=cuda_dev)
+    h3b.token_merge(dm, x, xm)
+    torch.cuda.synchronize()
+    ref = oracle.token_merge(np64(x), wl)
+    assert np.array_equal(xm.cpu().numpy(), ref.astype(np.float32))
+    back = torch.empty_like(x)
+    h3b.token_unmerge(dm, xm, back)
+    torch.cuda.synchronize()
+    assert np.array_equal(back.cpu().numpy(), oracle.token_unmerge(ref, wl).astype(np.float32))
+
+
+def test_merge_rejects_odd_width(cuda_dev):
+    wl = wlmod.Workload("g", 2, 3, 5, 1, 128, 1, 128, 512, 1, 0, 0, False)
+    x = torch.zeros((31, 128), device=cuda_dev)
+    xm = torch.zeros((31, 128), device=cuda_dev)
+    with pytest.raises(h3b.H3bError) as e:
+        h3b.token_merge(h3b.dims_of(wl), x, xm)
+    assert e.value.status == -3
+
+
+def test_merge_unmerge_identity_pair_constant(cuda_dev):
+    wl = small_dims(3, 4, 8, 7, 256, 2, 1024)
+    dm = h3b.dims_of(wl)
+    m = wlmod.normal_tensor((h3b.seq_len(dm, True), 256), 5, cuda_dev)
+    x = torch.empty((h3b.seq_len(dm), 256), dtype=torch.float32, device=cuda_dev)
+    h3b.token_unmerge(dm, m, x)
+    m2 = torch.empty_like(m)
+    h3b.token_merge(dm, x, m2)
+    x2 = torch.empty_like(x)
+    h3b.token_unmerge(dm, m2, x2)
+    assert torch.equal(m2, m) and torch.equal(x2, x)
+
+
+# ----------------------------------------------------------------------------- RoPE table
+@pytest.mark.parametrize("merged", [False, True])
+@pytest.mark.parametrize("hd", [64, 128])
+def test_rope_table(cuda_dev, merged, hd):
+    wl = small_dims(3, 5, 84, 37, 2 * hd, 2, 8 * hd)
+    dm = h3b.dims_of(wl)
+    tab = h3b.rope_table(dm, merged)
+    torch.cuda.synchronize()
+    ang = oracle.rope_angles(wl, merged)
+    t = tab.cpu().double().numpy()
+    assert t.shape[:2] == ang.shape
+    assert np.max(np.abs(t[..., 0] - np.cos(ang))) < 1e-6
+    assert np.max(np.abs(t[..., 1] - np.sin(ang))) < 1e-6
+
+
+# ----------------------------------------------------------------------------- RMSNorm
+@pytest.mark.parametrize("rows,d", [(1, 128), (37, 256), (300, 3072), (129, 5120), (3, 8192)])
+def test_rmsnorm_bf16(cuda_dev, rows, d):
+    x = wlmod.normal_tensor((rows, d), 6, cuda_dev) * 2.0
+    g = wlmod.uniform_tensor((d,), 7, cuda_dev, 0.5, 1.5)
+    u = h3b.rmsnorm(x, g, 1e-6)
+    torch.cuda.synchronize()
+    ref = oracle.rmsnorm(np64(x), np64(g), 1e-6)
+    # one bf16 rounding of an fp32 value: relative error <= 2^-8
+    assert np.all(np.abs(np64(u) - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-30)
+
+
+@pytest.mark.parametrize("rows,d", [(37, 256), (300, 5120)])
+def test_rmsnorm_int8(cuda_dev, rows, d):
+    x = wlmod.normal_tensor((rows, d), 8, cuda_dev)
+    g = torch.ones(d, device=cuda_dev)
+    q, s = h3b.rmsnorm(x, g, 1e-6, int8=True)
+    torch.cuda.synchronize()
+    u = oracle.rmsnorm(np64(x), np.ones(d), 1e-6)
+    qr, sr = oracle.quantize_rows(u)
+    # the kernel's u is fp32 arithmetic, the oracle's fp64: scales agree to fp32
+    # rounding, codes agree except at rare near-ties (never by more than 1)
+    assert np.allclose(s.cpu().numpy(), sr, rtol=1e-6)
+    dq = np.abs(q.cpu().numpy().astype(int) - qr.astype(int))
+    assert dq.max() <= 1 and (dq > 0).mean() < 1e-3
+
+
+# ----------------------------------------------------------------------------- quantisation
+@pytest.mark.parametrize("rows,k", [(1, 8), (33, 256), (300, 5120), (17, 20480), (5, 32768)])
+def test_quantize_weights_bitexact(cuda_dev, rows, k):
+    w = (wlmod.normal_tensor((rows, k), 9, cuda_dev) * 0.02).to(torch.bfloat16)
+    w[0, :] = 0  # zero row -> s = 0, q = 0
+    q, s = h3b.quantize_weights(w)
+    torch.cuda.synchronize()
+    qr, sr = oracle.quantize_rows(w.float().cpu().numpy())
+    assert np.array_equal(s.cpu().numpy(), sr)
+    assert np.array_equal(q.cpu().numpy(), qr)
+
+
+def test_quantize_rows_absmax_bitexact(cuda_dev):
+    a = (wlmod.normal_tensor((77, 1024), 10, cuda_dev) * 3).to(torch.bfloat16)
+    amax = a.float().abs().amax(dim=1).contiguous()
+    q, s = h3b.quantize_rows_absmax(a, amax)
+    torch.cuda.synchronize()
+    qr, sr = oracle.quantize_rows(a.float().cpu().numpy())
+    assert np.array_equal(s.cpu().numpy(), sr) and np.array_equal(q.cpu().numpy(), qr)
+
+
+# ----------------------------------------------------------------------------- GEMM
+GEMM_SHAPES = [(1, 256, 64), (300, 768, 512), (129, 288, 1024), (1000, 1536, 3072), (6528, 512, 128)]
+
+
+@pytest.mark.parametrize("M,N,K", GEMM_SHAPES)
+def test_gemm_bf16_f32(cuda_dev, M, N, K):
+    A = wlmod.normal_tensor((M, K), 11, cuda_dev, dtype=torch.bfloat16)
+    B = wlmod.normal_tensor((N, K), 12, cuda_dev, 0.02, dtype=torch.bfloat16)
+    C = torch.full((M, N), float("nan"), device=cuda_dev)
+    h3b.gemm(A, B, h3b.EPI_F32, C)
+    torch.cuda.synchronize()
+    ref = oracle.linear(np64(A), np64(B))
+    assert np.isfinite(C.cpu().numpy()).all()
+    # fp32 accumulation of exact bf16 products
+    assert max_abs(C, ref) <= 2e-5 * np.sqrt(K) * np.abs(ref).max() + 1e-6
+    assert rel_l2(C, ref) < 1e-5
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 256, 128), (300, 512, 1024), (129, 288, 2048), (700, 1024, 5120)])
+def test_gemm_int8_i32_bitexact(cuda_dev, M, N, K):
+    A = wlmod.int8_tensor((M, K), 13, cuda_dev)
+    B = wlmod.int8_tensor((N, K), 14, cuda_dev)
+    C = torch.zeros((M, N), dtype=torch.int32, device=cuda_dev)
+    h3b.gemm(A, B, h3b.EPI_I32, C)
+    torch.cuda.synchronize()
+    ref = oracle.int8_matmul(A.cpu().numpy(), B.cpu().numpy())
+    assert np.array_equal(C.cpu().numpy().astype(np.int64), ref)
+
+
+def test_gemm_int8_extremes_bitexact(cuda_dev):
+    K = 4096
+    A = torch.full((130, K), 127, dtype=torch.int8, device=cuda_dev)
+    A[1::2] = -127
+    B = torch.full((256, K), -127, dtype=torch.int8, device=cuda_dev)
+    C = torch.zeros((130, 256), dtype=torch.int32, device=cuda_dev)
+    h3b.gemm(A, B, h3b.EPI_I32, C)
+    torch.cuda.synchronize()
+    ref = oracle.int8_matmul(A.cpu().numpy(), B.cpu().numpy())
+    assert np.array_equal(C.cpu().numpy().astype(np.int64), ref)
+
+
+def test_gemm_int8_dequant(cuda_dev):
+    M, N, K = 300, 512, 1024
+    A = wlmod.int8_tensor((M, K), 15, cuda_dev)
+    B = wlmod.int8_tensor((N, K), 16, cuda_dev)
+    sa = wlmod.uniform_tensor((M,), 17, cuda_dev, 0.001, 0.01)
+    sb = wlmod.uniform_tensor((N,), 18, cuda_dev, 0.001, 0.01)
+    C = torch.empty((M, N), device=cuda_dev)
+    h3b.gemm(A, B, h3b.EPI_F32, C, scale_a=sa, scale_b=sb)
+    torch.cuda.synchronize()
+    acc = oracle.int8_matmul(A.cpu().numpy(), B.cpu().numpy()).astype(np.float64)
+    ref = acc * np64(sa)[:, None] * np64(sb)[None, :]
+    assert rel_l2(C, ref) < 1e-6
+
+
+@pytest.mark.parametrize("int8", [False, True])
+def test_gemm_resid_and_gelu(cuda_dev, int8):
+    M, N, K = 333, 768, 1024
+    if int8:
+        A, B = wlmod.int8_tensor((M, K), 19, cuda_dev), wlmod.int8_tensor((N, K), 20, cuda_dev)
+        sa = wlmod.uniform_tensor((M,), 21, cuda_dev, 0.001, 0.003)
+        sb = wlmod.uniform_tensor((N,), 22, cuda_dev, 0.001, 0.003)
+        acc = oracle.int8_matmul(A.cpu().numpy(), B.cpu().numpy()) * np64(sa)[:, None] * np64(sb)[None, :]
+    else:
+        A = wlmod.normal_tensor((M, K), 19, cuda_dev, dtype=torch.bfloat16)
+        B = wlmod.normal_tensor((N, K), 20, cuda_dev, 0.05, dtype=torch.bfloat16)
+        sa = sb = None
+        acc = oracle.linear(np64(A), np64(B))
+    x = wlmod.normal_tensor((M, N), 23, cuda_dev)
+    x0 = np64(x)
+    h3b.gemm(A, B, h3b.EPI_RESID, x, scale_a=sa, scale_b=sb)
+    g = torch.empty((M, N), dtype=torch.bfloat16, device=cuda_dev)
+    amax = torch.zeros(M, device=cuda_dev)
+    h3b.gemm(A, B, h3b.EPI_GELU, g, scale_a=sa, scale_b=sb, row_absmax=amax if int8 else None)
+    torch.cuda.synchronize()
+    assert rel_l2(np64(x) - x0, acc) < 1e-5
+    ref_g = oracle.gelu(acc)
+    assert np.all(np.abs(np64(g) - ref_g) <= 2.0 ** -8 * np.abs(ref_g) + 1e-5 * np.abs(acc).max())
+    if int8:
+        assert np.array_equal(amax.cpu().numpy(), g.float().abs().amax(dim=1).cpu().numpy())
+
+
+@pytest.mark.parametrize("int8", [False, True])
+@pytest.mark.parametrize("hd,merged", [(64, False), (128, False), (128, True)])
+def test_gemm_qkv_rope(cuda_dev, int8, hd, merged):
+    wl = small_dims(2, 4, 6, 19, 2 * hd, 2, 8 * hd)
+    dm = h3b.dims_of(wl)
+    S, d = h3b.seq_len(dm, merged), wl.d
+    tab = h3b.rope_table(dm, merged)
+    if int8:
+        A, B = wlmod.int8_tensor((S, d), 24, cuda_dev), wlmod.int8_tensor((3 * d, d), 25, cuda_dev)
+        sa = wlmod.uniform_tensor((S,), 26, cuda_dev, 0.001, 0.003)
+        sb = wlmod.uniform_tensor((3 * d,), 27, cuda_dev, 0.001, 0.003)
+        acc = oracle.int8_matmul(A.cpu().numpy(), B.cpu().numpy()) * np64(sa)[:, None] * np64(sb)[None, :]
+    else:
+        A = wlmod.normal_tensor((S, d), 24, cuda_dev, dtype=torch.bfloat16)
+        B = wlmod.normal_tensor((3 * d, d), 25, cuda_dev, 0.05, dtype=torch.bfloat16)
+        sa = sb = None
+        acc = oracle.linear(np64(A), np64(B))
+    C = torch.empty((S, 3 * d), dtype=torch.bfloat16, device=cuda_dev)
+    h3b.gemm(A, B, h3b.EPI_QKV_ROPE, C, scale_a=sa, scale_b=sb, rope=tab, dims=dm)
+    torch.cuda.synchronize()
+    ang = oracle.rope_angles(wl, merged)
+    ref = np.concatenate([oracle.apply_rope(acc[:, :d], ang, 2), oracle.apply_rope(acc[:, d:2 * d], ang, 2),
+                          acc[:, 2 * d:]], axis=1)
+    assert np.all(np.abs(np64(C) - ref) <= 2.0 ** -8 * np.abs(ref) + 2e-5 * np.abs(ref).max())
+
+
+# ----------------------------------------------------------------------------- attention
+@pytest.mark.parametrize("S,H,D", [(1, 1, 64), (100, 2, 64), (128, 2, 128), (288, 4, 64), (1000, 3, 128),
+                                   (2049, 2, 128)])
+def test_attention(cuda_dev, S, H, D):
+    qkv = wlmod.normal_tensor((S, 3 * H * D), 28, cuda_dev, 1.5, dtype=torch.bfloat16)
+    o = h3b.attention(qkv, H, D)
+    torch.cuda.synchronize()
+    assert h3b.device_error() == 0
+    q = np64(qkv)
+    d = H * D
+    ref = oracle.attention(q[:, :d], q[:, d:2 * d], q[:, 2 * d:], H)
+    assert np.isfinite(np64(o)).all()
+    assert rel_l2(o, ref) < 1e-2
+    assert max_abs(o, ref) < 3e-2
+
+
+def test_attention_large_scores(cuda_dev):
+    """Growing row maxima across key tiles exercise the lazy O rescale."""
+    S, H, D = 700, 2, 128
+    g = torch.Generator(device="cpu").manual_seed(3)
+    qkv = torch.randn((S, 3 * H * D), generator=g) * 0.3
+    qkv[:, :H * D] *= 6.0
+    ramp = torch.linspace(0.2, 4.0, S)[:, None]
+    qkv[:, H * D:2 * H * D] *= ramp  # later keys have larger norms -> maxima grow along the sweep
+    qkv = qkv.to(torch.bfloat16).to(cuda_dev)
+    o = h3b.attention(qkv, H, D)
+    torch.cuda.synchronize()
+    q = np64(qkv)
+    d = H * D
+    ref = oracle.attention(q[:, :d], q[:, d:2 * d], q[:, 2 * d:], H)
+    assert rel_l2(o, ref) < 1e-2
