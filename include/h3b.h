@@ -167,6 +167,31 @@ int h3b_token_unmerge(const h3b_dims* dims, const float* xm, float* x, void* str
 int h3b_flow_step(float* x, const float* v, float sigma_cur, float sigma_next, size_t n,
                   float* x_copy, void* stream);
 
+/* Allocation-free block forward (no counterpart on the pages; added for
+ * callers that may not allocate device memory -- e.g. code hosted in an
+ * application that owns and accounts for all device memory through its own
+ * pool, or a latency-critical thread that must not call cudaMalloc, which can
+ * synchronise the device).  Same computation, arguments and results as
+ * h3b_block_forward, without the workspace: the scratch is a fixed array of
+ * H3B_NOALLOC_MAX_BYTES inside the library's device image, held on every GPU
+ * that loads the library until the process exits.
+ *   - Sizes whose workspace (h3b_workspace_bytes(dims, dtype, 0)) exceeds
+ *     H3B_NOALLOC_MAX_BYTES are rejected with H3B_ERR_WORKSPACE; nothing is
+ *     enqueued.  32 MiB covers e.g. d = 256 at S = 288 and d = 1024 at
+ *     S ~ 3000 tokens.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current); make that first call
+ *     before any stream capture.
+ *   - Calls allocate nothing (no cudaMalloc/cudaFree, no allocating library
+ *     routine).
+ *   - Every call shares the one array per device, which keeps the previous
+ *     call's contents; what must start at zero is cleared inside each call.
+ *     Calls whose work overlaps on the GPU (other streams, other host
+ *     threads) race on that array: order them on one stream. */
+#define H3B_NOALLOC_MAX_BYTES (32u << 20)
+int h3b_block_forward_noalloc(const h3b_dims* dims, const h3b_block_weights* w, float* x, int merged,
+                              void* stream);
+
 /* ---------------------------------------------------------------------------
  * Unit-level entry points: the individual kernels the block is made of, for
  * kernel-by-kernel parity tests and timing.  Same conventions as above.
