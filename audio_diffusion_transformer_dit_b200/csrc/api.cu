@@ -532,6 +532,17 @@ int h3b_attention(const void* qkv, int S, int n_heads, int head_dim, void* o, vo
   return H3B_OK;
 }
 
+int h3b_exp2_poly(const float* x, float* y, int n, void* stream) {
+  if (n < 0) return H3B_ERR_DIMS;
+  if (n == 0) return H3B_OK;
+  if (!x || !y) return H3B_ERR_NULL;
+  if (!aligned16(x) || !aligned16(y)) return H3B_ERR_ALIGN;
+  Ctx c;
+  H3B_TRY(device_ctx(static_cast<cudaStream_t>(stream), &c));
+  H3B_CU(KID_ATTN, launch_exp2_poly(c, x, y, n));
+  return H3B_OK;
+}
+
 int h3b_device_error(void* stream) {
   Ctx c;
   H3B_TRY(device_ctx(static_cast<cudaStream_t>(stream), &c));

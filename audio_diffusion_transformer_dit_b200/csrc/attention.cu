@@ -1,22 +1,30 @@
 // Bidirectional flash attention over the joint video + audio sequence,
 // o = softmax(q k^T / sqrt(D)) v per head, on the sm_100a tcgen05 path.
 //
-// One CTA per (128-query tile, head); 6 warps:
-//   warps 0..3  softmax: thread t owns query row t (= TMEM lane t); reads the
-//               score row from TMEM, keeps the running max m and sum l,
-//               writes P (bf16) into shared memory in the 128-byte-swizzled
-//               K-major layout the MMA reads, and rescales O in TMEM when the
-//               running max grows by more than 2^8 (lazy rescale: the result
-//               o = O / l is exact for any reference max, the threshold only
-//               bounds P <= 256).
-//   warp 4      TMA producer: Q once, then K and V tiles of 128 keys through
+// One CTA per (pair of 128-query tiles A and B, head); both tiles share every
+// K/V tile loaded into shared memory.  10 warps:
+//   warps 0..3  softmax of tile A, warps 4..7 softmax of tile B: thread t of a
+//               warpgroup owns query row t (= TMEM lane t); it reads the score
+//               row S from TMEM, keeps the running max m and sum l, and writes
+//               P (bf16 pairs) back into the same TMEM columns, where the PV
+//               MMA reads it as its A operand.  O is rescaled in TMEM only when
+//               the running max grows by more than 2^8 (lazy rescale: o = O/l
+//               is exact for any reference max, the threshold bounds P <= 256).
+//   warp 8      TMA producer: Q_A, Q_B once; K and V tiles of 128 keys through
 //               two-stage rings.
-//   warp 5      MMA issuer: S_j = Q K_j^T into one of two TMEM score buffers
-//               (128 columns each), then O += P_{j-1} V_{j-1} (O: D columns of
-//               TMEM), so the scores of tile j are computed while the softmax
-//               of tile j-1 runs.
-// Keys past S in the last tile are masked to -inf; query rows past S are
-// computed on zero-filled rows and not stored.
+//   warp 9      MMA issuer: per key tile j, PV_A(j), S_A(j+1), PV_B(j),
+//               S_B(j+1).  MMAs from one thread execute in issue order, so
+//               S_A(j+1) may overwrite the columns PV_A(j) reads P from.
+// TMEM (512 columns): S/P of A [0,128), O of A [128,256), S/P of B
+// [256,384), O of B [384,512).
+//
+// exp2 is split between the MUFU unit (ex2.approx) and the FMA pipe: one pair
+// of every four is evaluated as 2^x = 2^n * p(f), n = rint(x), f = x - n in
+// [-1/2, 1/2], p a degree-3 polynomial fitted to 2^f on that interval by
+// iteratively reweighted least squares on relative error (max relative
+// error 7.5e-5, below the bf16 rounding of P).  Keys past S in the last tile
+// are masked to zero probability (MUFU path only on that tile); query rows
+// past S are computed on zero-filled rows and not stored.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -24,50 +32,139 @@ namespace h3b {
 
 namespace {
 
-constexpr int BQ = 128, BKV = 128, THREADS = 192;
-constexpr int TILE_BYTES_MAX = BQ * 128 * 2;  // 128 rows x D=128 bf16
-constexpr int SMEM_BYTES = 1024 + TILE_BYTES_MAX * 6 + 32 * 8 + 16;
+constexpr int BQ = 128, BKV = 128, THREADS = 320, KS = 2, VS = 2;
 constexpr float RESCALE_LOG2 = 8.0f;
-constexpr int S_COL0 = 0, O_COL = 2 * BKV, TMEM_COLS = 512;
+// TMEM column of tile t's S/P and O regions
+__host__ __device__ constexpr uint32_t s_col(int t) { return t * 256u; }
+__host__ __device__ constexpr uint32_t o_col(int t) { return t * 256u + 128u; }
+constexpr int TMEM_COLS = 512;
+constexpr int NUM_BARS = 16;
+
+template <int D>
+constexpr int smem_bytes() {
+  return 1024 + (2 + KS + VS) * 128 * D * 2 + NUM_BARS * 8 + 16;
+}
+
+// ---------------------------------------------------------------- packed fp32 helpers
+__device__ __forceinline__ uint64_t f2_pack(float a, float b) {
+  return (static_cast<uint64_t>(__float_as_uint(b)) << 32) | __float_as_uint(a);
+}
+__device__ __forceinline__ float f2_lo(uint64_t v) { return __uint_as_float(static_cast<uint32_t>(v)); }
+__device__ __forceinline__ float f2_hi(uint64_t v) { return __uint_as_float(static_cast<uint32_t>(v >> 32)); }
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float ex2_mufu(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float m;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(m) : "f"(a), "f"(b), "f"(c));
+  return m;
+}
+__device__ __forceinline__ uint32_t cvt_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// 2^x for a pair, on the FMA pipe (x >= -126 after clamping; callers never pass -inf).
+__device__ __forceinline__ uint64_t ex2_poly2(uint64_t x) {
+  constexpr float C0 = 0.9999280571937561f, C1 = 0.6932609677314758f, C2 = 0.2426111400127411f,
+                  C3 = 0.0551716685295105f;
+  float x0 = fmaxf(f2_lo(x), -126.f), x1 = fmaxf(f2_hi(x), -126.f);
+  const float t0 = x0 + 12582912.f, t1 = x1 + 12582912.f;  // 1.5 * 2^23: low mantissa bits = rint(x)
+  const uint64_t f = f2_pack(x0 - (t0 - 12582912.f), x1 - (t1 - 12582912.f));
+  uint64_t p = f2_fma(f2_pack(C3, C3), f, f2_pack(C2, C2));
+  p = f2_fma(p, f, f2_pack(C1, C1));
+  p = f2_fma(p, f, f2_pack(C0, C0));
+  const uint32_t e0 = __float_as_uint(t0) << 23, e1 = __float_as_uint(t1) << 23;  // n << 23
+  return f2_pack(__uint_as_float(__float_as_uint(f2_lo(p)) + e0), __uint_as_float(__float_as_uint(f2_hi(p)) + e1));
+}
+
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Half a score tile (64 keys starting at key k0) of one row: exps, partial row
+// sums, bf16 pairs.  LAST: keys >= valid are masked to probability 0.
+template <bool LAST>
+__device__ __forceinline__ void softmax_half(const uint32_t (&r)[64], uint32_t (&pk)[32], uint64_t c2, uint64_t nm2,
+                                             int k0, int valid, uint64_t (&acc)[4]) {
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const uint64_t x = f2_fma(f2_pack(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])), c2, nm2);
+    uint64_t p;
+    if (!LAST && (i & 3) == 3) {
+      p = ex2_poly2(x);
+    } else {
+      float p0 = ex2_mufu(f2_lo(x)), p1 = ex2_mufu(f2_hi(x));
+      if (LAST) {
+        if (k0 + 2 * i >= valid) p0 = 0.f;
+        if (k0 + 2 * i + 1 >= valid) p1 = 0.f;
+      }
+      p = f2_pack(p0, p1);
+    }
+    acc[i & 3] = f2_add(acc[i & 3], p);
+    pk[i] = cvt_bf16x2(f2_lo(p), f2_hi(p));
+  }
+}
 
 template <int D>
 __global__ void __launch_bounds__(THREADS, 1)
     k_attention(const __grid_constant__ CUtensorMap tm, int S, int n_heads, __nv_bfloat16* __restrict__ out,
                 int* err) {
-  constexpr int KB = D / 64;                 // 64-column (128-byte) blocks per head row
-  constexpr int TILE = 128 * D * 2;          // bytes of a 128-row Q/K/V tile
-  constexpr int BLK = 128 * 128;             // bytes of one 128-row x 128-byte block
+  constexpr int KB = D / 64;         // 128-byte column blocks per head row
+  constexpr int TILE = 128 * D * 2;  // bytes of a 128-row Q/K/V tile
+  constexpr int BLK = 128 * 128;     // bytes of one 128-row x 128-byte block
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem;
-  uint8_t* sK = sQ + TILE;        // 2 stages
-  uint8_t* sV = sK + 2 * TILE;    // 2 stages
-  uint8_t* sP = sV + 2 * TILE;    // 128 x 128 bf16 = 2 blocks
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + 2 * BLK);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 32);
+  uint8_t* sQ = smem;               // tiles A, B
+  uint8_t* sK = sQ + 2 * TILE;      // KS stages
+  uint8_t* sV = sK + KS * TILE;     // VS stages
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + VS * TILE);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NUM_BARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const uint32_t b0 = smem_u32(bars);
-  const uint32_t q_full = b0, k_full = b0 + 8, k_empty = b0 + 24, v_full = b0 + 40, v_empty = b0 + 56,
-                 s_full = b0 + 72, s_free = b0 + 88, p_full = b0 + 104, o_done = b0 + 112, mma_done = b0 + 120;
+  const uint32_t q_full = b0, k_full = b0 + 8, k_empty = k_full + 8 * KS, v_full = k_empty + 8 * KS,
+                 v_empty = v_full + 8 * VS, s_full = v_empty + 8 * VS, p_full = s_full + 16, o_final = p_full + 16,
+                 mma_done = o_final + 16;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int qb = blockIdx.x, h = blockIdx.y;
+  const int q0 = blockIdx.x * 2 * BQ, h = blockIdx.y;
   const int d_model = n_heads * D;
   const int nkv = (S + BKV - 1) / BKV;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < KS; ++s) {
       mbar_init(k_full + 8 * s, 1);
       mbar_init(k_empty + 8 * s, 1);
+    }
+    for (int s = 0; s < VS; ++s) {
       mbar_init(v_full + 8 * s, 1);
       mbar_init(v_empty + 8 * s, 1);
-      mbar_init(s_full + 8 * s, 1);
-      mbar_init(s_free + 8 * s, 4);
     }
-    mbar_init(p_full, 4);
-    mbar_init(o_done, 1);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(s_full + 8 * t, 1);
+      mbar_init(p_full + 8 * t, 4);
+      mbar_init(o_final + 8 * t, 1);
+    }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -82,187 +179,199 @@ __global__ void __launch_bounds__(THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       uint32_t k_issued = 0, v_issued = 0, k_par = 0, v_par = 0;
-      mbar_arrive_expect_tx(q_full, TILE);
-      for (int kb = 0; kb < KB; ++kb) tma_load_2d(smem_u32(sQ + kb * BLK), &tm, q_full, h * D + 64 * kb, qb * BQ);
+      mbar_arrive_expect_tx(q_full, 2 * TILE);
+      for (int t = 0; t < 2; ++t)
+        for (int kb = 0; kb < KB; ++kb)
+          tma_load_2d(smem_u32(sQ + t * TILE + kb * BLK), &tm, q_full, h * D + 64 * kb, q0 + t * BQ);
       for (int j = 0; j < nkv; ++j) {
-        const int st = j & 1;
-        const uint32_t ph = (j >> 1) & 1;
-        if (!mbar_wait(k_empty + 8 * st, ph ^ 1, abort_flag, err, (EK_ATTN << 8) | 1)) break;
-        mbar_arrive_expect_tx(k_full + 8 * st, TILE);
+        const int ks = j % KS, vs = j % VS;
+        const uint32_t kph = (j / KS) & 1, vph = (j / VS) & 1;
+        if (!mbar_wait(k_empty + 8 * ks, kph ^ 1, abort_flag, err, (EK_ATTN << 8) | 1)) break;
+        mbar_arrive_expect_tx(k_full + 8 * ks, TILE);
         for (int kb = 0; kb < KB; ++kb)
-          tma_load_2d(smem_u32(sK + st * TILE + kb * BLK), &tm, k_full + 8 * st, d_model + h * D + 64 * kb, j * BKV);
-        k_issued |= 1u << st;
-        k_par = (k_par & ~(1u << st)) | (ph << st);
-        if (!mbar_wait(v_empty + 8 * st, ph ^ 1, abort_flag, err, (EK_ATTN << 8) | 2)) break;
-        mbar_arrive_expect_tx(v_full + 8 * st, TILE);
+          tma_load_2d(smem_u32(sK + ks * TILE + kb * BLK), &tm, k_full + 8 * ks, d_model + h * D + 64 * kb, j * BKV);
+        k_issued |= 1u << ks;
+        k_par = (k_par & ~(1u << ks)) | (kph << ks);
+        if (!mbar_wait(v_empty + 8 * vs, vph ^ 1, abort_flag, err, (EK_ATTN << 8) | 2)) break;
+        mbar_arrive_expect_tx(v_full + 8 * vs, TILE);
         for (int kb = 0; kb < KB; ++kb)
-          tma_load_2d(smem_u32(sV + st * TILE + kb * BLK), &tm, v_full + 8 * st, 2 * d_model + h * D + 64 * kb,
+          tma_load_2d(smem_u32(sV + vs * TILE + kb * BLK), &tm, v_full + 8 * vs, 2 * d_model + h * D + 64 * kb,
                       j * BKV);
-        v_issued |= 1u << st;
-        v_par = (v_par & ~(1u << st)) | (ph << st);
+        v_issued |= 1u << vs;
+        v_par = (v_par & ~(1u << vs)) | (vph << vs);
       }
       mbar_drain(q_full, 0);
-      for (int s = 0; s < 2; ++s) {
+      for (int s = 0; s < KS; ++s)
         if ((k_issued >> s) & 1) mbar_drain(k_full + 8 * s, (k_par >> s) & 1);
+      for (int s = 0; s < VS; ++s)
         if ((v_issued >> s) & 1) mbar_drain(v_full + 8 * s, (v_par >> s) & 1);
-      }
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16(BQ, BKV, false);
       constexpr uint32_t idesc_o = idesc_bf16(BQ, D, true);  // V is MN-major (D contiguous)
-      const uint32_t q0 = smem_u32(sQ), p0 = smem_u32(sP);
-      bool ok = mbar_wait(q_full, 0, abort_flag, err, (EK_ATTN << 8) | 3);
-      tc_fence_after();
-      for (int j = 0; ok && j <= nkv; ++j) {
-        if (j < nkv) {  // S_j = Q K_j^T
-          const int st = j & 1;
-          const uint32_t ph = (j >> 1) & 1;
-          ok = mbar_wait(k_full + 8 * st, ph, abort_flag, err, (EK_ATTN << 8) | 4);
-          if (ok && j >= 2) ok = mbar_wait(s_free + 8 * st, ph ^ 1, abort_flag, err, (EK_ATTN << 8) | 5);
-          if (!ok) break;
-          tc_fence_after();
-          const uint32_t k0 = smem_u32(sK + st * TILE);
+      auto issue_s = [&](int t, int ks) {
+        const uint32_t qa = smem_u32(sQ + t * TILE), ka = smem_u32(sK + ks * TILE);
 #pragma unroll
-          for (int i = 0; i < D / 16; ++i) {
-            const uint32_t off = (i >> 2) * BLK + (i & 3) * 32;
-            mma_bf16_ss(tmem + S_COL0 + st * BKV, desc_sw128_k(q0 + off), desc_sw128_k(k0 + off), idesc_s, i != 0);
-          }
-          tc_commit(s_full + 8 * st);
-          tc_commit(k_empty + 8 * st);
+        for (int i = 0; i < D / 16; ++i) {
+          const uint32_t off = (i >> 2) * BLK + (i & 3) * 32;
+          mma_bf16_ss(tmem + s_col(t), desc_sw128_k(qa + off), desc_sw128_k(ka + off), idesc_s, i != 0);
         }
-        if (j >= 1) {  // O += P_{j-1} V_{j-1}
-          const int jj = j - 1, st = jj & 1;
-          ok = mbar_wait(p_full, jj & 1, abort_flag, err, (EK_ATTN << 8) | 6);
-          if (ok) ok = mbar_wait(v_full + 8 * st, (jj >> 1) & 1, abort_flag, err, (EK_ATTN << 8) | 7);
+      };
+      auto issue_pv = [&](int t, int vs, bool acc) {
+        const uint32_t va = smem_u32(sV + vs * TILE);
+#pragma unroll
+        for (int i = 0; i < BKV / 16; ++i)
+          mma_bf16_ts(tmem + o_col(t), tmem + s_col(t) + 8 * i, desc_sw128_mn(va + i * 16 * 128, BLK), idesc_o,
+                      acc || i != 0);
+      };
+      bool ok = mbar_wait(q_full, 0, abort_flag, err, (EK_ATTN << 8) | 3) &&
+                mbar_wait(k_full, 0, abort_flag, err, (EK_ATTN << 8) | 4);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, 0);
+        tc_commit(s_full);
+        issue_s(1, 0);
+        tc_commit(s_full + 8);
+        tc_commit(k_empty);
+      }
+      for (int j = 0; ok && j < nkv; ++j) {
+        const int vs = j % VS, ks = (j + 1) % KS;
+        const bool more = j + 1 < nkv;
+        ok = mbar_wait(v_full + 8 * vs, (j / VS) & 1, abort_flag, err, (EK_ATTN << 8) | 5) &&
+             mbar_wait(p_full, j & 1, abort_flag, err, (EK_ATTN << 8) | 6);
+        if (!ok) break;
+        tc_fence_after();
+        issue_pv(0, vs, j > 0);
+        if (more) {
+          ok = mbar_wait(k_full + 8 * ks, ((j + 1) / KS) & 1, abort_flag, err, (EK_ATTN << 8) | 7);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t v0 = smem_u32(sV + st * TILE);
-#pragma unroll
-          for (int i = 0; i < BKV / 16; ++i) {
-            const uint64_t ad = desc_sw128_k(p0 + (i >> 2) * BLK + (i & 3) * 32);
-            const uint64_t bd = desc_sw128_mn(v0 + i * 16 * 128, BLK);
-            mma_bf16_ss(tmem + O_COL, ad, bd, idesc_o, (jj | i) != 0);
-          }
-          tc_commit(o_done);
-          tc_commit(v_empty + 8 * st);
+          issue_s(0, ks);
+          tc_commit(s_full);
+        } else {
+          tc_commit(o_final);
+        }
+        ok = mbar_wait(p_full + 8, j & 1, abort_flag, err, (EK_ATTN << 8) | 8);
+        if (!ok) break;
+        tc_fence_after();
+        issue_pv(1, vs, j > 0);
+        tc_commit(v_empty + 8 * vs);
+        if (more) {
+          issue_s(1, ks);
+          tc_commit(s_full + 8);
+          tc_commit(k_empty + 8 * ks);
+        } else {
+          tc_commit(o_final + 8);
         }
       }
       tc_commit(mma_done);
       mbar_drain(mma_done, 0);
     }
   } else {
-    // ------------------------------------------------------------ softmax (warps 0..3)
-    const int row = warp * 32 + lane;
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    // ------------------------------------------------------------ softmax (warps 0..7)
+    const int t = warp >> 2, q = warp & 3;
+    const int row = q * 32 + lane;
+    const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+    const uint32_t sc = tmem + lane_base + s_col(t), oc = tmem + lane_base + o_col(t);
     const float c = 1.4426950408889634f / sqrtf(static_cast<float>(D));  // log2(e) / sqrt(D)
     float m_use = -INFINITY, l = 0.f;
     bool ok = true;
-    const uint32_t prow = smem_u32(sP) + row * 128;
     for (int j = 0; j < nkv; ++j) {
-      const int st = j & 1;
-      ok = mbar_wait(s_full + 8 * st, (j >> 1) & 1, abort_flag, err, (EK_ATTN << 8) | 8);
+      ok = mbar_wait(s_full + 8 * t, j & 1, abort_flag, err, (EK_ATTN << 8) | 9);
       if (!__all_sync(0xffffffffu, ok)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      float s[BKV];
-#pragma unroll
-      for (int cc = 0; cc < BKV / 32; ++cc) {
-        uint32_t r[32];
-        tmem_ld32(tmem + lane_base + S_COL0 + st * BKV + cc * 32, r);
+      const int valid = S - j * BKV;  // keys of this tile that exist (>= 1)
+      float mx0 = -INFINITY, mx1 = -INFINITY;
+      {  // pass 1: row max over the 128 scores
+        uint32_t r[BKV];
+        tmem_ld32(sc + 0, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+        tmem_ld32(sc + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+        tmem_ld32(sc + 64, *reinterpret_cast<uint32_t(*)[32]>(&r[64]));
+        tmem_ld32(sc + 96, *reinterpret_cast<uint32_t(*)[32]>(&r[96]));
         tmem_ld_wait();
+        if (valid >= BKV) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) s[cc * 32 + i] = __uint_as_float(r[i]);
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(s_free + 8 * st);  // score buffer may be overwritten
-
-      const int valid = S - j * BKV;  // keys of this tile that exist
-      float mx = -INFINITY;
+          for (int i = 0; i < BKV; i += 4) {
+            mx0 = max3(mx0, __uint_as_float(r[i]), __uint_as_float(r[i + 1]));
+            mx1 = max3(mx1, __uint_as_float(r[i + 2]), __uint_as_float(r[i + 3]));
+          }
+        } else {
 #pragma unroll
-      for (int i = 0; i < BKV; ++i) {
-        if (i >= valid) s[i] = -INFINITY;
-        mx = fmaxf(mx, s[i]);
+          for (int i = 0; i < BKV; ++i)
+            if (i < valid) mx0 = fmaxf(mx0, __uint_as_float(r[i]));
+        }
       }
-      const float m_new = mx * c;
+      const float m_new = fmaxf(mx0, mx1) * c;
       float alpha = 1.f;
       bool rescale = false;
       if (j == 0) {
         m_use = m_new;
       } else if (m_new > m_use + RESCALE_LOG2) {
-        alpha = exp2f(m_use - m_new);
+        alpha = ex2_mufu(m_use - m_new);
         m_use = m_new;
         rescale = true;
       }
-      float sum = 0.f;
-      uint32_t pk[BKV / 2];
-#pragma unroll
-      for (int i = 0; i < BKV / 2; ++i) {
-        const float p0 = exp2f(fmaf(s[2 * i], c, -m_use));
-        const float p1 = exp2f(fmaf(s[2 * i + 1], c, -m_use));
-        sum += p0 + p1;
-        pk[i] = pack_bf16x2(p0, p1);
-      }
-      l = l * alpha + sum;
-
-      if (j >= 1) {  // PV_{j-1} must be done before P is overwritten or O rescaled
-        ok = mbar_wait(o_done, (j - 1) & 1, abort_flag, err, (EK_ATTN << 8) | 9);
-        if (!__all_sync(0xffffffffu, ok)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        if (__any_sync(0xffffffffu, rescale)) {
+      // The commit behind s_full(j) follows PV(j-1), so O is complete here.
+      if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll 1
-          for (int cc = 0; cc < D / 32; ++cc) {
-            uint32_t r[32];
-            const uint32_t ta = tmem + lane_base + O_COL + cc * 32;
-            tmem_ld32(ta, r);
-            tmem_ld_wait();
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t o[32];
+          tmem_ld32(oc + cc * 32, o);
+          tmem_ld_wait();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-            tmem_st32(ta, r);
-          }
-          tmem_st_wait();
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st32(oc + cc * 32, o);
         }
       }
-      // P row -> shared memory, 128-byte swizzle (16-byte chunk c of row r at c ^ (r % 8))
+      // pass 2: probabilities, 64 keys at a time; P (bf16 pairs) of keys
+      // [64h, 64h+64) goes to columns [32h, 32h+32), already read.
+      const uint64_t c2 = f2_pack(c, c), nm2 = f2_pack(-m_use, -m_use);
+      uint64_t acc[4] = {0, 0, 0, 0};
 #pragma unroll
-      for (int cc = 0; cc < BKV / 8; ++cc) {
-        const uint32_t addr = prow + (cc >> 3) * BLK + ((((cc & 7) ^ (row & 7))) << 4);
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[4 * cc]), "r"(pk[4 * cc + 1]),
-                     "r"(pk[4 * cc + 2]), "r"(pk[4 * cc + 3])
-                     : "memory");
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t r[64];
+        uint32_t pk[32];
+        tmem_ld32(sc + 64 * hh, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+        tmem_ld32(sc + 64 * hh + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+        tmem_ld_wait();
+        if (valid >= BKV)
+          softmax_half<false>(r, pk, c2, nm2, 64 * hh, valid, acc);
+        else
+          softmax_half<true>(r, pk, c2, nm2, 64 * hh, valid, acc);
+        tmem_st32(sc + 32 * hh, pk);
       }
-      fence_proxy_async_smem();
+      const uint64_t sum2 = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
+      l = l * alpha + (f2_lo(sum2) + f2_hi(sum2));
+      tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
+      if (lane == 0) mbar_arrive(p_full + 8 * t);
     }
     if (ok) {
-      ok = mbar_wait(o_done, (nkv - 1) & 1, abort_flag, err, (EK_ATTN << 8) | 10);
+      ok = mbar_wait(o_final + 8 * t, 0, abort_flag, err, (EK_ATTN << 8) | 10);
       if (__all_sync(0xffffffffu, ok)) {
         tc_fence_after();
-        const int grow = qb * BQ + row;
+        const int grow = q0 + t * BQ + row;
         const float inv = 1.f / l;
 #pragma unroll 1
         for (int cc = 0; cc < D / 32; ++cc) {
-          uint32_t r[32];
-          tmem_ld32(tmem + lane_base + O_COL + cc * 32, r);
+          uint32_t o[32];
+          tmem_ld32(oc + cc * 32, o);
           tmem_ld_wait();
           if (grow < S) {
             uint32_t w[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i)
-              w[i] = pack_bf16x2(__uint_as_float(r[2 * i]) * inv, __uint_as_float(r[2 * i + 1]) * inv);
+              w[i] = cvt_bf16x2(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
             uint4* dst = reinterpret_cast<uint4*>(out + static_cast<size_t>(grow) * d_model + h * D + cc * 32);
 #pragma unroll
             for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
@@ -281,7 +390,25 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 }
 
+__global__ void k_exp2_poly(const float* __restrict__ x, float* __restrict__ y, int n) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i + 1 < n) {
+    const uint64_t r = ex2_poly2(f2_pack(x[i], x[i + 1]));
+    y[i] = f2_lo(r);
+    y[i + 1] = f2_hi(r);
+  } else if (i < n) {
+    y[i] = f2_lo(ex2_poly2(f2_pack(x[i], 0.f)));
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_exp2_poly(const Ctx& c, const float* x, float* y, int n) {
+  if (n <= 0) return cudaSuccess;
+  const int threads = 256, blocks = (n / 2 + threads) / threads;
+  k_exp2_poly<<<blocks, threads, 0, c.stream>>>(x, y, n);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_attention(const Ctx& c, const void* qkv, int S, int n_heads, int head_dim, void* o) {
   if (S == 0) return cudaSuccess;
@@ -289,11 +416,14 @@ cudaError_t launch_attention(const Ctx& c, const void* qkv, int S, int n_heads, 
   CUtensorMap tm;
   if (!encode_tmap_2d(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, qkv, 3ull * d_model, S, 3ull * d_model * 2, 64, 128))
     return cudaErrorInvalidValue;
-  auto kern = head_dim == 128 ? k_attention<128> : k_attention<64>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+  const bool d128 = head_dim == 128;
+  auto kern = d128 ? k_attention<128> : k_attention<64>;
+  // both sizes ask for the D=128 footprint: one CTA per SM (it holds all 512 TMEM columns)
+  const int smem = smem_bytes<128>();
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  dim3 grid((S + BQ - 1) / BQ, n_heads);
-  kern<<<grid, THREADS, SMEM_BYTES, c.stream>>>(tm, S, n_heads, static_cast<__nv_bfloat16*>(o), c.err);
+  dim3 grid((S + 2 * BQ - 1) / (2 * BQ), n_heads);
+  kern<<<grid, THREADS, smem, c.stream>>>(tm, S, n_heads, static_cast<__nv_bfloat16*>(o), c.err);
   return cudaGetLastError();
 }
 

@@ -57,6 +57,7 @@ _SIGS = {
     "h3b_gemm": (_i, [_p, _p, _i, _i, _i, _i, _i, _p, _p, _p, _p, ctypes.POINTER(Dims), _p, _p]),
     "h3b_quantize_rows_absmax": (_i, [_p, _p, _i, _i, _p, _p, _p]),
     "h3b_attention": (_i, [_p, _i, _i, _i, _p, _p]),
+    "h3b_exp2_poly": (_i, [_p, _p, _i, _p]),
     "h3b_device_error": (_i, [_p]),
     "h3b_trace_start": (_i, [_i]),
     "h3b_trace_stop": (_i, [ctypes.POINTER(_i)]),
@@ -280,6 +281,12 @@ def attention(qkv: torch.Tensor, n_heads: int, head_dim: int, o: Optional[torch.
     _check(lib.h3b_attention(_ptr(qkv, torch.bfloat16, "qkv"), S, n_heads, head_dim, _ptr(o, torch.bfloat16, "o"),
                              _stream()), "h3b_attention")
     return o
+
+
+def exp2_poly(x: torch.Tensor) -> torch.Tensor:
+    y = torch.empty_like(x)
+    _check(lib.h3b_exp2_poly(_ptr(x, torch.float32, "x"), y.data_ptr(), x.numel(), _stream()), "h3b_exp2_poly")
+    return y
 
 
 def device_error() -> int:

@@ -240,6 +240,12 @@ int h3b_quantize_rows_absmax(const void* a, const float* absmax, int rows, int k
  * (Q heads, then K heads, then V heads); o: bf16 [S, n_heads*head_dim]. */
 int h3b_attention(const void* qkv, int S, int n_heads, int head_dim, void* o, void* stream);
 
+/* The attention kernel's FMA-pipe exp2 (used for one key pair in four):
+ * y = 2^n * p(x - n), n = rint(x), p a degree-3 polynomial fitted to 2^f on
+ * [-1/2, 1/2] (max relative error 7.5e-5); x is clamped to >= -126.
+ * x, y: fp32 [n] device buffers.  For accuracy tests of that approximation. */
+int h3b_exp2_poly(const float* x, float* y, int n, void* stream);
+
 /* ---------------------------------------------------------------------------
  * Device error word and tracing
  * ------------------------------------------------------------------------- */

@@ -282,3 +282,15 @@ def test_attention_large_scores(cuda_dev):
     d = H * D
     ref = oracle.attention(q[:, :d], q[:, d:2 * d], q[:, 2 * d:], H)
     assert rel_l2(o, ref) < 1e-2
+
+
+def test_exp2_poly_error_bound(cuda_dev):
+    """The FMA-pipe exp2 of the attention kernel against 2^x in fp64."""
+    x = torch.cat([torch.linspace(-125.0, 8.0, 1_000_001), torch.tensor([0.0, -0.5, 0.5, 1.0, -1.0, 7.5])])
+    x = x.float().to(cuda_dev)
+    y = h3b.exp2_poly(x)
+    torch.cuda.synchronize()
+    ref = np.exp2(np64(x))
+    rel = np.abs(np64(y) - ref) / ref
+    assert rel.max() < 1e-4
+    assert np64(h3b.exp2_poly(torch.tensor([-300.0, -126.0], device=cuda_dev))).max() < 2.0 ** -125
