@@ -207,6 +207,9 @@ GemmArgs gemm_args(int M, int N, int K, void* C, const float* sa, const float* s
   a.head_dim = dm.head_dim;
   a.row_absmax = amax;
   a.err = err;
+  a.full_tiles = 0;
+  a.split = 1;
+  a.partial = nullptr;
   return a;
 }
 
@@ -225,14 +228,19 @@ int block_impl(const Ctx& c, const h3b_dims& dm, const h3b_block_weights& w, flo
     H3B_CU(KID_RMSNORM, launch_rmsnorm(c, x, w.g_attn, S, d, dm.eps, u1, nullptr, 0));
     H3B_CU(KID_GEMM_QKV, launch_gemm(c, u1, w.w_qkv, 0, H3B_EPI_QKV_ROPE,
                                      gemm_args(S, 3 * d, d, qkv, nullptr, nullptr, rope, dm, nullptr, c.err)));
-    H3B_CU(KID_ATTN, launch_attention(c, qkv, S, dm.n_heads, dm.head_dim, o));
+    // the norm-1 arena is dead once the QKV GEMM has run: key-split attention partials
+    H3B_CU(KID_ATTN, launch_attention(c, qkv, S, dm.n_heads, dm.head_dim, o, reinterpret_cast<float*>(u1),
+                                      2 * static_cast<size_t>(d) * S));
+    // O-proj: the dead QKV arena holds split-K partials; FC2: the dead MLP-input arena
     H3B_CU(KID_GEMM_O, launch_gemm(c, o, w.w_o, 0, H3B_EPI_RESID,
-                                   gemm_args(S, d, d, x, nullptr, nullptr, nullptr, dm, nullptr, c.err)));
+                                   gemm_args(S, d, d, x, nullptr, nullptr, nullptr, dm, nullptr, c.err),
+                                   reinterpret_cast<float*>(A + p.qkv), p.o - p.qkv));
     H3B_CU(KID_RMSNORM, launch_rmsnorm(c, x, w.g_mlp, S, d, dm.eps, u2, nullptr, 0));
     H3B_CU(KID_GEMM_FC1, launch_gemm(c, u2, w.w_fc1, 0, H3B_EPI_GELU,
                                      gemm_args(S, f, d, g, nullptr, nullptr, nullptr, dm, nullptr, c.err)));
     H3B_CU(KID_GEMM_FC2, launch_gemm(c, g, w.w_fc2, 0, H3B_EPI_RESID,
-                                     gemm_args(S, d, f, x, nullptr, nullptr, nullptr, dm, nullptr, c.err)));
+                                     gemm_args(S, d, f, x, nullptr, nullptr, nullptr, dm, nullptr, c.err),
+                                     reinterpret_cast<float*>(A + p.u2), p.g - p.u2));
   } else {
     int8_t* oq = reinterpret_cast<int8_t*>(A + p.oq);
     int8_t* gq = reinterpret_cast<int8_t*>(A + p.gq);
@@ -241,17 +249,20 @@ int block_impl(const Ctx& c, const h3b_dims& dm, const h3b_block_weights& w, flo
     H3B_CU(KID_RMSNORM, launch_rmsnorm(c, x, w.g_attn, S, d, dm.eps, u1, s_act, 1));
     H3B_CU(KID_GEMM_QKV, launch_gemm(c, u1, w.w_qkv, 1, H3B_EPI_QKV_ROPE,
                                      gemm_args(S, 3 * d, d, qkv, s_act, w.s_qkv, rope, dm, nullptr, c.err)));
-    H3B_CU(KID_ATTN, launch_attention(c, qkv, S, dm.n_heads, dm.head_dim, o));
+    H3B_CU(KID_ATTN, launch_attention(c, qkv, S, dm.n_heads, dm.head_dim, o, reinterpret_cast<float*>(u1),
+                                      static_cast<size_t>(d) * S));
     H3B_CU(KID_QUANT_ROWS, launch_quant_rows(c, o, S, d, oq, s_act));
     H3B_CU(KID_GEMM_O, launch_gemm(c, oq, w.w_o, 1, H3B_EPI_RESID,
-                                   gemm_args(S, d, d, x, s_act, w.s_o, nullptr, dm, nullptr, c.err)));
+                                   gemm_args(S, d, d, x, s_act, w.s_o, nullptr, dm, nullptr, c.err),
+                                   reinterpret_cast<float*>(A + p.qkv), p.o - p.qkv));
     H3B_CU(KID_RMSNORM, launch_rmsnorm(c, x, w.g_mlp, S, d, dm.eps, u2, s_act, 1));
     H3B_CU(KID_MEMSET, cudaMemsetAsync(amax, 0, sizeof(float) * S, c.stream));
     H3B_CU(KID_GEMM_FC1, launch_gemm(c, u2, w.w_fc1, 1, H3B_EPI_GELU,
                                      gemm_args(S, f, d, g, s_act, w.s_fc1, nullptr, dm, amax, c.err)));
     H3B_CU(KID_QUANT_ABSMAX, launch_quant_absmax(c, g, amax, S, f, gq, s_g));
     H3B_CU(KID_GEMM_FC2, launch_gemm(c, gq, w.w_fc2, 1, H3B_EPI_RESID,
-                                     gemm_args(S, d, f, x, s_g, w.s_fc2, nullptr, dm, nullptr, c.err)));
+                                     gemm_args(S, d, f, x, s_g, w.s_fc2, nullptr, dm, nullptr, c.err),
+                                     reinterpret_cast<float*>(A + p.u2), p.g - p.u2));
   }
   return H3B_OK;
 }
@@ -495,7 +506,7 @@ int h3b_rmsnorm(const float* x, const float* g, int rows, int d, float eps, void
 
 int h3b_gemm(const void* A, const void* B, int M, int N, int K, int ab_dtype, int epilogue, void* C,
              const float* scale_a, const float* scale_b, const float* rope_table, const h3b_dims* dims,
-             float* row_absmax, void* stream) {
+             float* row_absmax, void* scratch, size_t scratch_bytes, void* stream) {
   if (!A || !B || !C) return H3B_ERR_NULL;
   if (!aligned16(A) || !aligned16(B) || !aligned16(C)) return H3B_ERR_ALIGN;
   if (ab_dtype != H3B_BF16 && ab_dtype != H3B_INT8) return H3B_ERR_DTYPE;
@@ -517,18 +528,22 @@ int h3b_gemm(const void* A, const void* B, int M, int N, int K, int ab_dtype, in
   if (epilogue == H3B_EPI_GELU && ab_dtype == H3B_INT8 && !row_absmax) return H3B_ERR_NULL;
   Ctx c;
   H3B_TRY(device_ctx(static_cast<cudaStream_t>(stream), &c));
+  if (scratch && !aligned16(scratch)) return H3B_ERR_ALIGN;
   H3B_CU(KID_GEMM, launch_gemm(c, A, B, ab_dtype == H3B_INT8, epilogue,
-                               gemm_args(M, N, K, C, scale_a, scale_b, rope_table, dm, row_absmax, c.err)));
+                               gemm_args(M, N, K, C, scale_a, scale_b, rope_table, dm, row_absmax, c.err),
+                               static_cast<float*>(scratch), scratch ? scratch_bytes : 0));
   return H3B_OK;
 }
 
-int h3b_attention(const void* qkv, int S, int n_heads, int head_dim, void* o, void* stream) {
+int h3b_attention(const void* qkv, int S, int n_heads, int head_dim, void* o, void* scratch, size_t scratch_bytes,
+                  void* stream) {
   if (!qkv || !o) return H3B_ERR_NULL;
-  if (!aligned16(qkv) || !aligned16(o)) return H3B_ERR_ALIGN;
+  if (!aligned16(qkv) || !aligned16(o) || (scratch && !aligned16(scratch))) return H3B_ERR_ALIGN;
   if (S < 0 || n_heads <= 0 || (head_dim != 64 && head_dim != 128)) return H3B_ERR_DIMS;
   Ctx c;
   H3B_TRY(device_ctx(static_cast<cudaStream_t>(stream), &c));
-  H3B_CU(KID_ATTN, launch_attention(c, qkv, S, n_heads, head_dim, o));
+  H3B_CU(KID_ATTN, launch_attention(c, qkv, S, n_heads, head_dim, o, static_cast<float*>(scratch),
+                                    scratch ? scratch_bytes : 0));
   return H3B_OK;
 }
 

@@ -2,7 +2,7 @@
 // o = softmax(q k^T / sqrt(D)) v per head, on the sm_100a tcgen05 path.
 //
 // One CTA per (pair of 128-query tiles A and B, head); both tiles share every
-// K/V tile loaded into shared memory.  10 warps:
+// K/V tile loaded into shared memory.  12 warps (warps 10, 11 idle):
 //   warps 0..3  softmax of tile A, warps 4..7 softmax of tile B: thread t of a
 //               warpgroup owns query row t (= TMEM lane t); it reads the score
 //               row S from TMEM, keeps the running max m and sum l, and writes
@@ -18,8 +18,8 @@
 // TMEM (512 columns): S/P of A [0,128), O of A [128,256), S/P of B
 // [256,384), O of B [384,512).
 //
-// exp2 is split between the MUFU unit (ex2.approx) and the FMA pipe: one pair
-// of every four is evaluated as 2^x = 2^n * p(f), n = rint(x), f = x - n in
+// exp2 runs on the MUFU unit (ex2.approx).  POLY_OF_8 > 0 moves that many
+// key pairs of every eight to the FMA pipe, evaluated as 2^x = 2^n * p(f), n = rint(x), f = x - n in
 // [-1/2, 1/2], p a degree-3 polynomial fitted to 2^f on that interval by
 // iteratively reweighted least squares on relative error (max relative
 // error 7.5e-5, below the bf16 rounding of P).  Keys past S in the last tile
@@ -32,13 +32,32 @@ namespace h3b {
 
 namespace {
 
-constexpr int BQ = 128, BKV = 128, THREADS = 320, KS = 2, VS = 2;
+constexpr int BQ = 128, BKV = 128, THREADS = 384, KS = 2, VS = 2;
+// Register split (setmaxnreg): launch 384 x 168 = 64512; softmax warpgroups
+// 2 x 128 x 216 = 55296 plus control warpgroup 128 x 56 = 7168 -> 62464.
+constexpr int REG_SOFTMAX = 216, REG_CONTROL = 56;
 constexpr float RESCALE_LOG2 = 8.0f;
+constexpr int POLY_OF_8 = 0;   // key pairs (of every 8) that take the FMA-pipe exp2 (0: all on MUFU, measured fastest)
 // TMEM column of tile t's S/P and O regions
 __host__ __device__ constexpr uint32_t s_col(int t) { return t * 256u; }
 __host__ __device__ constexpr uint32_t o_col(int t) { return t * 256u + 128u; }
 constexpr int TMEM_COLS = 512;
-constexpr int NUM_BARS = 16;
+constexpr int NUM_BARS = 18;
+
+struct AttnArgs {
+  int S, n_heads;
+  __nv_bfloat16* out;
+  int* err;
+  int pairs;       // 256-row query pairs per head
+  int n_full;      // work items (pair, head) run whole; the rest are split along keys
+  int ks;          // key-range parts per split item
+  float* partial;  // split parts: O [256][D] fp32, then m [256], l [256] per part
+};
+
+template <int D>
+constexpr int slot_floats() {
+  return 256 * D + 2 * 256;
+}
 
 template <int D>
 constexpr int smem_bytes() {
@@ -100,34 +119,36 @@ __device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
       : "memory");
 }
 
-// Half a score tile (64 keys starting at key k0) of one row: exps, partial row
-// sums, bf16 pairs.  LAST: keys >= valid are masked to probability 0.
-template <bool LAST>
-__device__ __forceinline__ void softmax_half(const uint32_t (&r)[64], uint32_t (&pk)[32], uint64_t c2, uint64_t nm2,
-                                             int k0, int valid, uint64_t (&acc)[4]) {
+// Probabilities of keys [64h, 64h+64) of one row, in place: pair i (keys 2i,
+// 2i+1) reads r[2i], r[2i+1] and leaves its bf16 pair in r[i], a slot already
+// consumed.  Partial row sums go to acc.  LAST: keys >= valid get 0.
+template <bool LAST, int HALF>
+__device__ __forceinline__ void softmax_half(uint32_t (&r)[BKV], uint64_t c2, uint64_t nm2, int valid,
+                                             uint64_t (&acc)[4]) {
 #pragma unroll
-  for (int i = 0; i < 32; ++i) {
+  for (int i = 32 * HALF; i < 32 * HALF + 32; ++i) {
     const uint64_t x = f2_fma(f2_pack(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])), c2, nm2);
     uint64_t p;
-    if (!LAST && (i & 3) == 3) {
+    if (!LAST && (i % 8) >= 8 - POLY_OF_8) {
       p = ex2_poly2(x);
     } else {
       float p0 = ex2_mufu(f2_lo(x)), p1 = ex2_mufu(f2_hi(x));
       if (LAST) {
-        if (k0 + 2 * i >= valid) p0 = 0.f;
-        if (k0 + 2 * i + 1 >= valid) p1 = 0.f;
+        if (2 * i >= valid) p0 = 0.f;
+        if (2 * i + 1 >= valid) p1 = 0.f;
       }
       p = f2_pack(p0, p1);
     }
     acc[i & 3] = f2_add(acc[i & 3], p);
-    pk[i] = cvt_bf16x2(f2_lo(p), f2_hi(p));
+    r[i] = cvt_bf16x2(f2_lo(p), f2_hi(p));
   }
 }
 
 template <int D>
 __global__ void __launch_bounds__(THREADS, 1)
-    k_attention(const __grid_constant__ CUtensorMap tm, int S, int n_heads, __nv_bfloat16* __restrict__ out,
-                int* err) {
+    k_attention(const __grid_constant__ CUtensorMap tm, const AttnArgs a) {
+  const int S = a.S, n_heads = a.n_heads;
+  int* const err = a.err;
   constexpr int KB = D / 64;         // 128-byte column blocks per head row
   constexpr int TILE = 128 * D * 2;  // bytes of a 128-row Q/K/V tile
   constexpr int BLK = 128 * 128;     // bytes of one 128-row x 128-byte block
@@ -142,13 +163,24 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   const uint32_t b0 = smem_u32(bars);
   const uint32_t q_full = b0, k_full = b0 + 8, k_empty = k_full + 8 * KS, v_full = k_empty + 8 * KS,
-                 v_empty = v_full + 8 * VS, s_full = v_empty + 8 * VS, p_full = s_full + 16, o_final = p_full + 16,
-                 mma_done = o_final + 16;
+                 v_empty = v_full + 8 * VS, s_full = v_empty + 8 * VS, p_full = s_full + 16, o_final = p_full + 32,
+                 mma_done = o_final + 16;  // p_full: [tile][half]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int q0 = blockIdx.x * 2 * BQ, h = blockIdx.y;
   const int d_model = n_heads * D;
-  const int nkv = (S + BKV - 1) / BKV;
+  const int nkv_all = (S + BKV - 1) / BKV;
+  // work item (query pair, head) and key-tile range [kv0, kv0 + nkv)
+  int item, kv0 = 0, nkv = nkv_all, slot = -1;
+  if (static_cast<int>(blockIdx.x) < a.n_full) {
+    item = blockIdx.x;
+  } else {
+    slot = blockIdx.x - a.n_full;
+    item = a.n_full + slot / a.ks;
+    const int part = slot % a.ks;
+    kv0 = part * nkv_all / a.ks;
+    nkv = (part + 1) * nkv_all / a.ks - kv0;
+  }
+  const int q0 = (item % a.pairs) * 2 * BQ, h = item / a.pairs;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -162,7 +194,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(s_full + 8 * t, 1);
-      mbar_init(p_full + 8 * t, 4);
+      mbar_init(p_full + 16 * t, 4);
+      mbar_init(p_full + 16 * t + 8, 4);
       mbar_init(o_final + 8 * t, 1);
     }
     mbar_init(mma_done, 1);
@@ -178,7 +211,9 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-
+  if (warp >= 8) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REG_CONTROL));
+  }
   if (warp == 8) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -187,9 +222,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int t = 0; t < 2; ++t)
         for (int kb = 0; kb < KB; ++kb)
           tma_load_2d(smem_u32(sQ + t * TILE + kb * BLK), &tm, q_full, h * D + 64 * kb, q0 + t * BQ);
-      for (int j = 0; j < nkv; ++j) {
-        const int ks = j % KS, vs = j % VS;
-        const uint32_t kph = (j / KS) & 1, vph = (j / VS) & 1;
+      for (int jj = 0; jj < nkv; ++jj) {
+        const int j = kv0 + jj;
+        const int ks = jj % KS, vs = jj % VS;
+        const uint32_t kph = (jj / KS) & 1, vph = (jj / VS) & 1;
         if (!mbar_wait(k_empty + 8 * ks, kph ^ 1, abort_flag, err, (EK_ATTN << 8) | 1)) break;
         mbar_arrive_expect_tx(k_full + 8 * ks, TILE);
         for (int kb = 0; kb < KB; ++kb)
@@ -223,12 +259,20 @@ __global__ void __launch_bounds__(THREADS, 1)
           mma_bf16_ss(tmem + s_col(t), desc_sw128_k(qa + off), desc_sw128_k(ka + off), idesc_s, i != 0);
         }
       };
-      auto issue_pv = [&](int t, int vs, bool acc) {
+      // O_t += P_t V: keys [0,64) once the first half of P is published, then [64,128)
+      auto issue_pv = [&](int t, int vs, bool acc, int j) -> bool {
         const uint32_t va = smem_u32(sV + vs * TILE);
 #pragma unroll
-        for (int i = 0; i < BKV / 16; ++i)
-          mma_bf16_ts(tmem + o_col(t), tmem + s_col(t) + 8 * i, desc_sw128_mn(va + i * 16 * 128, BLK), idesc_o,
-                      acc || i != 0);
+        for (int half = 0; half < 2; ++half) {
+          if (!mbar_wait(p_full + 16 * t + 8 * half, j & 1, abort_flag, err, (EK_ATTN << 8) | (6 + half)))
+            return false;
+          tc_fence_after();
+#pragma unroll
+          for (int i = 4 * half; i < 4 * half + 4; ++i)
+            mma_bf16_ts(tmem + o_col(t), tmem + s_col(t) + 8 * i, desc_sw128_mn(va + i * 16 * 128, BLK), idesc_o,
+                        acc || i != 0);
+        }
+        return true;
       };
       bool ok = mbar_wait(q_full, 0, abort_flag, err, (EK_ATTN << 8) | 3) &&
                 mbar_wait(k_full, 0, abort_flag, err, (EK_ATTN << 8) | 4);
@@ -240,14 +284,12 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc_commit(s_full + 8);
         tc_commit(k_empty);
       }
-      for (int j = 0; ok && j < nkv; ++j) {
+      for (int j = 0; ok && j < nkv; ++j) {  // j: index inside this CTA's key range
         const int vs = j % VS, ks = (j + 1) % KS;
         const bool more = j + 1 < nkv;
         ok = mbar_wait(v_full + 8 * vs, (j / VS) & 1, abort_flag, err, (EK_ATTN << 8) | 5) &&
-             mbar_wait(p_full, j & 1, abort_flag, err, (EK_ATTN << 8) | 6);
+             issue_pv(0, vs, j > 0, j);
         if (!ok) break;
-        tc_fence_after();
-        issue_pv(0, vs, j > 0);
         if (more) {
           ok = mbar_wait(k_full + 8 * ks, ((j + 1) / KS) & 1, abort_flag, err, (EK_ATTN << 8) | 7);
           if (!ok) break;
@@ -257,10 +299,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         } else {
           tc_commit(o_final);
         }
-        ok = mbar_wait(p_full + 8, j & 1, abort_flag, err, (EK_ATTN << 8) | 8);
+        ok = issue_pv(1, vs, j > 0, j);
         if (!ok) break;
-        tc_fence_after();
-        issue_pv(1, vs, j > 0);
         tc_commit(v_empty + 8 * vs);
         if (more) {
           issue_s(1, ks);
@@ -273,8 +313,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc_commit(mma_done);
       mbar_drain(mma_done, 0);
     }
-  } else {
+  } else if (warp < 8) {
     // ------------------------------------------------------------ softmax (warps 0..7)
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(REG_SOFTMAX));
     const int t = warp >> 2, q = warp & 3;
     const int row = q * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
@@ -282,33 +323,32 @@ __global__ void __launch_bounds__(THREADS, 1)
     const float c = 1.4426950408889634f / sqrtf(static_cast<float>(D));  // log2(e) / sqrt(D)
     float m_use = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int j = 0; j < nkv; ++j) {
+    for (int j = 0; j < nkv; ++j) {  // j: index inside this CTA's key range
       ok = mbar_wait(s_full + 8 * t, j & 1, abort_flag, err, (EK_ATTN << 8) | 9);
       if (!__all_sync(0xffffffffu, ok)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const int valid = S - j * BKV;  // keys of this tile that exist (>= 1)
+      const int valid = S - (kv0 + j) * BKV;  // keys of this tile that exist (>= 1)
+      // the whole score row, one TMEM round trip
+      uint32_t r[BKV];
+      tmem_ld32(sc + 0, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+      tmem_ld32(sc + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+      tmem_ld32(sc + 64, *reinterpret_cast<uint32_t(*)[32]>(&r[64]));
+      tmem_ld32(sc + 96, *reinterpret_cast<uint32_t(*)[32]>(&r[96]));
+      tmem_ld_wait();
       float mx0 = -INFINITY, mx1 = -INFINITY;
-      {  // pass 1: row max over the 128 scores
-        uint32_t r[BKV];
-        tmem_ld32(sc + 0, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-        tmem_ld32(sc + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
-        tmem_ld32(sc + 64, *reinterpret_cast<uint32_t(*)[32]>(&r[64]));
-        tmem_ld32(sc + 96, *reinterpret_cast<uint32_t(*)[32]>(&r[96]));
-        tmem_ld_wait();
-        if (valid >= BKV) {
+      if (valid >= BKV) {
 #pragma unroll
-          for (int i = 0; i < BKV; i += 4) {
-            mx0 = max3(mx0, __uint_as_float(r[i]), __uint_as_float(r[i + 1]));
-            mx1 = max3(mx1, __uint_as_float(r[i + 2]), __uint_as_float(r[i + 3]));
-          }
-        } else {
-#pragma unroll
-          for (int i = 0; i < BKV; ++i)
-            if (i < valid) mx0 = fmaxf(mx0, __uint_as_float(r[i]));
+        for (int i = 0; i < BKV; i += 4) {
+          mx0 = max3(mx0, __uint_as_float(r[i]), __uint_as_float(r[i + 1]));
+          mx1 = max3(mx1, __uint_as_float(r[i + 2]), __uint_as_float(r[i + 3]));
         }
+      } else {
+#pragma unroll
+        for (int i = 0; i < BKV; ++i)
+          if (i < valid) mx0 = fmaxf(mx0, __uint_as_float(r[i]));
       }
       const float m_new = fmaxf(mx0, mx1) * c;
       float alpha = 1.f;
@@ -332,33 +372,51 @@ __global__ void __launch_bounds__(THREADS, 1)
           tmem_st32(oc + cc * 32, o);
         }
       }
-      // pass 2: probabilities, 64 keys at a time; P (bf16 pairs) of keys
-      // [64h, 64h+64) goes to columns [32h, 32h+32), already read.
+      // P of keys [0,64) -> TMEM columns [0,32), published; then keys [64,128) -> [32,64)
       const uint64_t c2 = f2_pack(c, c), nm2 = f2_pack(-m_use, -m_use);
       uint64_t acc[4] = {0, 0, 0, 0};
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        uint32_t r[64];
-        uint32_t pk[32];
-        tmem_ld32(sc + 64 * hh, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-        tmem_ld32(sc + 64 * hh + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
-        tmem_ld_wait();
-        if (valid >= BKV)
-          softmax_half<false>(r, pk, c2, nm2, 64 * hh, valid, acc);
-        else
-          softmax_half<true>(r, pk, c2, nm2, 64 * hh, valid, acc);
-        tmem_st32(sc + 32 * hh, pk);
-      }
+      if (valid >= BKV)
+        softmax_half<false, 0>(r, c2, nm2, valid, acc);
+      else
+        softmax_half<true, 0>(r, c2, nm2, valid, acc);
+      tmem_st32(sc + 0, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full + 16 * t);
+      if (valid >= BKV)
+        softmax_half<false, 1>(r, c2, nm2, valid, acc);
+      else
+        softmax_half<true, 1>(r, c2, nm2, valid, acc);
+      tmem_st32(sc + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
       const uint64_t sum2 = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
       l = l * alpha + (f2_lo(sum2) + f2_hi(sum2));
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full + 8 * t);
+      if (lane == 0) mbar_arrive(p_full + 16 * t + 8);
     }
     if (ok) {
       ok = mbar_wait(o_final + 8 * t, 0, abort_flag, err, (EK_ATTN << 8) | 10);
-      if (__all_sync(0xffffffffu, ok)) {
+      if (__all_sync(0xffffffffu, ok) && slot >= 0) {
+        // key-range part: unnormalised O, reference max m (log2 units) and sum l
+        tc_fence_after();
+        float* base = a.partial + static_cast<size_t>(slot) * slot_floats<D>();
+        const int prow = t * BQ + row;
+#pragma unroll 1
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t o[32];
+          tmem_ld32(oc + cc * 32, o);
+          tmem_ld_wait();
+          float4* dst = reinterpret_cast<float4*>(base + static_cast<size_t>(prow) * D + cc * 32);
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            dst[i] = make_float4(__uint_as_float(o[4 * i]), __uint_as_float(o[4 * i + 1]),
+                                 __uint_as_float(o[4 * i + 2]), __uint_as_float(o[4 * i + 3]));
+        }
+        base[256 * D + prow] = m_use;
+        base[256 * D + 256 + prow] = l;
+      } else if (__all_sync(0xffffffffu, ok)) {
         tc_fence_after();
         const int grow = q0 + t * BQ + row;
         const float inv = 1.f / l;
@@ -372,7 +430,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
             for (int i = 0; i < 16; ++i)
               w[i] = cvt_bf16x2(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
-            uint4* dst = reinterpret_cast<uint4*>(out + static_cast<size_t>(grow) * d_model + h * D + cc * 32);
+            uint4* dst = reinterpret_cast<uint4*>(a.out + static_cast<size_t>(grow) * d_model + h * D + cc * 32);
 #pragma unroll
             for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
           }
@@ -388,6 +446,27 @@ __global__ void __launch_bounds__(THREADS, 1)
     tc_fence_after();
     tmem_dealloc(tmem, TMEM_COLS);
   }
+}
+
+// Merge the key-range parts of the split items: with M = max_c m_c,
+// o = sum_c O_c 2^(m_c - M) / sum_c l_c 2^(m_c - M), parts in fixed order.
+template <int D>
+__global__ void __launch_bounds__(D) k_attn_combine(const AttnArgs a) {
+  const int ti = blockIdx.x / 256, r = blockIdx.x % 256, col = threadIdx.x;
+  const int item = a.n_full + ti;
+  const int grow = (item % a.pairs) * 2 * BQ + r, h = item / a.pairs;
+  if (grow >= a.S) return;
+  const float* base = a.partial + static_cast<size_t>(ti) * a.ks * slot_floats<D>();
+  float M = -INFINITY;
+  for (int c = 0; c < a.ks; ++c) M = fmaxf(M, base[static_cast<size_t>(c) * slot_floats<D>() + 256 * D + r]);
+  float L = 0.f, acc = 0.f;
+  for (int c = 0; c < a.ks; ++c) {
+    const float* sl = base + static_cast<size_t>(c) * slot_floats<D>();
+    const float w = exp2f(sl[256 * D + r] - M);
+    L += sl[256 * D + 256 + r] * w;
+    acc += sl[static_cast<size_t>(r) * D + col] * w;
+  }
+  a.out[static_cast<size_t>(grow) * (a.n_heads * D) + h * D + col] = __float2bfloat16_rn(acc / L);
 }
 
 __global__ void k_exp2_poly(const float* __restrict__ x, float* __restrict__ y, int n) {
@@ -410,7 +489,8 @@ cudaError_t launch_exp2_poly(const Ctx& c, const float* x, float* y, int n) {
   return cudaGetLastError();
 }
 
-cudaError_t launch_attention(const Ctx& c, const void* qkv, int S, int n_heads, int head_dim, void* o) {
+cudaError_t launch_attention(const Ctx& c, const void* qkv, int S, int n_heads, int head_dim, void* o,
+                             float* scratch, size_t scratch_bytes) {
   if (S == 0) return cudaSuccess;
   const int d_model = n_heads * head_dim;
   CUtensorMap tm;
@@ -422,8 +502,39 @@ cudaError_t launch_attention(const Ctx& c, const void* qkv, int S, int n_heads, 
   const int smem = smem_bytes<128>();
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  dim3 grid((S + 2 * BQ - 1) / (2 * BQ), n_heads);
-  kern<<<grid, THREADS, smem, c.stream>>>(tm, S, n_heads, static_cast<__nv_bfloat16*>(o), c.err);
+  AttnArgs a;
+  a.S = S;
+  a.n_heads = n_heads;
+  a.out = static_cast<__nv_bfloat16*>(o);
+  a.err = c.err;
+  a.pairs = (S + 2 * BQ - 1) / (2 * BQ);
+  const int items = a.pairs * n_heads, nkv = (S + BKV - 1) / BKV;
+  a.n_full = items;
+  a.ks = 1;
+  a.partial = nullptr;
+  // Items left after the last full wave, when they fill at most half of it,
+  // are cut along the keys over the idle SMs and merged by a second kernel.
+  const int tail = items % c.num_sms;
+  const size_t slot_bytes = sizeof(float) * (d128 ? slot_floats<128>() : slot_floats<64>());
+  if (scratch && items > c.num_sms && tail > 0 && 2 * tail <= c.num_sms) {
+    int ks = c.num_sms / tail;
+    if (ks > nkv / 2) ks = nkv / 2;
+    if (static_cast<size_t>(tail) * ks * slot_bytes > scratch_bytes)
+      ks = static_cast<int>(scratch_bytes / (static_cast<size_t>(tail) * slot_bytes));
+    if (ks >= 2) {
+      a.n_full = items - tail;
+      a.ks = ks;
+      a.partial = scratch;
+    }
+  }
+  const int grid = a.n_full + (items - a.n_full) * a.ks;
+  kern<<<grid, THREADS, smem, c.stream>>>(tm, a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess || a.ks == 1) return e;
+  if (d128)
+    k_attn_combine<128><<<(items - a.n_full) * 256, 128, 0, c.stream>>>(a);
+  else
+    k_attn_combine<64><<<(items - a.n_full) * 256, 64, 0, c.stream>>>(a);
   return cudaGetLastError();
 }
 

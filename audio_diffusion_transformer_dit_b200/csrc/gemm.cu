@@ -8,8 +8,9 @@
 //               B tile [256 x 128 B] per stage, 4 stages.
 //   warp 1      MMA issuer (one thread): 4 MMAs of 128x256xK16 (bf16) or
 //               128x256xK32 (int8) per stage; commits free the stage.
-//   warps 2..5  epilogue: warp w reads TMEM lanes 32*(w%4).. (one output row
-//               per thread), 32 columns at a time.
+//   warps 2..9  epilogue: warp w reads TMEM lanes 32*(w%4).. (one output row
+//               per thread) and writes half of the tile's columns (warps 2..5
+//               the first 128, warps 6..9 the rest), 32 columns at a time.
 // Two 256-column accumulators (all 512 TMEM columns) let the epilogue of
 // tile i overlap the MMAs of tile i+1.
 //
@@ -28,7 +29,8 @@ constexpr int BM = 128, BN = 256, KBYTES = 128, STAGES = 4;
 constexpr int A_STAGE = BM * KBYTES;  // 16 KB
 constexpr int B_STAGE = BN * KBYTES;  // 32 KB
 constexpr int TMEM_COLS = 2 * BN;     // two fp32 / int32 accumulators
-constexpr int THREADS = 192;
+constexpr int EPI_WARPS = 8;  // two warps per TMEM lane quarter, each half of the columns
+constexpr int THREADS = 64 + 32 * EPI_WARPS;
 constexpr int NUM_BARS = 2 * STAGES + 5;
 constexpr int SMEM_BYTES = 1024 + STAGES * (A_STAGE + B_STAGE) + NUM_BARS * 8 + 16;
 constexpr int GROUP_N = 8;  // N tiles per raster group (L2 reuse of A rows)
@@ -43,6 +45,25 @@ __device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int& mb
   const int local = t - g * per_group;
   mb = local / gs;
   nb = first_n + local % gs;
+}
+
+// Work unit u -> (tile t, k-block range [kb0, kb1), split part or -1).  Units
+// below full_tiles are whole tiles; when split > 1 the tiles left after the
+// last full wave are cut into `split` consecutive K ranges each.
+__device__ __forceinline__ void unit_range(int u, int full_tiles, int split, int num_kb, int& t, int& kb0, int& kb1,
+                                           int& part) {
+  if (split <= 1 || u < full_tiles) {
+    t = u;
+    kb0 = 0;
+    kb1 = num_kb;
+    part = -1;
+    return;
+  }
+  const int v = u - full_tiles;
+  t = full_tiles + v / split;
+  part = v % split;
+  kb0 = part * num_kb / split;
+  kb1 = (part + 1) * num_kb / split;
 }
 
 template <bool INT8, int EPI>
@@ -152,7 +173,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(tfull0 + 8 * a, 1);
-      mbar_init(tempty0 + 8 * a, 4);  // one arrival per epilogue warp
+      mbar_init(tempty0 + 8 * a, EPI_WARPS);  // one arrival per epilogue warp
     }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
@@ -170,6 +191,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   const uint32_t tmem_base = *tmem_slot;
 
   const int num_m = (p.M + BM - 1) / BM, num_n = (p.N + BN - 1) / BN, num_tiles = num_m * num_n;
+  const int num_units = p.split > 1 ? p.full_tiles + (num_tiles - p.full_tiles) * p.split : num_tiles;
   constexpr int KE = INT8 ? 128 : 64;  // K elements per stage
   const int num_kb = p.K / KE;
 
@@ -177,11 +199,12 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0, issued = 0, issued_par = 0;
-      for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
-        int mb, nb;
+      for (int u = blockIdx.x; u < num_units; u += gridDim.x) {
+        int t, kb0, kb1, part, mb, nb;
+        unit_range(u, p.full_tiles, p.split, num_kb, t, kb0, kb1, part);
         tile_coords(t, num_m, num_n, mb, nb);
         bool ok = true;
-        for (int kb = 0; kb < num_kb; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(empty0 + 8 * stage, phase ^ 1, abort_flag, p.err, (EK_GEMM << 8) | 1)) {
             ok = false;
             break;
@@ -208,12 +231,14 @@ __global__ void __launch_bounds__(THREADS, 1)
       constexpr uint32_t idesc = INT8 ? idesc_i8(BM, BN) : idesc_bf16(BM, BN, false);
       int stage = 0, acc = 0;
       uint32_t phase = 0, acc_phase = 0;
-      for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+      for (int u = blockIdx.x; u < num_units; u += gridDim.x) {
+        int t, kb0, kb1, part;
+        unit_range(u, p.full_tiles, p.split, num_kb, t, kb0, kb1, part);
         if (!mbar_wait(tempty0 + 8 * acc, acc_phase ^ 1, abort_flag, p.err, (EK_GEMM << 8) | 2)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
         bool ok = true;
-        for (int kb = 0; kb < num_kb; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(full0 + 8 * stage, phase, abort_flag, p.err, (EK_GEMM << 8) | 3)) {
             ok = false;
             break;
@@ -224,9 +249,9 @@ __global__ void __launch_bounds__(THREADS, 1)
           for (int k = 0; k < KBYTES / 32; ++k) {
             const uint64_t ad = desc_sw128_k(a0 + 32 * k), bd = desc_sw128_k(b0 + 32 * k);
             if (INT8)
-              mma_i8_ss(d_tmem, ad, bd, idesc, (kb | k) != 0);
+              mma_i8_ss(d_tmem, ad, bd, idesc, (kb > kb0) || k != 0);
             else
-              mma_bf16_ss(d_tmem, ad, bd, idesc, (kb | k) != 0);
+              mma_bf16_ss(d_tmem, ad, bd, idesc, (kb > kb0) || k != 0);
           }
           tc_commit(empty0 + 8 * stage);  // frees the stage once these MMAs have read it
           if (++stage == STAGES) {
@@ -244,11 +269,13 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_drain(mma_done, 0);
     }
   } else {
-    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int q = warp & 3;              // TMEM lane quarter this warp may access
+    const int ch = (warp - 2) >> 2;      // column half of the tile this warp writes
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
-      int mb, nb;
+    for (int u = blockIdx.x; u < num_units; u += gridDim.x) {
+      int t, kb0, kb1, part, mb, nb;
+      unit_range(u, p.full_tiles, p.split, num_kb, t, kb0, kb1, part);
       tile_coords(t, num_m, num_n, mb, nb);
       const bool ok = mbar_wait(tfull0 + 8 * acc, acc_phase, abort_flag, p.err, (EK_GEMM << 8) | 4);
       if (!__all_sync(0xffffffffu, ok)) break;
@@ -256,13 +283,32 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int m = mb * BM + q * 32 + lane;
       float row_amax = 0.f;
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
+      for (int c = ch * (BN / 64); c < (ch + 1) * (BN / 64); ++c) {
         const int n = nb * BN + c * 32;
         if (n >= p.N) break;
         uint32_t r[32];
         tmem_ld32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN + c * 32, r);
         tmem_ld_wait();
-        if (m < p.M) epilogue_chunk<INT8, EPI>(p, m, n, r, row_amax);
+        if (EPI == H3B_EPI_RESID && part >= 0) {
+          // K-part of a tail tile: fp32 partial into its scratch slot (added into C later, in part order)
+          float4* dst = reinterpret_cast<float4*>(p.partial + (static_cast<size_t>(t - p.full_tiles) * p.split + part) *
+                                                                  (BM * BN) + (q * 32 + lane) * BN + c * 32);
+          if (INT8) {
+            float v[32];
+            const float sa = m < p.M ? p.sa[m] : 0.f;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = static_cast<float>(static_cast<int>(r[i])) * sa * __ldg(p.sb + n + i);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              dst[i] = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
+                                   __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
+          }
+        } else if (m < p.M) {
+          epilogue_chunk<INT8, EPI>(p, m, n, r, row_amax);
+        }
       }
       if (INT8 && EPI == H3B_EPI_GELU && m < p.M)
         atomicMax(reinterpret_cast<int*>(p.row_absmax) + m, __float_as_int(row_amax));
@@ -282,6 +328,21 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 }
 
+// C[m, n] += sum over parts of the tail tiles' fp32 partials, in part order
+// (deterministic).  One CTA per (tail tile, row), one thread per column.
+__global__ void __launch_bounds__(BN) k_splitk_add(float* __restrict__ C, const float* __restrict__ partial, int M,
+                                                   int N, int full_tiles, int split, int num_m, int num_n) {
+  const int i = blockIdx.x / BM, r = blockIdx.x % BM, col = threadIdx.x;
+  int mb, nb;
+  tile_coords(full_tiles + i, num_m, num_n, mb, nb);
+  const int m = mb * BM + r, n = nb * BN + col;
+  if (m >= M || n >= N) return;
+  const float* src = partial + static_cast<size_t>(i) * split * (BM * BN) + r * BN + col;
+  float acc = 0.f;
+  for (int q = 0; q < split; ++q) acc += src[static_cast<size_t>(q) * (BM * BN)];
+  C[static_cast<size_t>(m) * N + n] += acc;
+}
+
 using GemmKernel = void (*)(const CUtensorMap, const CUtensorMap, const GemmArgs);
 
 template <bool INT8>
@@ -299,7 +360,9 @@ GemmKernel pick(int epi) {
 
 }  // namespace
 
-cudaError_t launch_gemm(const Ctx& c, const void* A, const void* B, int ab_int8, int epi, const GemmArgs& args) {
+cudaError_t launch_gemm(const Ctx& c, const void* A, const void* B, int ab_int8, int epi, const GemmArgs& args_in,
+                        float* scratch, size_t scratch_bytes) {
+  GemmArgs args = args_in;
   GemmKernel kern = ab_int8 ? pick<true>(epi) : pick<false>(epi);
   if (!kern) return cudaErrorInvalidValue;
   const int eb = ab_int8 ? 1 : 2;
@@ -310,10 +373,33 @@ cudaError_t launch_gemm(const Ctx& c, const void* A, const void* B, int ab_int8,
     return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  const int tiles = ((args.M + BM - 1) / BM) * ((args.N + BN - 1) / BN);
+  const int num_m = (args.M + BM - 1) / BM, num_n = (args.N + BN - 1) / BN;
+  const int tiles = num_m * num_n;
   const int grid = tiles < c.num_sms ? tiles : c.num_sms;
   if (grid == 0) return cudaSuccess;
+  // Residual GEMMs whose last wave is at most a third full: cut the tail
+  // tiles along K over the idle SMs (partials in the caller's scratch).
+  args.split = 1;
+  args.full_tiles = tiles;
+  args.partial = nullptr;
+  const int num_kb = args.K / (KBYTES / eb);
+  const int rem = tiles % grid;
+  if (epi == H3B_EPI_RESID && scratch && tiles > grid && rem > 0 && 3 * rem <= grid) {
+    int split = grid / rem;
+    if (split > num_kb / 2) split = num_kb / 2;
+    const size_t per_split = static_cast<size_t>(rem) * BM * BN * sizeof(float);
+    if (static_cast<size_t>(split) * per_split > scratch_bytes) split = static_cast<int>(scratch_bytes / per_split);
+    if (split >= 2) {
+      args.split = split;
+      args.full_tiles = tiles - rem;
+      args.partial = scratch;
+    }
+  }
   kern<<<grid, THREADS, SMEM_BYTES, c.stream>>>(ta, tb, args);
+  cudaError_t le = cudaGetLastError();
+  if (le != cudaSuccess || args.split <= 1) return le;
+  k_splitk_add<<<rem * BM, BN, 0, c.stream>>>(static_cast<float*>(args.C), args.partial, args.M, args.N,
+                                              args.full_tiles, args.split, num_m, num_n);
   return cudaGetLastError();
 }
 

@@ -55,12 +55,19 @@ struct GemmArgs {
   int d, head_dim;
   float* row_absmax;
   int* err;
+  // split-K of the tail tiles (residual epilogue only; set by launch_gemm)
+  int full_tiles, split;
+  float* partial;
 };
 
-// A [M,K], B [N,K] K-major (bf16 or int8); C per epilogue.
-cudaError_t launch_gemm(const Ctx& c, const void* A, const void* B, int ab_int8, int epi, const GemmArgs& args);
+// A [M,K], B [N,K] K-major (bf16 or int8); C per epilogue.  scratch (may be
+// NULL) lets a residual GEMM split its last partial wave along K.
+cudaError_t launch_gemm(const Ctx& c, const void* A, const void* B, int ab_int8, int epi, const GemmArgs& args,
+                        float* scratch = nullptr, size_t scratch_bytes = 0);
 
-cudaError_t launch_attention(const Ctx& c, const void* qkv, int S, int n_heads, int head_dim, void* o);
+// scratch (may be NULL) lets the last partial wave of work items split along the keys.
+cudaError_t launch_attention(const Ctx& c, const void* qkv, int S, int n_heads, int head_dim, void* o,
+                             float* scratch = nullptr, size_t scratch_bytes = 0);
 cudaError_t launch_exp2_poly(const Ctx& c, const float* x, float* y, int n);
 
 // tensor-map encoding through the driver entry point (no libcuda link)

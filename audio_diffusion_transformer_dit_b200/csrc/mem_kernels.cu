@@ -252,20 +252,37 @@ __global__ void __launch_bounds__(kThreads) k_quant_rows(const uint4* __restrict
   if (threadIdx.x == 0) scale[row] = s;
 }
 
-// Known row maxima: purely elementwise.
-__global__ void k_quant_absmax(const uint4* __restrict__ a, const float* __restrict__ absmax, int rows, int k8,
+// Known row maxima: purely elementwise.  Grid (chunks, rows); each thread
+// turns 16 bf16 (two 16-byte loads) into 16 codes (one 16-byte store).
+__global__ void k_quant_absmax(const uint4* __restrict__ a, const float* __restrict__ absmax, int k16,
                                int8_t* __restrict__ q, float* __restrict__ scale) {
-  const size_t total = static_cast<size_t>(rows) * k8;
-  const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
-  uint2* q2 = reinterpret_cast<uint2*>(q);
-  for (size_t e = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < total; e += stride) {
-    const size_t row = e / k8;
-    const float s = absmax[row] / 127.0f;
-    float f[8];
-    bf16x8_to_f32(__ldcs(a + e), f);
-    q2[e] = quant8(f, s);
-    if (e - row * k8 == 0) scale[row] = s;
+  const int row = blockIdx.y;
+  const float s = absmax[row] / 127.0f;
+  const uint4* ar = a + static_cast<size_t>(row) * k16 * 2;
+  uint4* qr = reinterpret_cast<uint4*>(q) + static_cast<size_t>(row) * k16;
+  for (int c = blockIdx.x * blockDim.x + threadIdx.x; c < k16; c += gridDim.x * blockDim.x) {
+    float f0[8], f1[8];
+    bf16x8_to_f32(__ldcs(ar + 2 * c), f0);
+    bf16x8_to_f32(__ldcs(ar + 2 * c + 1), f1);
+    const uint2 lo = quant8(f0, s), hi = quant8(f1, s);
+    qr[c] = make_uint4(lo.x, lo.y, hi.x, hi.y);
   }
+  if (blockIdx.x == 0 && threadIdx.x == 0) scale[row] = s;
+}
+
+// Same with 8 elements per thread (k a multiple of 8 but not of 16).
+__global__ void k_quant_absmax8(const uint4* __restrict__ a, const float* __restrict__ absmax, int k8,
+                                int8_t* __restrict__ q, float* __restrict__ scale) {
+  const int row = blockIdx.y;
+  const float s = absmax[row] / 127.0f;
+  const uint4* ar = a + static_cast<size_t>(row) * k8;
+  uint2* qr = reinterpret_cast<uint2*>(q) + static_cast<size_t>(row) * k8;
+  for (int c = blockIdx.x * blockDim.x + threadIdx.x; c < k8; c += gridDim.x * blockDim.x) {
+    float f[8];
+    bf16x8_to_f32(__ldcs(ar + c), f);
+    qr[c] = quant8(f, s);
+  }
+  if (blockIdx.x == 0 && threadIdx.x == 0) scale[row] = s;
 }
 
 int grid_for(size_t work_items, int num_sms, int per_sm = 8) {
@@ -306,7 +323,7 @@ cudaError_t launch_rope_table(const Ctx& c, const h3b_dims& dm, int merged, floa
   const int wc = merged ? dm.cols / 2 : dm.cols;
   const size_t total = static_cast<size_t>(dm.frames * dm.rows * wc + dm.n_audio) * (dm.head_dim / 2);
   if (total == 0) return cudaSuccess;
-  k_rope_table<<<grid_for(total, c.num_sms, 4), kThreads, 0, c.stream>>>(
+  k_rope_table<<<grid_for(total, c.num_sms, 64), kThreads, 0, c.stream>>>(
       reinterpret_cast<float2*>(table), dm.frames, dm.rows, wc, dm.n_audio, dm.head_dim, dm.rope_theta, merged);
   return cudaGetLastError();
 }
@@ -353,10 +370,19 @@ cudaError_t launch_quant_rows(const Ctx& c, const void* a, int rows, int k, int8
 
 cudaError_t launch_quant_absmax(const Ctx& c, const void* a, const float* absmax, int rows, int k, int8_t* q,
                                 float* s) {
-  const size_t total = static_cast<size_t>(rows) * (k / 8);
-  if (total == 0) return cudaSuccess;
-  k_quant_absmax<<<grid_for(total, c.num_sms), kThreads, 0, c.stream>>>(reinterpret_cast<const uint4*>(a), absmax,
-                                                                         rows, k / 8, q, s);
+  if (rows == 0 || k == 0) return cudaSuccess;
+  const int per_thread = (k % 16 == 0) ? 16 : 8;
+  const int chunks = k / per_thread;
+  const int bx = (chunks + kThreads - 1) / kThreads;
+  for (int r0 = 0; r0 < rows; r0 += 65535) {  // grid.y limit
+    const int nr = rows - r0 < 65535 ? rows - r0 : 65535;
+    const dim3 grid(bx, nr);
+    const uint4* a4 = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(a) + static_cast<size_t>(r0) * k);
+    if (per_thread == 16)
+      k_quant_absmax<<<grid, kThreads, 0, c.stream>>>(a4, absmax + r0, chunks, q + static_cast<size_t>(r0) * k, s + r0);
+    else
+      k_quant_absmax8<<<grid, kThreads, 0, c.stream>>>(a4, absmax + r0, chunks, q + static_cast<size_t>(r0) * k, s + r0);
+  }
   return cudaGetLastError();
 }
 

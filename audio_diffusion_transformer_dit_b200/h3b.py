@@ -54,9 +54,9 @@ _SIGS = {
     "h3b_flow_step": (_i, [_p, _p, _f, _f, _sz, _p, _p]),
     "h3b_rope_table": (_i, [ctypes.POINTER(Dims), _i, _p, _p]),
     "h3b_rmsnorm": (_i, [_p, _p, _i, _i, _f, _p, _p, _i, _p]),
-    "h3b_gemm": (_i, [_p, _p, _i, _i, _i, _i, _i, _p, _p, _p, _p, ctypes.POINTER(Dims), _p, _p]),
+    "h3b_gemm": (_i, [_p, _p, _i, _i, _i, _i, _i, _p, _p, _p, _p, ctypes.POINTER(Dims), _p, _p, _sz, _p]),
     "h3b_quantize_rows_absmax": (_i, [_p, _p, _i, _i, _p, _p, _p]),
-    "h3b_attention": (_i, [_p, _i, _i, _i, _p, _p]),
+    "h3b_attention": (_i, [_p, _i, _i, _i, _p, _p, _sz, _p]),
     "h3b_exp2_poly": (_i, [_p, _p, _i, _p]),
     "h3b_device_error": (_i, [_p]),
     "h3b_trace_start": (_i, [_i]),
@@ -254,14 +254,16 @@ def rmsnorm(x: torch.Tensor, g: torch.Tensor, eps: float, int8: bool = False):
 
 
 def gemm(A: torch.Tensor, B: torch.Tensor, epilogue: int, C: torch.Tensor, scale_a=None, scale_b=None,
-         rope: Optional[torch.Tensor] = None, dims: Optional[Dims] = None, row_absmax=None) -> torch.Tensor:
+         rope: Optional[torch.Tensor] = None, dims: Optional[Dims] = None, row_absmax=None,
+         scratch: Optional[torch.Tensor] = None) -> torch.Tensor:
     M, K = A.shape
     N = B.shape[0]
     ab = INT8 if A.dtype == torch.int8 else BF16
     _check(lib.h3b_gemm(_ptr(A, None, "A"), _ptr(B, A.dtype, "B"), M, N, K, ab, epilogue, _ptr(C, None, "C"),
                         _ptr(scale_a, torch.float32, "scale_a"), _ptr(scale_b, torch.float32, "scale_b"),
                         _ptr(rope, torch.float32, "rope"), None if dims is None else ctypes.byref(dims),
-                        _ptr(row_absmax, torch.float32, "row_absmax"), _stream()), "h3b_gemm")
+                        _ptr(row_absmax, torch.float32, "row_absmax"), _ptr(scratch, None, "scratch"),
+                        0 if scratch is None else scratch.numel() * scratch.element_size(), _stream()), "h3b_gemm")
     return C
 
 
@@ -274,12 +276,15 @@ def quantize_rows_absmax(a: torch.Tensor, absmax: torch.Tensor):
     return q, s
 
 
-def attention(qkv: torch.Tensor, n_heads: int, head_dim: int, o: Optional[torch.Tensor] = None) -> torch.Tensor:
+def attention(qkv: torch.Tensor, n_heads: int, head_dim: int, o: Optional[torch.Tensor] = None,
+              scratch: Optional[torch.Tensor] = None) -> torch.Tensor:
     S = qkv.shape[0]
     if o is None:
         o = torch.empty((S, n_heads * head_dim), dtype=torch.bfloat16, device=qkv.device)
     _check(lib.h3b_attention(_ptr(qkv, torch.bfloat16, "qkv"), S, n_heads, head_dim, _ptr(o, torch.bfloat16, "o"),
-                             _stream()), "h3b_attention")
+                             _ptr(scratch, None, "scratch"),
+                             0 if scratch is None else scratch.numel() * scratch.element_size(), _stream()),
+           "h3b_attention")
     return o
 
 

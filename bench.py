@@ -58,6 +58,21 @@ def peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+def max_over_ranks(ms: float, device) -> float:
+    """Slowest rank's time (the job's time) when a process group is up."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return ms
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_value(units_per_step: float, steps: int, world: int, ms: float) -> float:
+    """Units all replicas processed per second of the slowest replica's time."""
+    return units_per_step * steps * world / (ms / 1e3)
+
+
 def dist_env():
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -240,12 +255,7 @@ def run_ours(args, wl):
         torch.cuda.synchronize()
     barrier()
     clocks = sampler.stop()
-    ms = e0.elapsed_time(e1)
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(e0.elapsed_time(e1), dev)
     assert h3b.device_error() == 0, "device error word set during the timed region"
 
     # per-kernel shares from the live trace
@@ -277,7 +287,7 @@ def run_ours(args, wl):
                 "peak_source": f"{src} ({'sustained bf16' if bound == 'tensor' else 'copy'})",
                 "work_per_launch": amount}
 
-    value = units * args.steps * world / (ms / 1e3)
+    value = whole_job_value(units, args.steps, world, ms)
     if loop:
         metric, unit_v, hib = "s per denoise step", "s/step", False
         value = ms / 1e3 / args.steps / wl.steps
@@ -311,14 +321,9 @@ def run_ours(args, wl):
         f1.record(stream)
         torch.cuda.synchronize()
         barrier()
-        ms2 = f0.elapsed_time(f1)
-        if world > 1:
-            import torch.distributed as dist
-            t = torch.tensor([ms2], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms2 = float(t.item())
+        ms2 = max_over_ranks(f0.elapsed_time(f1), dev)
         nb = x.numel() * 4
-        e2e = {"value": round(units * k2 * world / (ms2 / 1e3), 2), "unit": unit_v, "h2d_bytes_per_step": nb,
+        e2e = {"value": round(whole_job_value(units, k2, world, ms2), 2), "unit": unit_v, "h2d_bytes_per_step": nb,
                "d2h_bytes_per_step": nb, "steps": k2}
 
     line = {

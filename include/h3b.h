@@ -225,10 +225,15 @@ int h3b_rmsnorm(const float* x, const float* g, int rows, int d, float eps,
  * multiple of 32.  H3B_EPI_QKV_ROPE needs rope_table (h3b_rope_table of the
  * same sequence) and dims (for d, head_dim).  H3B_EPI_GELU with INT8 needs
  * row_absmax fp32 [M], zeroed by the caller, which receives max |GELU| of
- * each row (after bf16 rounding). */
+ * each row (after bf16 rounding).  scratch (optional, device, scratch_bytes
+ * long): with H3B_EPI_RESID, when the last wave of output tiles would leave
+ * most SMs idle, those tail tiles are split along K over the idle SMs; their
+ * fp32 partials go to scratch (up to 148 tiles x 128 KB) and are added into C
+ * in a fixed order by a second kernel (deterministic).  NULL disables it. */
 int h3b_gemm(const void* A, const void* B, int M, int N, int K, int ab_dtype, int epilogue,
              void* C, const float* scale_a, const float* scale_b, const float* rope_table,
-             const h3b_dims* dims, float* row_absmax, void* stream);
+             const h3b_dims* dims, float* row_absmax, void* scratch, size_t scratch_bytes,
+             void* stream);
 
 /* Quantise bf16 rows with a known max |row| (e.g. from H3B_EPI_GELU):
  * s[r] = absmax[r] / 127, q = rint(a / s) clamped, as h3b_quantize_weights. */
@@ -237,8 +242,14 @@ int h3b_quantize_rows_absmax(const void* a, const float* absmax, int rows, int k
 
 /* Bidirectional attention over the whole sequence, per head:
  * o = softmax(q k^T / sqrt(head_dim)) v.  qkv: bf16 [S, 3*n_heads*head_dim]
- * (Q heads, then K heads, then V heads); o: bf16 [S, n_heads*head_dim]. */
-int h3b_attention(const void* qkv, int S, int n_heads, int head_dim, void* o, void* stream);
+ * (Q heads, then K heads, then V heads); o: bf16 [S, n_heads*head_dim].
+ * scratch (optional, device): when the work items (256 query rows x head)
+ * leave a last wave at most half full, those items are split along the keys
+ * over the idle SMs; each part writes its unnormalised O, running max and sum
+ * to scratch (up to 148 x 130 KB) and a second kernel merges the parts in a
+ * fixed order.  NULL disables it. */
+int h3b_attention(const void* qkv, int S, int n_heads, int head_dim, void* o, void* scratch,
+                  size_t scratch_bytes, void* stream);
 
 /* The attention kernel's FMA-pipe exp2 (used for one key pair in four):
  * y = 2^n * p(x - n), n = rint(x), p a degree-3 polynomial fitted to 2^f on

@@ -94,10 +94,10 @@ def test_stack_and_denoise_argument_errors():
 def test_gemm_argument_errors():
     g = h3b.lib.h3b_gemm
     fake = 1 << 20
-    assert g(fake, fake, 128, 100, 128, 0, 0, fake, None, None, None, None, None, None) == -3   # N % 32
-    assert g(fake, fake, 128, 128, 96, 0, 0, fake, None, None, None, None, None, None) == -3    # K % 64
-    assert g(fake, fake, 128, 128, 64, 1, 0, fake, None, None, None, None, None, None) == -3    # int8 K % 128
-    assert g(fake, fake, 128, 128, 128, 0, 5, fake, None, None, None, None, None, None) == -4   # I32 needs int8
-    assert g(fake, fake, 128, 128, 128, 1, 0, fake, None, None, None, None, None, None) == -1   # scales
-    assert g(fake, fake, 128, 128, 128, 0, 9, fake, None, None, None, None, None, None) == -4
-    assert g(fake, fake + 8, 128, 128, 128, 0, 0, fake, None, None, None, None, None, None) == -2
+    assert g(fake, fake, 128, 100, 128, 0, 0, fake, None, None, None, None, None, None, 0, None) == -3   # N % 32
+    assert g(fake, fake, 128, 128, 96, 0, 0, fake, None, None, None, None, None, None, 0, None) == -3    # K % 64
+    assert g(fake, fake, 128, 128, 64, 1, 0, fake, None, None, None, None, None, None, 0, None) == -3    # int8 K % 128
+    assert g(fake, fake, 128, 128, 128, 0, 5, fake, None, None, None, None, None, None, 0, None) == -4   # I32 needs int8
+    assert g(fake, fake, 128, 128, 128, 1, 0, fake, None, None, None, None, None, None, 0, None) == -1   # scales
+    assert g(fake, fake, 128, 128, 128, 0, 9, fake, None, None, None, None, None, None, 0, None) == -4
+    assert g(fake, fake + 8, 128, 128, 128, 0, 0, fake, None, None, None, None, None, None, 0, None) == -2

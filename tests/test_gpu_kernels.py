@@ -294,3 +294,54 @@ def test_exp2_poly_error_bound(cuda_dev):
     rel = np.abs(np64(y) - ref) / ref
     assert rel.max() < 1e-4
     assert np64(h3b.exp2_poly(torch.tensor([-300.0, -126.0], device=cuda_dev))).max() < 2.0 ** -125
+
+
+@pytest.mark.parametrize("int8", [False, True])
+def test_gemm_resid_split_tail(cuda_dev, int8):
+    """A residual GEMM with a nearly empty last wave (600 tiles on 148 SMs)
+    splits its tail tiles along K; with and without scratch it matches the
+    oracle, and two split runs agree bit for bit."""
+    M, N, K = 6400, 3072, 1024
+    if int8:
+        A, B = wlmod.int8_tensor((M, K), 31, cuda_dev), wlmod.int8_tensor((N, K), 32, cuda_dev)
+        sa = wlmod.uniform_tensor((M,), 33, cuda_dev, 0.001, 0.003)
+        sb = wlmod.uniform_tensor((N,), 34, cuda_dev, 0.001, 0.003)
+        acc = (A.double() @ B.double().T).cpu().numpy() * np64(sa)[:, None] * np64(sb)[None, :]
+    else:
+        A = wlmod.normal_tensor((M, K), 31, cuda_dev, dtype=torch.bfloat16)
+        B = wlmod.normal_tensor((N, K), 32, cuda_dev, 0.05, dtype=torch.bfloat16)
+        sa = sb = None
+        acc = oracle.linear(np64(A), np64(B))
+    x0 = wlmod.normal_tensor((M, N), 35, cuda_dev)
+    scratch = torch.empty(64 << 20, dtype=torch.uint8, device=cuda_dev)
+    outs = []
+    for sc in (None, scratch, scratch):
+        x = x0.clone()
+        h3b.gemm(A, B, h3b.EPI_RESID, x, scale_a=sa, scale_b=sb, scratch=sc)
+        torch.cuda.synchronize()
+        outs.append(x)
+        assert rel_l2(np64(x) - np64(x0), acc) < 1e-5
+    assert torch.equal(outs[1], outs[2])
+    assert rel_l2(outs[1], outs[0]) < 1e-6
+
+
+@pytest.mark.parametrize("S,H,D", [(6400, 24, 128), (6528, 40, 128), (3000, 52, 64)])
+def test_attention_key_split_tail(cuda_dev, S, H, D):
+    """Work-item counts whose last wave is nearly empty (e.g. 600 items on 148
+    SMs) split the tail items along the keys: same result with and without the
+    split (within bf16 rounding), bit-identical across runs, and sampled rows
+    agree with the oracle."""
+    qkv = wlmod.normal_tensor((S, 3 * H * D), 36, cuda_dev, 1.5, dtype=torch.bfloat16)
+    scratch = torch.empty(64 << 20, dtype=torch.uint8, device=cuda_dev)
+    o_plain = h3b.attention(qkv, H, D)
+    o_split = h3b.attention(qkv, H, D, scratch=scratch)
+    o_again = h3b.attention(qkv, H, D, scratch=scratch)
+    torch.cuda.synchronize()
+    assert h3b.device_error() == 0
+    assert torch.equal(o_split, o_again)
+    assert rel_l2(o_split, o_plain) < 4e-3
+    rows = np.unique(np.concatenate([np.arange(S - 300, S), np.linspace(0, S - 1, 64).astype(int)]))
+    q = np64(qkv)
+    d = H * D
+    ref = oracle.attention(q[rows, :d], q[:, d:2 * d], q[:, 2 * d:], H)
+    assert rel_l2(np64(o_split)[rows], ref) < 1e-2
