@@ -558,6 +558,14 @@ int h3b_exp2_poly(const float* x, float* y, int n, void* stream) {
   return H3B_OK;
 }
 
+int h3b_selftest_wait_timeout(int timeout_us, void* stream) {
+  if (timeout_us <= 0 || timeout_us > 1000000) return H3B_ERR_DIMS;
+  Ctx c;
+  H3B_TRY(device_ctx(static_cast<cudaStream_t>(stream), &c));
+  H3B_CU(KID_MEMSET, launch_selftest_wait(c, 1000ull * static_cast<unsigned long long>(timeout_us)));
+  return H3B_OK;
+}
+
 int h3b_device_error(void* stream) {
   Ctx c;
   H3B_TRY(device_ctx(static_cast<cudaStream_t>(stream), &c));

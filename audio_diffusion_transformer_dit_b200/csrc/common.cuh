@@ -20,7 +20,7 @@ namespace h3b {
 constexpr unsigned long long WAIT_TIMEOUT_NS = 2000000000ull;  // 2 s per wait
 
 // Device error word codes: (kernel << 8) | site.
-enum ErrKernel { EK_GEMM = 1, EK_ATTN = 2 };
+enum ErrKernel { EK_GEMM = 1, EK_ATTN = 2, EK_SELFTEST = 3 };
 
 struct Launch {
   cudaStream_t stream;
@@ -76,7 +76,7 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
 // Wait until the phase with the given parity has completed.  Bounded: gives
 // up when the CTA abort flag is raised or after WAIT_TIMEOUT_NS.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                          int* err, int code) {
+                                          int* err, int code, unsigned long long timeout_ns = WAIT_TIMEOUT_NS) {
   if (mbar_test(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   while (true) {
@@ -84,7 +84,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
     for (int i = 0; i < 16; ++i)
       if (mbar_test(bar, parity)) return true;
     if (*abort_flag) return false;
-    if (global_ns() - t0 > WAIT_TIMEOUT_NS) {
+    if (global_ns() - t0 > timeout_ns) {
       *abort_flag = 1;
       atomicCAS(err, 0, code);
       return false;

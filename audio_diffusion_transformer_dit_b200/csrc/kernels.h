@@ -69,6 +69,7 @@ cudaError_t launch_gemm(const Ctx& c, const void* A, const void* B, int ab_int8,
 cudaError_t launch_attention(const Ctx& c, const void* qkv, int S, int n_heads, int head_dim, void* o,
                              float* scratch = nullptr, size_t scratch_bytes = 0);
 cudaError_t launch_exp2_poly(const Ctx& c, const float* x, float* y, int n);
+cudaError_t launch_selftest_wait(const Ctx& c, unsigned long long timeout_ns);
 
 // tensor-map encoding through the driver entry point (no libcuda link)
 bool encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, int elem_bytes, const void* base, uint64_t inner,

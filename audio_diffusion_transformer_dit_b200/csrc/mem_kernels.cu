@@ -285,6 +285,22 @@ __global__ void k_quant_absmax8(const uint4* __restrict__ a, const float* __rest
   if (blockIdx.x == 0 && threadIdx.x == 0) scale[row] = s;
 }
 
+// Failure-path self-test: wait on an mbarrier that nothing will complete,
+// with a short limit; the bounded wait must give up, record its code in the
+// device error word and let the kernel exit normally.
+__global__ void k_selftest_wait(int* err, unsigned long long timeout_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(smem_u32(&bar), 0, &abort_flag, err, (EK_SELFTEST << 8) | 1, timeout_ns);
+  __syncthreads();
+}
+
 int grid_for(size_t work_items, int num_sms, int per_sm = 8) {
   const size_t want = (work_items + kThreads - 1) / kThreads;
   const size_t cap = static_cast<size_t>(num_sms) * per_sm;
@@ -383,6 +399,11 @@ cudaError_t launch_quant_absmax(const Ctx& c, const void* a, const float* absmax
     else
       k_quant_absmax8<<<grid, kThreads, 0, c.stream>>>(a4, absmax + r0, chunks, q + static_cast<size_t>(r0) * k, s + r0);
   }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_selftest_wait(const Ctx& c, unsigned long long timeout_ns) {
+  k_selftest_wait<<<1, 32, 0, c.stream>>>(c.err, timeout_ns);
   return cudaGetLastError();
 }
 

@@ -59,6 +59,7 @@ _SIGS = {
     "h3b_attention": (_i, [_p, _i, _i, _i, _p, _p, _sz, _p]),
     "h3b_exp2_poly": (_i, [_p, _p, _i, _p]),
     "h3b_device_error": (_i, [_p]),
+    "h3b_selftest_wait_timeout": (_i, [_i, _p]),
     "h3b_trace_start": (_i, [_i]),
     "h3b_trace_stop": (_i, [ctypes.POINTER(_i)]),
     "h3b_trace_read": (_i, [_p, _p, _i]),

@@ -261,6 +261,13 @@ int h3b_exp2_poly(const float* x, float* y, int n, void* stream);
  * Device error word and tracing
  * ------------------------------------------------------------------------- */
 
+/* Failure-path self-test: one small kernel waits, with a limit of
+ * timeout_us microseconds (1..1000000), on an mbarrier that nothing
+ * completes.  The bounded wait gives up, records code (3 << 8) | 1 in the
+ * device error word and the kernel exits normally; the context stays usable.
+ * Read the code with h3b_device_error. */
+int h3b_selftest_wait_timeout(int timeout_us, void* stream);
+
 /* Reads and clears the device error word of the current device
  * (synchronises the stream).  0 = no error; otherwise a code naming the
  * kernel and wait that gave up. */

@@ -212,3 +212,18 @@ def test_misaligned_pointer_is_rejected(cuda_dev):
     st = h3b.lib.h3b_block_forward(h3b.ctypes.byref(dm), h3b.ctypes.byref(blk.c), buf.data_ptr() + 4, 0,
                                    ws.data_ptr(), ws.numel(), h3b._stream())
     assert st == -2
+
+
+def test_bounded_wait_reports_and_context_survives(cuda_dev):
+    """A device wait that can never complete gives up after its limit, sets the
+    error word, and later work on the same context runs normally."""
+    assert h3b.device_error() == 0
+    assert h3b.lib.h3b_selftest_wait_timeout(2000, h3b._stream()) == 0
+    torch.cuda.synchronize()
+    assert h3b.device_error() == (3 << 8) | 1
+    assert h3b.device_error() == 0  # cleared by the read
+    x = torch.ones(1024, device=cuda_dev)
+    h3b.flow_step(x, torch.ones_like(x), 1.0, 0.5)
+    torch.cuda.synchronize()
+    assert torch.all(x == 0.5)
+    assert h3b.lib.h3b_selftest_wait_timeout(0, h3b._stream()) == -3
