@@ -3,7 +3,10 @@
 // tcgen05.mma (bf16 -> fp32, or int8 -> int32) with the accumulator in TMEM ->
 // epilogue warps read TMEM and apply the fused epilogue.
 //
-// Structure (one CTA per SM, persistent over output tiles):
+// Two variants, both persistent over output tiles with one CTA per SM: the
+// single-CTA kernel below (128x256 tiles) and a CTA-pair kernel (256x256
+// tiles, tcgen05 cta_group::2, further down) used when the pair tiles fill at
+// least one wave.  Single-CTA structure:
 //   warp 0      TMA producer (one elected thread): A tile [128 x 128 B] and
 //               B tile [256 x 128 B] per stage, 4 stages.
 //   warp 1      MMA issuer (one thread): 4 MMAs of 128x256xK16 (bf16) or
@@ -330,20 +333,294 @@ __global__ void __launch_bounds__(THREADS, 1)
 
 // C[m, n] += sum over parts of the tail tiles' fp32 partials, in part order
 // (deterministic).  One CTA per (tail tile, row), one thread per column.
+template <int TM>
 __global__ void __launch_bounds__(BN) k_splitk_add(float* __restrict__ C, const float* __restrict__ partial, int M,
                                                    int N, int full_tiles, int split, int num_m, int num_n) {
-  const int i = blockIdx.x / BM, r = blockIdx.x % BM, col = threadIdx.x;
+  const int i = blockIdx.x / TM, r = blockIdx.x % TM, col = threadIdx.x;
   int mb, nb;
   tile_coords(full_tiles + i, num_m, num_n, mb, nb);
-  const int m = mb * BM + r, n = nb * BN + col;
+  const int m = mb * TM + r, n = nb * BN + col;
   if (m >= M || n >= N) return;
-  const float* src = partial + static_cast<size_t>(i) * split * (BM * BN) + r * BN + col;
+  const float* src = partial + static_cast<size_t>(i) * split * (TM * BN) + r * BN + col;
   float acc = 0.f;
-  for (int q = 0; q < split; ++q) acc += src[static_cast<size_t>(q) * (BM * BN)];
+  for (int q = 0; q < split; ++q) acc += src[static_cast<size_t>(q) * (TM * BN)];
   C[static_cast<size_t>(m) * N + n] += acc;
 }
 
+// ---------------------------------------------------------------------------
+// 2-SM variant: a cluster of two CTAs computes a 256x256 tile with
+// tcgen05.mma.cta_group::2.  CTA rank r loads rows [128r, 128r+128) of the A
+// tile and rows [128r, 128r+128) of the B tile (its half of N) into its own
+// shared memory; the pair's MMA (issued by rank 0) reads both halves and
+// leaves rows [128r, 128r+128) x all 256 columns of D in rank r's TMEM.  Per
+// SM this feeds 32 KB per 64-wide K step instead of 48 KB.  Both ranks' TMA
+// loads complete on rank 0's stage barrier; rank 0's commits arrive on both
+// ranks' barriers (multicast commit); rank 1's epilogue releases the
+// accumulator on rank 0's barrier.  No TMA load uses multicast.
+constexpr int BM2 = 256;
+constexpr int HALF_STAGE = 128 * KBYTES;  // 16 KB: 128 rows of A or B
+constexpr int STAGES2 = 6;
+constexpr int NUM_BARS2 = 2 * STAGES2 + 5;
+constexpr int SMEM2_BYTES = 1024 + STAGES2 * 2 * HALF_STAGE + NUM_BARS2 * 8 + 16;
+constexpr uint32_t PEER_BIT_CLEAR = 0xFEFFFFFFu;  // shared::cluster address of the same offset in rank 0
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t smem_in_rank(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar_rank0, int x,
+                                                 int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], "
+      "[%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_rank0), "r"(x), "r"(y)
+      : "memory");
+}
+__device__ __forceinline__ void mma2_bf16(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+__device__ __forceinline__ void mma2_i8(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+// arrive (once the issued MMAs complete) on the barrier at this offset in both ranks
+__device__ __forceinline__ void commit2_both(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+                   bar),
+               "h"(static_cast<uint16_t>(3))
+               : "memory");
+}
+__device__ __forceinline__ void commit2_local(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+
+template <bool INT8, int EPI>
+__global__ void __launch_bounds__(THREADS, 1)
+    k_gemm2(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const GemmArgs p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES2 * HALF_STAGE;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES2 * HALF_STAGE);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NUM_BARS2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const bool leader = rank == 0;
+  const int cid = blockIdx.x >> 1, nclusters = gridDim.x >> 1;
+  const uint32_t bar0 = smem_u32(bars);
+  // full[s] (rank 0's are used), empty[s], tmem_full[2], tmem_empty[2] (rank 0's are used), mma_done
+  const uint32_t full0 = bar0, empty0 = bar0 + 8 * STAGES2, tfull0 = bar0 + 16 * STAGES2, tempty0 = tfull0 + 16,
+                 mma_done = tempty0 + 16;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES2; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull0 + 8 * a, 1);
+      mbar_init(tempty0 + 8 * a, 2 * EPI_WARPS);  // epilogue warps of both ranks
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // both ranks' barriers exist before any cross-rank arrival
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int num_m = (p.M + BM2 - 1) / BM2, num_n = (p.N + BN - 1) / BN, num_tiles = num_m * num_n;
+  const int num_units = p.split > 1 ? p.full_tiles + (num_tiles - p.full_tiles) * p.split : num_tiles;
+  constexpr int KE = INT8 ? 128 : 64;
+  const int num_kb = p.K / KE;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0, issued = 0, issued_par = 0;
+      for (int u = cid; u < num_units; u += nclusters) {
+        int t, kb0, kb1, part, mb, nb;
+        unit_range(u, p.full_tiles, p.split, num_kb, t, kb0, kb1, part);
+        tile_coords(t, num_m, num_n, mb, nb);
+        bool ok = true;
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(empty0 + 8 * stage, phase ^ 1, abort_flag, p.err, (EK_GEMM << 8) | 5)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = full0 + 8 * stage;
+          if (leader) mbar_arrive_expect_tx(fb, 4 * HALF_STAGE);  // both ranks' A and B halves
+          tma_load_2d_pair(smem_u32(sA + stage * HALF_STAGE), &tmA, fb & PEER_BIT_CLEAR, kb * KE,
+                           mb * BM2 + 128 * rank);
+          tma_load_2d_pair(smem_u32(sB + stage * HALF_STAGE), &tmB, fb & PEER_BIT_CLEAR, kb * KE,
+                           nb * BN + 128 * rank);
+          issued |= 1u << stage;
+          issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+          if (++stage == STAGES2) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+      }
+      if (leader)  // rank 0's stage barriers count both ranks' bytes
+        for (int s = 0; s < STAGES2; ++s)
+          if ((issued >> s) & 1) mbar_drain(full0 + 8 * s, (issued_par >> s) & 1);
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      constexpr uint32_t idesc = INT8 ? idesc_i8(BM2, BN) : idesc_bf16(BM2, BN, false);
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      for (int u = cid; u < num_units; u += nclusters) {
+        int t, kb0, kb1, part;
+        unit_range(u, p.full_tiles, p.split, num_kb, t, kb0, kb1, part);
+        if (!mbar_wait(tempty0 + 8 * acc, acc_phase ^ 1, abort_flag, p.err, (EK_GEMM << 8) | 6)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        bool ok = true;
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(full0 + 8 * stage, phase, abort_flag, p.err, (EK_GEMM << 8) | 7)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + stage * HALF_STAGE), b0 = smem_u32(sB + stage * HALF_STAGE);
+#pragma unroll
+          for (int k = 0; k < KBYTES / 32; ++k) {
+            const uint64_t ad = desc_sw128_k(a0 + 32 * k), bd = desc_sw128_k(b0 + 32 * k);
+            if (INT8)
+              mma2_i8(d_tmem, ad, bd, idesc, (kb > kb0) || k != 0);
+            else
+              mma2_bf16(d_tmem, ad, bd, idesc, (kb > kb0) || k != 0);
+          }
+          commit2_both(empty0 + 8 * stage);  // frees the stage in both ranks
+          if (++stage == STAGES2) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        commit2_both(tfull0 + 8 * acc);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1;
+      }
+      commit2_local(mma_done);
+      mbar_drain(mma_done, 0);
+    }
+  } else {
+    const int q = warp & 3;
+    const int ch = (warp - 2) >> 2;
+    const uint32_t tempty_rank0 = smem_in_rank(tempty0, 0);
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int u = cid; u < num_units; u += nclusters) {
+      int t, kb0, kb1, part, mb, nb;
+      unit_range(u, p.full_tiles, p.split, num_kb, t, kb0, kb1, part);
+      tile_coords(t, num_m, num_n, mb, nb);
+      const bool ok = mbar_wait(tfull0 + 8 * acc, acc_phase, abort_flag, p.err, (EK_GEMM << 8) | 8);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      const int trow = 128 * rank + q * 32 + lane;  // row inside the 256-row tile
+      const int m = mb * BM2 + trow;
+      float row_amax = 0.f;
+#pragma unroll 1
+      for (int c = ch * (BN / 64); c < (ch + 1) * (BN / 64); ++c) {
+        const int n = nb * BN + c * 32;
+        if (n >= p.N) break;
+        uint32_t r[32];
+        tmem_ld32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN + c * 32, r);
+        tmem_ld_wait();
+        if (EPI == H3B_EPI_RESID && part >= 0) {
+          float4* dst = reinterpret_cast<float4*>(
+              p.partial + (static_cast<size_t>(t - p.full_tiles) * p.split + part) * (BM2 * BN) + trow * BN + c * 32);
+          if (INT8) {
+            float v[32];
+            const float sa = m < p.M ? p.sa[m] : 0.f;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = static_cast<float>(static_cast<int>(r[i])) * sa * __ldg(p.sb + n + i);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              dst[i] = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
+                                   __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
+          }
+        } else if (m < p.M) {
+          epilogue_chunk<INT8, EPI>(p, m, n, r, row_amax);
+        }
+      }
+      if (INT8 && EPI == H3B_EPI_GELU && m < p.M)
+        atomicMax(reinterpret_cast<int*>(p.row_absmax) + m, __float_as_int(row_amax));
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (leader)
+          mbar_arrive(tempty0 + 8 * acc);
+        else
+          mbar_arrive_remote(tempty_rank0 + 8 * acc);
+      }
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // rank 0's MMAs are done and rank 1 no longer touches rank 0's barriers
+  if (warp == 0) {
+    __syncwarp();
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS) : "memory");
+  }
+}
+
 using GemmKernel = void (*)(const CUtensorMap, const CUtensorMap, const GemmArgs);
+
+template <bool INT8>
+GemmKernel pick2(int epi) {
+  switch (epi) {
+    case H3B_EPI_F32: return k_gemm2<INT8, H3B_EPI_F32>;
+    case H3B_EPI_BF16: return k_gemm2<INT8, H3B_EPI_BF16>;
+    case H3B_EPI_QKV_ROPE: return k_gemm2<INT8, H3B_EPI_QKV_ROPE>;
+    case H3B_EPI_RESID: return k_gemm2<INT8, H3B_EPI_RESID>;
+    case H3B_EPI_GELU: return k_gemm2<INT8, H3B_EPI_GELU>;
+    case H3B_EPI_I32: return INT8 ? k_gemm2<INT8, H3B_EPI_I32> : nullptr;
+    default: return nullptr;
+  }
+}
 
 template <bool INT8>
 GemmKernel pick(int epi) {
@@ -363,19 +640,47 @@ GemmKernel pick(int epi) {
 cudaError_t launch_gemm(const Ctx& c, const void* A, const void* B, int ab_int8, int epi, const GemmArgs& args_in,
                         float* scratch, size_t scratch_bytes) {
   GemmArgs args = args_in;
-  GemmKernel kern = ab_int8 ? pick<true>(epi) : pick<false>(epi);
-  if (!kern) return cudaErrorInvalidValue;
   const int eb = ab_int8 ? 1 : 2;
   const CUtensorMapDataType dt = ab_int8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  // CTA pairs (256x256 tiles) when they fill at least one wave of pairs;
+  // single CTAs (128x256 tiles) otherwise, for more parallelism.
+  const int tiles2 = ((args.M + BM2 - 1) / BM2) * ((args.N + BN - 1) / BN);
+  const bool pair = c.num_sms >= 2 && tiles2 >= c.num_sms / 2;
+  const int TM = pair ? BM2 : BM;
+  GemmKernel kern = pair ? (ab_int8 ? pick2<true>(epi) : pick2<false>(epi))
+                         : (ab_int8 ? pick<true>(epi) : pick<false>(epi));
+  if (!kern) return cudaErrorInvalidValue;
   CUtensorMap ta, tb;
-  if (!encode_tmap_2d(&ta, dt, eb, A, args.K, args.M, static_cast<uint64_t>(args.K) * eb, KBYTES / eb, BM) ||
-      !encode_tmap_2d(&tb, dt, eb, B, args.K, args.N, static_cast<uint64_t>(args.K) * eb, KBYTES / eb, BN))
+  if (!encode_tmap_2d(&ta, dt, eb, A, args.K, args.M, static_cast<uint64_t>(args.K) * eb, KBYTES / eb, 128) ||
+      !encode_tmap_2d(&tb, dt, eb, B, args.K, args.N, static_cast<uint64_t>(args.K) * eb, KBYTES / eb,
+                      pair ? 128 : BN))
     return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+  const int smem = pair ? SMEM2_BYTES : SMEM_BYTES;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  const int num_m = (args.M + BM - 1) / BM, num_n = (args.N + BN - 1) / BN;
+  const int num_m = (args.M + TM - 1) / TM, num_n = (args.N + BN - 1) / BN;
   const int tiles = num_m * num_n;
-  const int grid = tiles < c.num_sms ? tiles : c.num_sms;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  int slots = c.num_sms;  // tiles in flight at once
+  if (pair) {
+    cfg.blockDim = dim3(THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = c.stream;
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    // pairs must sit in one GPC: ask how many can be resident at once
+    cfg.gridDim = dim3(c.num_sms);
+    int active = 0;
+    e = cudaOccupancyMaxActiveClusters(&active, kern, &cfg);
+    if (e != cudaSuccess) return e;
+    slots = active > 0 ? active : 1;
+  }
+  const int grid = tiles < slots ? tiles : slots;
   if (grid == 0) return cudaSuccess;
   // Residual GEMMs whose last wave is at most a third full: cut the tail
   // tiles along K over the idle SMs (partials in the caller's scratch).
@@ -387,7 +692,7 @@ cudaError_t launch_gemm(const Ctx& c, const void* A, const void* B, int ab_int8,
   if (epi == H3B_EPI_RESID && scratch && tiles > grid && rem > 0 && 3 * rem <= grid) {
     int split = grid / rem;
     if (split > num_kb / 2) split = num_kb / 2;
-    const size_t per_split = static_cast<size_t>(rem) * BM * BN * sizeof(float);
+    const size_t per_split = static_cast<size_t>(rem) * TM * BN * sizeof(float);
     if (static_cast<size_t>(split) * per_split > scratch_bytes) split = static_cast<int>(scratch_bytes / per_split);
     if (split >= 2) {
       args.split = split;
@@ -395,11 +700,21 @@ cudaError_t launch_gemm(const Ctx& c, const void* A, const void* B, int ab_int8,
       args.partial = scratch;
     }
   }
-  kern<<<grid, THREADS, SMEM_BYTES, c.stream>>>(ta, tb, args);
-  cudaError_t le = cudaGetLastError();
-  if (le != cudaSuccess || args.split <= 1) return le;
-  k_splitk_add<<<rem * BM, BN, 0, c.stream>>>(static_cast<float*>(args.C), args.partial, args.M, args.N,
-                                              args.full_tiles, args.split, num_m, num_n);
+  if (pair) {
+    cfg.gridDim = dim3(2 * grid);
+    e = cudaLaunchKernelEx(&cfg, kern, ta, tb, args);
+    if (e != cudaSuccess) return e;
+  } else {
+    kern<<<grid, THREADS, smem, c.stream>>>(ta, tb, args);
+  }
+  e = cudaGetLastError();
+  if (e != cudaSuccess || args.split <= 1) return e;
+  if (pair)
+    k_splitk_add<BM2><<<rem * BM2, BN, 0, c.stream>>>(static_cast<float*>(args.C), args.partial, args.M, args.N,
+                                                      args.full_tiles, args.split, num_m, num_n);
+  else
+    k_splitk_add<BM><<<rem * BM, BN, 0, c.stream>>>(static_cast<float*>(args.C), args.partial, args.M, args.N,
+                                                    args.full_tiles, args.split, num_m, num_n);
   return cudaGetLastError();
 }
 

@@ -345,3 +345,72 @@ def test_attention_key_split_tail(cuda_dev, S, H, D):
     d = H * D
     ref = oracle.attention(q[rows, :d], q[:, d:2 * d], q[:, 2 * d:], H)
     assert rel_l2(np64(o_split)[rows], ref) < 1e-2
+
+
+# shapes whose 256x256 tiles fill a wave of CTA pairs -> the 2-SM (cta_group::2) kernel
+PAIR_SHAPES = [(2048, 2560, 1024), (2100, 2592, 512), (6528, 3072, 256)]
+
+
+@pytest.mark.parametrize("M,N,K", PAIR_SHAPES)
+def test_gemm_pair_bf16(cuda_dev, M, N, K):
+    A = wlmod.normal_tensor((M, K), 41, cuda_dev, dtype=torch.bfloat16)
+    B = wlmod.normal_tensor((N, K), 42, cuda_dev, 0.02, dtype=torch.bfloat16)
+    C = torch.full((M, N), float("nan"), device=cuda_dev)
+    h3b.gemm(A, B, h3b.EPI_F32, C)
+    torch.cuda.synchronize()
+    assert h3b.device_error() == 0
+    ref = oracle.linear(np64(A), np64(B))
+    assert np.isfinite(C.cpu().numpy()).all()
+    assert rel_l2(C, ref) < 1e-5
+
+
+@pytest.mark.parametrize("M,N,K", PAIR_SHAPES)
+def test_gemm_pair_int8_i32_bitexact(cuda_dev, M, N, K):
+    K = max(K, 128)
+    A = wlmod.int8_tensor((M, K), 43, cuda_dev)
+    B = wlmod.int8_tensor((N, K), 44, cuda_dev)
+    C = torch.zeros((M, N), dtype=torch.int32, device=cuda_dev)
+    h3b.gemm(A, B, h3b.EPI_I32, C)
+    torch.cuda.synchronize()
+    rows = np.unique(np.concatenate([np.arange(0, 8), np.arange(120, 136), np.arange(M - 140, M),
+                                     np.linspace(0, M - 1, 40).astype(int)]))
+    ref = oracle.int8_matmul(A.cpu().numpy()[rows], B.cpu().numpy())
+    assert np.array_equal(C.cpu().numpy()[rows].astype(np.int64), ref)
+
+
+@pytest.mark.parametrize("int8", [False, True])
+def test_gemm_pair_epilogues(cuda_dev, int8):
+    """RoPE, GELU(+row max) and residual epilogues on the pair kernel."""
+    wl = wlmod.Workload("p", 4, 16, 30, 100, 1024, 8, 128, 4096, 1, 0, 0, False)  # S = 2020
+    dm = h3b.dims_of(wl)
+    S, d = h3b.seq_len(dm), wl.d
+    tab = h3b.rope_table(dm)
+    if int8:
+        A, B = wlmod.int8_tensor((S, d), 45, cuda_dev), wlmod.int8_tensor((3 * d, d), 46, cuda_dev)
+        sa = wlmod.uniform_tensor((S,), 47, cuda_dev, 0.001, 0.003)
+        sb = wlmod.uniform_tensor((3 * d,), 48, cuda_dev, 0.001, 0.003)
+        acc = (A.double() @ B.double().T).cpu().numpy() * np64(sa)[:, None] * np64(sb)[None, :]
+    else:
+        A = wlmod.normal_tensor((S, d), 45, cuda_dev, dtype=torch.bfloat16)
+        B = wlmod.normal_tensor((3 * d, d), 46, cuda_dev, 0.05, dtype=torch.bfloat16)
+        sa = sb = None
+        acc = oracle.linear(np64(A), np64(B))
+    C = torch.empty((S, 3 * d), dtype=torch.bfloat16, device=cuda_dev)
+    h3b.gemm(A, B, h3b.EPI_QKV_ROPE, C, scale_a=sa, scale_b=sb, rope=tab, dims=dm)
+    G = torch.empty((S, 3 * d), dtype=torch.bfloat16, device=cuda_dev)
+    amax = torch.zeros(S, device=cuda_dev)
+    h3b.gemm(A, B, h3b.EPI_GELU, G, scale_a=sa, scale_b=sb, row_absmax=amax if int8 else None)
+    X0 = wlmod.normal_tensor((S, 3 * d), 49, cuda_dev)
+    X = X0.clone()
+    h3b.gemm(A, B, h3b.EPI_RESID, X, scale_a=sa, scale_b=sb)
+    torch.cuda.synchronize()
+    assert h3b.device_error() == 0
+    ang = oracle.rope_angles(wl)
+    ref = np.concatenate([oracle.apply_rope(acc[:, :d], ang, 8), oracle.apply_rope(acc[:, d:2 * d], ang, 8),
+                          acc[:, 2 * d:]], axis=1)
+    assert np.all(np.abs(np64(C) - ref) <= 2.0 ** -8 * np.abs(ref) + 2e-5 * np.abs(ref).max())
+    ref_g = oracle.gelu(acc)
+    assert np.all(np.abs(np64(G) - ref_g) <= 2.0 ** -8 * np.abs(ref_g) + 1e-5 * np.abs(acc).max())
+    if int8:
+        assert np.array_equal(amax.cpu().numpy(), G.float().abs().amax(dim=1).cpu().numpy())
+    assert rel_l2(np64(X) - np64(X0), acc) < 1e-5
