@@ -186,6 +186,53 @@ def block_forward(dims: Dims, block: Block, x: torch.Tensor, ws: torch.Tensor, m
     return x
 
 
+class HostPipeline:
+    """Streams token batches that live in host memory through the block (or
+    stack) on the device.  Copy-in of step i+1 and copy-out of step i-1 run on
+    their own CUDA streams while step i computes, with ``depth`` device buffers
+    in rotation; the workspace is used by one compute stream, in order.
+
+    ``submit(x_in, x_out)`` enqueues one step: x_in (pinned host, [S, d] fp32)
+    is copied in, processed, and the result copied to x_out (pinned host).
+    The call returns at once; x_in must stay untouched and x_out is valid only
+    after ``synchronize()`` (or once a later submit has reused its buffer)."""
+
+    def __init__(self, dims: Dims, blocks, ws: torch.Tensor, shape, depth: int = 2, merge_first: int = -1,
+                 merge_last: int = -1):
+        self.dims, self.ws = dims, ws
+        self.blocks = list(blocks) if isinstance(blocks, (list, tuple)) else [blocks]
+        self.mf, self.ml = merge_first, merge_last
+        self.bufs = [torch.empty(shape, dtype=torch.float32, device="cuda") for _ in range(depth)]
+        self.s_in, self.s_run, self.s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+        self.ev_in = [torch.cuda.Event() for _ in range(depth)]
+        self.ev_run = [torch.cuda.Event() for _ in range(depth)]
+        self.ev_out = [torch.cuda.Event() for _ in range(depth)]
+        self.i = 0
+
+    def submit(self, x_in: torch.Tensor, x_out: torch.Tensor):
+        b = self.i % len(self.bufs)
+        buf = self.bufs[b]
+        self.s_in.wait_event(self.ev_out[b])  # the previous copy-out from this buffer is done
+        with torch.cuda.stream(self.s_in):
+            buf.copy_(x_in, non_blocking=True)
+            self.ev_in[b].record(self.s_in)
+        self.s_run.wait_event(self.ev_in[b])
+        with torch.cuda.stream(self.s_run):
+            if len(self.blocks) == 1 and self.mf < 0:
+                block_forward(self.dims, self.blocks[0], buf, self.ws)
+            else:
+                stack_forward(self.dims, self.blocks, buf, self.ws, self.mf, self.ml)
+            self.ev_run[b].record(self.s_run)
+        self.s_out.wait_event(self.ev_run[b])
+        with torch.cuda.stream(self.s_out):
+            x_out.copy_(buf, non_blocking=True)
+            self.ev_out[b].record(self.s_out)
+        self.i += 1
+
+    def synchronize(self):
+        self.s_out.synchronize()
+
+
 def stack_forward(dims: Dims, blocks: Sequence[Block], x: torch.Tensor, ws: torch.Tensor,
                   merge_first: int = -1, merge_last: int = -1) -> torch.Tensor:
     arr = _blocks_array(blocks)
