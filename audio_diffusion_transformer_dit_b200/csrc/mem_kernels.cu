@@ -39,8 +39,15 @@ __device__ __forceinline__ float block_reduce(float v, float* red) {
   return r;
 }
 
-__device__ __forceinline__ int8_t quant1(float v, float s) {
-  float q = s > 0.f ? rintf(v / s) : 0.f;  // IEEE divide, round half to even
+// Code of v for row scale s: rint(v / s) with the IEEE fp32 quotient,
+// half-even, clamped to [-127, 127].  rs = 1/s.  v*rs is within a few ulp of
+// v/s (|v/s| <= 127), so it rounds to the same integer unless the quotient lies
+// within 1e-4 of a half-integer; only then is the exact quotient computed.
+__device__ __forceinline__ int8_t quant1(float v, float s, float rs) {
+  if (!(s > 0.f)) return 0;
+  const float y = v * rs;
+  float q = rintf(y);
+  if (fabsf(fabsf(y - q) - 0.5f) < 1e-4f) q = rintf(v / s);
   q = fminf(fmaxf(q, -127.f), 127.f);
   return static_cast<int8_t>(static_cast<int>(q));
 }
@@ -130,10 +137,13 @@ __global__ void k_rope_table(float2* __restrict__ table, int F, int H, int Wc, i
     } else {
       pos = s - n_video; jl = j; n = D;
     }
-    const double ang = pos * pow(static_cast<double>(theta), -2.0 * jl / n);
-    double sn, cs;
-    sincos(ang, &sn, &cs);
-    table[e] = make_float2(static_cast<float>(cs), static_cast<float>(sn));
+    // fp64 angle, reduced to [-pi, pi] in fp64, then fp32 sin/cos of the remainder
+    const double ang = pos * exp2(-2.0 * jl / n * log2(static_cast<double>(theta)));
+    const double two_pi = 6.283185307179586;
+    const float red = static_cast<float>(fma(-rint(ang / two_pi), two_pi, ang));
+    float sn, cs;
+    sincosf(red, &sn, &cs);
+    table[e] = make_float2(cs, sn);
   }
 }
 
@@ -182,16 +192,16 @@ __global__ void __launch_bounds__(kThreads) k_rmsnorm(const float* __restrict__ 
   }
   if (INT8) {
     amax = block_reduce<true>(amax, red);
-    const float s = amax / 127.0f;
+    const float s = amax / 127.0f, rs = 1.0f / s;
 #pragma unroll
     for (int i = 0; i < VPT; ++i) {
       const int c = threadIdx.x + i * blockDim.x;
       if (c < d4) {
         char4 q;
-        q.x = quant1(v[i].x, s);
-        q.y = quant1(v[i].y, s);
-        q.z = quant1(v[i].z, s);
-        q.w = quant1(v[i].w, s);
+        q.x = quant1(v[i].x, s, rs);
+        q.y = quant1(v[i].y, s, rs);
+        q.z = quant1(v[i].z, s, rs);
+        q.w = quant1(v[i].w, s, rs);
         reinterpret_cast<char4*>(out)[static_cast<size_t>(row) * d4 + c] = q;
       }
     }
@@ -209,12 +219,12 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float (&f)[8]) {
   }
 }
 
-__device__ __forceinline__ uint2 quant8(const float (&f)[8], float s) {
+__device__ __forceinline__ uint2 quant8(const float (&f)[8], float s, float rs) {
   uint32_t lo = 0, hi = 0;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    lo |= (static_cast<uint32_t>(static_cast<uint8_t>(quant1(f[i], s)))) << (8 * i);
-    hi |= (static_cast<uint32_t>(static_cast<uint8_t>(quant1(f[4 + i], s)))) << (8 * i);
+    lo |= (static_cast<uint32_t>(static_cast<uint8_t>(quant1(f[i], s, rs)))) << (8 * i);
+    hi |= (static_cast<uint32_t>(static_cast<uint8_t>(quant1(f[4 + i], s, rs)))) << (8 * i);
   }
   return make_uint2(lo, hi);
 }
@@ -238,7 +248,7 @@ __global__ void __launch_bounds__(kThreads) k_quant_rows(const uint4* __restrict
     for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(f[j]));
   }
   amax = block_reduce<true>(amax, red);
-  const float s = amax / 127.0f;
+  const float s = amax / 127.0f, rs = 1.0f / s;
   uint2* qr = reinterpret_cast<uint2*>(q + static_cast<size_t>(row) * k8 * 8);
 #pragma unroll
   for (int i = 0; i < VPT; ++i) {
@@ -246,7 +256,7 @@ __global__ void __launch_bounds__(kThreads) k_quant_rows(const uint4* __restrict
     if (c < k8) {
       float f[8];
       bf16x8_to_f32(v[i], f);
-      qr[c] = quant8(f, s);
+      qr[c] = quant8(f, s, rs);
     }
   }
   if (threadIdx.x == 0) scale[row] = s;
@@ -257,14 +267,14 @@ __global__ void __launch_bounds__(kThreads) k_quant_rows(const uint4* __restrict
 __global__ void k_quant_absmax(const uint4* __restrict__ a, const float* __restrict__ absmax, int k16,
                                int8_t* __restrict__ q, float* __restrict__ scale) {
   const int row = blockIdx.y;
-  const float s = absmax[row] / 127.0f;
+  const float s = absmax[row] / 127.0f, rs = 1.0f / s;
   const uint4* ar = a + static_cast<size_t>(row) * k16 * 2;
   uint4* qr = reinterpret_cast<uint4*>(q) + static_cast<size_t>(row) * k16;
   for (int c = blockIdx.x * blockDim.x + threadIdx.x; c < k16; c += gridDim.x * blockDim.x) {
     float f0[8], f1[8];
     bf16x8_to_f32(__ldcs(ar + 2 * c), f0);
     bf16x8_to_f32(__ldcs(ar + 2 * c + 1), f1);
-    const uint2 lo = quant8(f0, s), hi = quant8(f1, s);
+    const uint2 lo = quant8(f0, s, rs), hi = quant8(f1, s, rs);
     qr[c] = make_uint4(lo.x, lo.y, hi.x, hi.y);
   }
   if (blockIdx.x == 0 && threadIdx.x == 0) scale[row] = s;
@@ -274,13 +284,13 @@ __global__ void k_quant_absmax(const uint4* __restrict__ a, const float* __restr
 __global__ void k_quant_absmax8(const uint4* __restrict__ a, const float* __restrict__ absmax, int k8,
                                 int8_t* __restrict__ q, float* __restrict__ scale) {
   const int row = blockIdx.y;
-  const float s = absmax[row] / 127.0f;
+  const float s = absmax[row] / 127.0f, rs = 1.0f / s;
   const uint4* ar = a + static_cast<size_t>(row) * k8;
   uint2* qr = reinterpret_cast<uint2*>(q) + static_cast<size_t>(row) * k8;
   for (int c = blockIdx.x * blockDim.x + threadIdx.x; c < k8; c += gridDim.x * blockDim.x) {
     float f[8];
     bf16x8_to_f32(__ldcs(ar + c), f);
-    qr[c] = quant8(f, s);
+    qr[c] = quant8(f, s, rs);
   }
   if (blockIdx.x == 0 && threadIdx.x == 0) scale[row] = s;
 }

@@ -414,3 +414,32 @@ def test_gemm_pair_epilogues(cuda_dev, int8):
     if int8:
         assert np.array_equal(amax.cpu().numpy(), G.float().abs().amax(dim=1).cpu().numpy())
     assert rel_l2(np64(X) - np64(X0), acc) < 1e-5
+
+
+def test_quantize_ties_and_near_ties_bitexact(cuda_dev):
+    """Rows scaled so that v/s is an exact half-integer (round-half-even ties),
+    plus the neighbouring bf16 values on either side, through both row
+    quantisation kernels: codes and scales equal the oracle's bit for bit."""
+    rows = []
+    for k in range(0, 6):                       # s = 2^-k exactly (row max 127 * 2^-k)
+        sc = 2.0 ** -k
+        halves = (np.arange(-127, 127) + 0.5) * sc
+        rows.append(np.concatenate([[127 * sc], halves]))
+    base = np.stack([r[:255] for r in rows]).astype(np.float32)
+    t = torch.tensor(base).to(torch.bfloat16)
+    bits = t.view(torch.int16)
+    nb_up = (bits + 1).view(torch.bfloat16)
+    nb_dn = (bits - 1).view(torch.bfloat16)
+    nb_up[:, 0] = t[:, 0]
+    nb_dn[:, 0] = t[:, 0]
+    w = torch.cat([t, nb_up, nb_dn], dim=0)
+    w = torch.cat([w, torch.zeros((w.shape[0], 1), dtype=torch.bfloat16)], dim=1)  # k = 256
+    w = w.contiguous().to(cuda_dev)
+    q, s = h3b.quantize_weights(w)
+    amax = w.float().abs().amax(dim=1).contiguous()
+    q2, s2 = h3b.quantize_rows_absmax(w, amax)
+    torch.cuda.synchronize()
+    qr, sr = oracle.quantize_rows(w.float().cpu().numpy())
+    assert np.array_equal(s.cpu().numpy(), sr) and np.array_equal(q.cpu().numpy(), qr)
+    assert np.array_equal(s2.cpu().numpy(), sr) and np.array_equal(q2.cpu().numpy(), qr)
+    assert set(np.abs(qr[0, 1:255]).tolist()) >= {0, 2, 126}  # half-even ties really occurred
