@@ -42,6 +42,7 @@ __all__ = [
     "attention", "block_forward", "stack_forward", "token_merge", "token_unmerge",
     "quantize_rows", "dequantize_rows", "int8_matmul", "dequant_weights", "block_forward_w8a8",
     "sigmas", "is_fresh", "fresh_steps", "flow_step", "denoise",
+    "token_unmerge_delta", "stack_forward_ex", "denoise_core",
 ]
 
 # Readings taken where the pages (and the workload specification) leave a step open.
@@ -63,6 +64,12 @@ READINGS = {
     "velocity": "the velocity is the stack output (no in/out projection is stated)",
     "euler": "x <- x + (sigma_{i+1} - sigma_i) * v over all S tokens at width d",
     "residual": "fp32 residual stream in every configuration",
+    "unmerge_delta": "alternative unmerge: the pre-merge tokens plus the merged blocks' update broadcast to "
+                     "both columns, x_pre + (y - m); audio rows take y",
+    "core_reuse": "core residual reuse (exclusive with whole-velocity reuse): every step evaluates the stack, "
+                  "but the core blocks run only on fresh-core steps (i % r == 0 or the last step); their update "
+                  "(output - input of the core) is cached and added on the other steps",
+    "layers": "--layers L: the stack is given the active blocks (the first L of the model in the workloads)",
 }
 
 # What pins each function to something other than itself (tests/test_oracle_*.py).
@@ -80,6 +87,10 @@ PINS = {
     "int8_matmul": "pure-Python integer dot products",
     "sigmas/fresh/denoise": "fresh counts 20/11/8 at 20 steps (control table); v = 0 identity; "
                             "single-step closed form",
+    "token_unmerge_delta": "explicit (f, r, c) loops; equals plain unmerge when x_pre is pair-constant; "
+                           "identity when the merged blocks change nothing",
+    "denoise_core": "core_reuse = 1 equals the plain loop; a core that adds a constant gives the closed form; "
+                    "hand-computed 3-step case",
 }
 
 
@@ -236,6 +247,73 @@ def token_unmerge(xm, dims):
     vid = xm[:V // 2].reshape(F, H, W // 2, -1)
     full = np.repeat(vid, 2, axis=2)
     return np.concatenate([full.reshape(V, -1), xm[V // 2:V // 2 + A]], axis=0)
+
+
+def token_unmerge_delta(x_pre, ym, xm0, dims):
+    """Delta-broadcast unmerge: full token (f, r, c) = x_pre(f, r, c) +
+    (ym - xm0)(f, r, c // 2), where xm0 is the merged sequence that entered
+    the merged blocks and ym what they returned; audio rows take ym."""
+    x_pre, ym, xm0 = _f64(x_pre), _f64(ym), _f64(xm0)
+    F, H, W, A = dims.frames, dims.rows, dims.cols, dims.n_audio
+    V = F * H * W
+    dv = (ym[:V // 2] - xm0[:V // 2]).reshape(F, H, W // 2, -1)
+    full = x_pre[:V].reshape(F, H, W, -1) + np.repeat(dv, 2, axis=2)
+    return np.concatenate([full.reshape(V, -1), ym[V // 2:V // 2 + A]], axis=0)
+
+
+def stack_forward_ex(x, blocks, dims, merge_first=-1, merge_last=-1, unmerge_delta=False, block_fn=None):
+    """stack_forward with the choice of unmerge: plain broadcast, or the
+    delta-broadcast form (pre-merge tokens plus the merged blocks' update)."""
+    if not unmerge_delta:
+        return stack_forward(x, blocks, dims, merge_first, merge_last, block_fn)
+    fn = block_forward if block_fn is None else block_fn
+    x = _f64(x)
+    x_pre = xm0 = None
+    for layer, w in enumerate(blocks):
+        if layer == merge_first:
+            x_pre = x
+            xm0 = token_merge(x, dims)
+            x = xm0
+        x = fn(x, w, dims, merged=merge_first >= 0 and merge_first <= layer <= merge_last)
+        if layer == merge_last and merge_first >= 0:
+            x = token_unmerge_delta(x_pre, x, xm0, dims)
+    return x
+
+
+def denoise_core(x0, blocks, dims, n_steps, core_reuse, core_first, core_last, merge_first=-1, merge_last=-1,
+                 unmerge_delta=False, block_fn=None):
+    """Flow-matching loop with core residual reuse: every step evaluates the
+    stack; the core blocks [core_first, core_last] (with the token-reduction
+    window, which lies inside the core or outside it) run only on fresh-core
+    steps (i % core_reuse == 0 or the last step), where their update
+    delta = core(v) - v is cached; other steps add the cached delta instead.
+    Returns (x_N, number of fresh-core steps)."""
+    inside = merge_first >= 0 and core_first <= merge_first and merge_last <= core_last
+    if not (inside or merge_first < 0 or merge_last < core_first or merge_first > core_last):
+        raise ValueError("the token-reduction window must lie inside the core window or outside it")
+    sig = sigmas(n_steps)
+    x = _f64(x0)
+    delta = None
+    n_core = 0
+
+    def part(v, lo, hi):  # blocks lo..hi with the merge window re-based if it lies in them
+        if lo > hi:
+            return v
+        mf, ml = (merge_first - lo, merge_last - lo) if merge_first >= 0 and lo <= merge_first <= hi else (-1, -1)
+        return stack_forward_ex(v, blocks[lo:hi + 1], dims, mf, ml, unmerge_delta, block_fn)
+
+    for i in range(n_steps):
+        v = part(x, 0, core_first - 1)
+        if is_fresh(i, n_steps, core_reuse):
+            out = part(v, core_first, core_last)
+            delta = out - v
+            v = out
+            n_core += 1
+        else:
+            v = v + delta
+        v = part(v, core_last + 1, len(blocks) - 1)
+        x = flow_step(x, v, sig[i], sig[i + 1])
+    return x, n_core
 
 
 def stack_forward(x, blocks, dims, merge_first=-1, merge_last=-1, block_fn=None):

@@ -421,3 +421,52 @@ def test_stack_merge_window():
     out = oracle.stack_forward(x, [None] * 6, dm, 2, 3, block_fn=fn)
     assert seen == [(19, False), (19, False), (11, True), (11, True), (19, False), (19, False)]
     assert np.allclose(out, oracle.token_unmerge(oracle.token_merge(x, dm), dm))
+
+
+# ----------------------------------------------------------------------------- next rows: delta unmerge, core reuse
+def test_unmerge_delta_explicit_and_special_cases():
+    F, H, W, A, d = 2, 3, 4, 2, 5
+    dm = dims_of(F, H, W, A, 8, 1, 8)
+    rng = np.random.default_rng(20)
+    x_pre = rng.normal(size=(F * H * W + A, d))
+    xm0 = oracle.token_merge(x_pre, dm)
+    ym = xm0 + rng.normal(size=xm0.shape)
+    out = oracle.token_unmerge_delta(x_pre, ym, xm0, dm)
+    for f in range(F):
+        for r in range(H):
+            for c in range(W):
+                i = (f * H + r) * W + c
+                j = (f * H + r) * (W // 2) + c // 2
+                assert np.allclose(out[i], x_pre[i] + ym[j] - xm0[j], rtol=0, atol=1e-14)
+    assert np.array_equal(out[F * H * W:], ym[F * H * W // 2:])
+    assert np.allclose(oracle.token_unmerge_delta(x_pre, xm0, xm0, dm)[:F * H * W], x_pre[:F * H * W])
+    pc = oracle.token_unmerge(rng.normal(size=xm0.shape), dm)          # pair-constant pre-merge tokens
+    pm = oracle.token_merge(pc, dm)
+    assert np.allclose(oracle.token_unmerge_delta(pc, ym, pm, dm), oracle.token_unmerge(ym, dm), atol=1e-13)
+
+
+def test_denoise_core_reuse_one_is_plain_loop():
+    dm = dims_of(1, 1, 2, 1, 4, 1, 4)
+    x0 = np.random.default_rng(21).normal(size=(3, 4))
+    fn = lambda x, w, d, merged: np.tanh(x * w)  # noqa: E731
+    ws = [0.9, 1.1, 0.7, 1.3]
+    a, na = oracle.denoise(x0, ws, dm, 6, 1, block_fn=fn)
+    b, nb = oracle.denoise_core(x0, ws, dm, 6, 1, 1, 2, block_fn=fn)
+    assert na == nb == 6 and np.allclose(a, b, rtol=1e-14)
+
+
+def test_denoise_core_hand_computed():
+    """pre x a, core x b, post x c; 3 steps, core reuse 2 -> core fresh at 0 and 2."""
+    dm = dims_of(1, 1, 2, 1, 4, 1, 4)
+    x0 = np.random.default_rng(22).normal(size=(3, 4))
+    a, b, c = 0.8, 1.25, 0.6
+    fn = lambda x, w, d, merged: x * w  # noqa: E731
+    got, nc = oracle.denoise_core(x0, [a, b, c], dm, 3, 2, 1, 1, block_fn=fn)
+    s = oracle.sigmas(3).astype(np.float64)
+    delta = (b - 1) * a * x0
+    x1 = x0 + (s[1] - s[0]) * c * b * a * x0
+    x2 = x1 + (s[2] - s[1]) * c * (a * x1 + delta)
+    x3 = x2 + (s[3] - s[2]) * c * b * a * x2
+    assert nc == 2 and np.allclose(got, x3, rtol=1e-14)
+    with pytest.raises(ValueError):
+        oracle.denoise_core(x0, [a, b, c], dm, 3, 2, 1, 1, merge_first=0, merge_last=1, block_fn=fn)
