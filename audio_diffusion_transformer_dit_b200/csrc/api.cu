@@ -67,7 +67,8 @@ struct Trace {
 
 const char* kKernelNames[KID_COUNT] = {"flow_step", "token_merge", "token_unmerge", "rope_table", "rmsnorm",
                                        "quant_rows", "quant_absmax", "gemm_qkv_rope", "gemm_o_resid",
-                                       "gemm_fc1_gelu", "gemm_fc2_resid", "gemm", "attention", "memset"};
+                                       "gemm_fc1_gelu", "gemm_fc2_resid", "gemm", "attention", "memset",
+                                       "token_unmerge_delta", "copy"};
 
 struct TraceScope {
   TraceRec* rec = nullptr;
@@ -115,10 +116,11 @@ struct Plan {
   size_t arena, naive;                // arena bytes, bytes without aliasing
   size_t s_act, s_g, amax;            // fp32 [S] scale / max vectors (INT8)
   size_t rope, rope_m, xm;            // RoPE tables, merged-sequence buffer
+  size_t xm0, delta;                  // merged input (delta unmerge), cached core update
   size_t total;
 };
 
-Plan plan(const h3b_dims& dm, int dtype, int reduction) {
+Plan plan(const h3b_dims& dm, int dtype, int reduction, int keep_merged_input = 0, int core = 0) {
   Plan p{};
   const size_t S = seq_len(dm, 0), d = dm.d, f = dm.ffn;
   if (dtype == H3B_INT8) {
@@ -162,6 +164,15 @@ Plan plan(const h3b_dims& dm, int dtype, int reduction) {
     off += al256(Sm * d * 4);
   } else {
     p.rope_m = p.xm = 0;
+  }
+  p.xm0 = p.delta = 0;
+  if (reduction && keep_merged_input) {
+    p.xm0 = off;
+    off += al256(static_cast<size_t>(seq_len(dm, 1)) * d * 4);
+  }
+  if (core) {
+    p.delta = off;
+    off += al256(S * d * 4);
   }
   p.total = off;
   return p;
@@ -267,26 +278,45 @@ int block_impl(const Ctx& c, const h3b_dims& dm, const h3b_block_weights& w, flo
   return H3B_OK;
 }
 
-int stack_impl(const Ctx& c, const h3b_dims& dm, const h3b_block_weights* blocks, int n_blocks, int mf, int ml,
-               float* x, uint8_t* ws, const Plan& p) {
-  const int on = mf >= 0;
+int fill_rope(const Ctx& c, const h3b_dims& dm, uint8_t* ws, const Plan& p, int reduction) {
+  H3B_CU(KID_ROPE_TABLE, launch_rope_table(c, dm, 0, reinterpret_cast<float*>(ws + p.rope)));
+  if (reduction) H3B_CU(KID_ROPE_TABLE, launch_rope_table(c, dm, 1, reinterpret_cast<float*>(ws + p.rope_m)));
+  return H3B_OK;
+}
+
+// Blocks lo..hi on x; the token-reduction window [mf, ml] is applied when it
+// lies inside [lo, hi] (merge before mf, unmerge after ml; udelta selects the
+// delta-broadcast unmerge).  RoPE tables must be filled.
+int run_blocks(const Ctx& c, const h3b_dims& dm, const h3b_block_weights* blocks, int lo, int hi, int mf, int ml,
+               int udelta, float* x, uint8_t* ws, const Plan& p) {
+  const bool on = mf >= 0 && lo <= mf && ml <= hi;
   float* rope = reinterpret_cast<float*>(ws + p.rope);
   float* rope_m = on ? reinterpret_cast<float*>(ws + p.rope_m) : nullptr;
   float* xm = on ? reinterpret_cast<float*>(ws + p.xm) : nullptr;
-  H3B_CU(KID_ROPE_TABLE, launch_rope_table(c, dm, 0, rope));
-  if (on) H3B_CU(KID_ROPE_TABLE, launch_rope_table(c, dm, 1, rope_m));
+  float* xm0 = on && udelta ? reinterpret_cast<float*>(ws + p.xm0) : nullptr;
   const int V = dm.frames * dm.rows * dm.cols;
-  for (int l = 0; l < n_blocks; ++l) {
-    if (on && l == mf) H3B_CU(KID_MERGE, launch_merge(c, x, xm, V, dm.n_audio, dm.d));
+  for (int l = lo; l <= hi; ++l) {
+    if (on && l == mf) H3B_CU(KID_MERGE, launch_merge(c, x, xm, V, dm.n_audio, dm.d, xm0));
     const bool merged = on && l >= mf && l <= ml;
     H3B_TRY(block_impl(c, dm, blocks[l], merged ? xm : x, merged, ws, p, merged ? rope_m : rope));
-    if (on && l == ml) H3B_CU(KID_UNMERGE, launch_unmerge(c, xm, x, V, dm.n_audio, dm.d));
+    if (on && l == ml) {
+      if (udelta)
+        H3B_CU(KID_UNMERGE_DELTA, launch_unmerge_delta(c, x, xm, xm0, V, dm.n_audio, dm.d));
+      else
+        H3B_CU(KID_UNMERGE, launch_unmerge(c, xm, x, V, dm.n_audio, dm.d));
+    }
   }
   return H3B_OK;
 }
 
+int stack_impl(const Ctx& c, const h3b_dims& dm, const h3b_block_weights* blocks, int n_blocks, int mf, int ml,
+               float* x, uint8_t* ws, const Plan& p, int udelta = 0) {
+  H3B_TRY(fill_rope(c, dm, ws, p, mf >= 0));
+  return run_blocks(c, dm, blocks, 0, n_blocks - 1, mf, ml, udelta, x, ws, p);
+}
+
 int check_stack_args(const h3b_dims* dims, const h3b_block_weights* blocks, int n_blocks, int mf, int ml, float* x,
-                     void* ws, size_t ws_bytes, Plan* out) {
+                     void* ws, size_t ws_bytes, Plan* out, int udelta = 0, int cf = -1, int cl = -1) {
   H3B_TRY(check_dims(dims));
   if (!blocks || !x || !ws) return H3B_ERR_NULL;
   if (!aligned16(x) || !aligned16(ws)) return H3B_ERR_ALIGN;
@@ -297,8 +327,54 @@ int check_stack_args(const h3b_dims* dims, const h3b_block_weights* blocks, int 
   const int dtype = n_blocks > 0 ? blocks[0].dtype : H3B_BF16;
   if (dtype != H3B_BF16 && dtype != H3B_INT8) return H3B_ERR_DTYPE;
   for (int l = 0; l < n_blocks; ++l) H3B_TRY(check_weights(&blocks[l], dtype));
-  *out = plan(*dims, dtype, mf >= 0);
+  if (cf >= 0) {
+    if (cl < cf || cl >= n_blocks) return H3B_ERR_DIMS;
+    // the reduction window lies inside the core window or outside it
+    if (mf >= 0 && !(cf <= mf && ml <= cl) && !(ml < cf || mf > cl)) return H3B_ERR_DIMS;
+  }
+  *out = plan(*dims, dtype, mf >= 0, mf >= 0 && udelta, cf >= 0);
   if (ws_bytes < out->total) return H3B_ERR_WORKSPACE;
+  return H3B_OK;
+}
+
+// Flow-matching loop.  Whole-velocity reuse: the stack runs on steps with
+// i % reuse == 0 or the last one.  Core reuse (cf >= 0, reuse == 1): the core
+// blocks run on steps with i % core_reuse == 0 or the last one; their update
+// is cached (as its negative, in ws at p.delta) and added on the other steps.
+int denoise_impl(const Ctx& c, const h3b_dims& dm, const h3b_block_weights* blocks, int n_blocks, int mf, int ml,
+                 int udelta, int cf, int cl, int n_steps, int reuse, int core_reuse, float* x, float* v, uint8_t* ws,
+                 const Plan& p, int* n_fresh, int* n_core) {
+  const size_t n = static_cast<size_t>(seq_len(dm, 0)) * dm.d;
+  auto fresh = [&](int i, int r) { return i % r == 0 || i == n_steps - 1; };
+  float* neg_delta = cf >= 0 ? reinterpret_cast<float*>(ws + p.delta) : nullptr;
+  int count = 0, core_count = 0;
+  H3B_TRY(fill_rope(c, dm, ws, p, mf >= 0));
+  H3B_CU(KID_COPY, cudaMemcpyAsync(v, x, n * sizeof(float), cudaMemcpyDeviceToDevice, c.stream));
+  for (int i = 0; i < n_steps; ++i) {
+    if (fresh(i, reuse)) {
+      if (cf < 0) {
+        H3B_TRY(run_blocks(c, dm, blocks, 0, n_blocks - 1, mf, ml, udelta, v, ws, p));
+      } else {
+        H3B_TRY(run_blocks(c, dm, blocks, 0, cf - 1, mf, ml, udelta, v, ws, p));
+        if (fresh(i, core_reuse)) {
+          H3B_CU(KID_COPY, cudaMemcpyAsync(neg_delta, v, n * sizeof(float), cudaMemcpyDeviceToDevice, c.stream));
+          H3B_TRY(run_blocks(c, dm, blocks, cf, cl, mf, ml, udelta, v, ws, p));
+          H3B_CU(KID_FLOW, launch_flow_step(c, neg_delta, v, -1.0f, n, nullptr));  // input - output
+          ++core_count;
+        } else {
+          H3B_CU(KID_FLOW, launch_flow_step(c, v, neg_delta, -1.0f, n, nullptr));  // + cached update
+        }
+        H3B_TRY(run_blocks(c, dm, blocks, cl + 1, n_blocks - 1, mf, ml, udelta, v, ws, p));
+      }
+      ++count;
+    }
+    const float s0 = static_cast<float>(1.0 - static_cast<double>(i) / n_steps);
+    const float s1 = static_cast<float>(1.0 - static_cast<double>(i + 1) / n_steps);
+    const bool next_fresh = i + 1 < n_steps && fresh(i + 1, reuse);
+    H3B_CU(KID_FLOW, launch_flow_step(c, x, v, s1 - s0, n, next_fresh ? v : nullptr));
+  }
+  if (n_fresh) *n_fresh = count;
+  if (n_core) *n_core = core_count;
   return H3B_OK;
 }
 
@@ -409,22 +485,45 @@ int h3b_denoise(const h3b_dims* dims, const h3b_block_weights* blocks, int n_blo
   if (n_steps <= 0 || reuse <= 0) return H3B_ERR_DIMS;
   Ctx c;
   H3B_TRY(device_ctx(static_cast<cudaStream_t>(stream), &c));
-  const size_t n = static_cast<size_t>(seq_len(*dims, 0)) * dims->d;
-  auto fresh = [&](int i) { return i % reuse == 0 || i == n_steps - 1; };
-  int count = 0;
-  H3B_CU(KID_MEMSET, cudaMemcpyAsync(v, x, n * sizeof(float), cudaMemcpyDeviceToDevice, c.stream));
-  for (int i = 0; i < n_steps; ++i) {
-    if (fresh(i)) {
-      H3B_TRY(stack_impl(c, *dims, blocks, n_blocks, merge_first, merge_last, v, static_cast<uint8_t*>(ws), p));
-      ++count;
-    }
-    const float s0 = static_cast<float>(1.0 - static_cast<double>(i) / n_steps);
-    const float s1 = static_cast<float>(1.0 - static_cast<double>(i + 1) / n_steps);
-    const bool next_fresh = i + 1 < n_steps && fresh(i + 1);
-    H3B_CU(KID_FLOW, launch_flow_step(c, x, v, s1 - s0, n, next_fresh ? v : nullptr));
-  }
-  if (n_fresh) *n_fresh = count;
-  return H3B_OK;
+  return denoise_impl(c, *dims, blocks, n_blocks, merge_first, merge_last, 0, -1, -1, n_steps, reuse, 1, x, v,
+                      static_cast<uint8_t*>(ws), p, n_fresh, nullptr);
+}
+
+size_t h3b_workspace_bytes_ex(const h3b_dims* dims, int dtype, const h3b_stack_opts* o) {
+  if (!o || check_dims(dims) != H3B_OK || (dtype != H3B_BF16 && dtype != H3B_INT8)) return 0;
+  const int red = o->merge_first >= 0;
+  if (red && (dims->cols & 1)) return 0;
+  return plan(*dims, dtype, red, red && o->unmerge_delta, o->core_first >= 0).total;
+}
+
+int h3b_stack_forward_ex(const h3b_dims* dims, const h3b_block_weights* blocks, int n_blocks,
+                         const h3b_stack_opts* o, float* x, void* ws, size_t ws_bytes, void* stream) {
+  if (!o) return H3B_ERR_NULL;
+  Plan p;
+  H3B_TRY(check_stack_args(dims, blocks, n_blocks, o->merge_first, o->merge_last, x, ws, ws_bytes, &p,
+                           o->unmerge_delta));
+  Ctx c;
+  H3B_TRY(device_ctx(static_cast<cudaStream_t>(stream), &c));
+  return stack_impl(c, *dims, blocks, n_blocks, o->merge_first, o->merge_last, x, static_cast<uint8_t*>(ws), p,
+                    o->unmerge_delta);
+}
+
+int h3b_denoise_ex(const h3b_dims* dims, const h3b_block_weights* blocks, int n_blocks, const h3b_stack_opts* o,
+                   int n_steps, int reuse, int core_reuse, float* x, float* v, void* ws, size_t ws_bytes,
+                   int* n_fresh, int* n_core_fresh, void* stream) {
+  if (!o) return H3B_ERR_NULL;
+  Plan p;
+  H3B_TRY(check_stack_args(dims, blocks, n_blocks, o->merge_first, o->merge_last, x, ws, ws_bytes, &p,
+                           o->unmerge_delta, o->core_first, o->core_last));
+  if (!v) return H3B_ERR_NULL;
+  if (!aligned16(v)) return H3B_ERR_ALIGN;
+  if (n_steps <= 0 || reuse <= 0 || core_reuse <= 0) return H3B_ERR_DIMS;
+  if (o->core_first >= 0 && reuse != 1) return H3B_ERR_DIMS;  // core reuse excludes whole-velocity reuse
+  Ctx c;
+  H3B_TRY(device_ctx(static_cast<cudaStream_t>(stream), &c));
+  return denoise_impl(c, *dims, blocks, n_blocks, o->merge_first, o->merge_last, o->unmerge_delta, o->core_first,
+                      o->core_last, n_steps, reuse, core_reuse, x, v, static_cast<uint8_t*>(ws), p, n_fresh,
+                      n_core_fresh);
 }
 
 int h3b_quantize_weights(const void* w, int rows, int k, int8_t* q, float* scale, void* stream) {

@@ -26,6 +26,8 @@ enum KernelId {
   KID_GEMM,
   KID_ATTN,
   KID_MEMSET,
+  KID_UNMERGE_DELTA,
+  KID_COPY,
   KID_COUNT
 };
 
@@ -37,7 +39,10 @@ struct Ctx {
 
 // returns cudaError_t of the launch
 cudaError_t launch_flow_step(const Ctx& c, float* x, const float* v, float dt, size_t n, float* x_copy);
-cudaError_t launch_merge(const Ctx& c, const float* x, float* xm, int n_video, int n_audio, int d);
+cudaError_t launch_merge(const Ctx& c, const float* x, float* xm, int n_video, int n_audio, int d,
+                         float* xm_copy = nullptr);
+cudaError_t launch_unmerge_delta(const Ctx& c, float* x, const float* ym, const float* xm0, int n_video, int n_audio,
+                                 int d);
 cudaError_t launch_unmerge(const Ctx& c, const float* xm, float* x, int n_video, int n_audio, int d);
 cudaError_t launch_rope_table(const Ctx& c, const h3b_dims& dm, int merged, float* table);
 cudaError_t launch_rmsnorm(const Ctx& c, const float* x, const float* g, int rows, int d, float eps, void* out,

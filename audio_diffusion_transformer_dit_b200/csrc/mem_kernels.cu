@@ -80,7 +80,8 @@ __global__ void k_flow(float* __restrict__ x, const float* __restrict__ v, float
 // ------------------------------------------------------------------ token reduction
 // Video token (f, r, 2c'+k) is row 2*((f*H + r)*(W/2) + c') + k of the full
 // sequence, so merged row i averages full rows 2i and 2i+1; audio rows follow.
-__global__ void k_merge(const float4* __restrict__ x, float4* __restrict__ xm, int half_video, int n_audio, int d4) {
+__global__ void k_merge(const float4* __restrict__ x, float4* __restrict__ xm, float4* __restrict__ xm_copy,
+                        int half_video, int n_audio, int d4) {
   const size_t total = static_cast<size_t>(half_video + n_audio) * d4;
   const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
   for (size_t e = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < total; e += stride) {
@@ -97,6 +98,7 @@ __global__ void k_merge(const float4* __restrict__ x, float4* __restrict__ xm, i
       o = __ldcs(x + (row + half_video) * d4 + col);  // audio: full row = V + a = merged row + V/2
     }
     xm[e] = o;
+    if (xm_copy) xm_copy[e] = o;
   }
 }
 
@@ -108,6 +110,30 @@ __global__ void k_unmerge(const float4* __restrict__ xm, float4* __restrict__ x,
     const size_t row = e / d4, col = e - row * d4;
     const size_t src = row < static_cast<size_t>(n_video) ? row / 2 : row - half;
     x[e] = xm[src * d4 + col];
+  }
+}
+
+// Delta-broadcast unmerge: full video row r gains ym[r/2] - xm0[r/2] (the
+// merged blocks' update); audio rows take ym.
+__global__ void k_unmerge_delta(float4* __restrict__ x, const float4* __restrict__ ym,
+                                const float4* __restrict__ xm0, int n_video, int n_audio, int d4) {
+  const size_t total = static_cast<size_t>(n_video + n_audio) * d4;
+  const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
+  const int half = n_video / 2;
+  for (size_t e = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < total; e += stride) {
+    const size_t row = e / d4, col = e - row * d4;
+    if (row < static_cast<size_t>(n_video)) {
+      const size_t src = (row / 2) * d4 + col;
+      const float4 y = ym[src], m = xm0[src];
+      float4 v = x[e];
+      v.x += y.x - m.x;
+      v.y += y.y - m.y;
+      v.z += y.z - m.z;
+      v.w += y.w - m.w;
+      x[e] = v;
+    } else {
+      x[e] = ym[(row - half) * d4 + col];
+    }
   }
 }
 
@@ -325,13 +351,24 @@ cudaError_t launch_flow_step(const Ctx& c, float* x, const float* v, float dt, s
   return cudaGetLastError();
 }
 
-cudaError_t launch_merge(const Ctx& c, const float* x, float* xm, int n_video, int n_audio, int d) {
+cudaError_t launch_merge(const Ctx& c, const float* x, float* xm, int n_video, int n_audio, int d, float* xm_copy) {
   const int d4 = d / 4;
   const size_t total = static_cast<size_t>(n_video / 2 + n_audio) * d4;
   if (total == 0) return cudaSuccess;
-  k_merge<<<grid_for(total, c.num_sms), kThreads, 0, c.stream>>>(reinterpret_cast<const float4*>(x),
-                                                                  reinterpret_cast<float4*>(xm), n_video / 2,
-                                                                  n_audio, d4);
+  k_merge<<<grid_for(total, c.num_sms), kThreads, 0, c.stream>>>(
+      reinterpret_cast<const float4*>(x), reinterpret_cast<float4*>(xm), reinterpret_cast<float4*>(xm_copy),
+      n_video / 2, n_audio, d4);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_unmerge_delta(const Ctx& c, float* x, const float* ym, const float* xm0, int n_video, int n_audio,
+                                 int d) {
+  const int d4 = d / 4;
+  const size_t total = static_cast<size_t>(n_video + n_audio) * d4;
+  if (total == 0) return cudaSuccess;
+  k_unmerge_delta<<<grid_for(total, c.num_sms), kThreads, 0, c.stream>>>(
+      reinterpret_cast<float4*>(x), reinterpret_cast<const float4*>(ym), reinterpret_cast<const float4*>(xm0),
+      n_video, n_audio, d4);
   return cudaGetLastError();
 }
 

@@ -39,6 +39,11 @@ class BlockWeights(ctypes.Structure):
                 ("s_o", _p), ("s_fc1", _p), ("s_fc2", _p), ("g_attn", _p), ("g_mlp", _p)]
 
 
+class StackOpts(ctypes.Structure):
+    _fields_ = [("merge_first", _i), ("merge_last", _i), ("unmerge_delta", _i), ("core_first", _i),
+                ("core_last", _i)]
+
+
 _SIGS = {
     "h3b_status_string": (ctypes.c_char_p, [_i]),
     "h3b_seq_len": (_i, [ctypes.POINTER(Dims), _i]),
@@ -48,6 +53,11 @@ _SIGS = {
     "h3b_stack_forward": (_i, [ctypes.POINTER(Dims), ctypes.POINTER(BlockWeights), _i, _i, _i, _p, _p, _sz, _p]),
     "h3b_denoise": (_i, [ctypes.POINTER(Dims), ctypes.POINTER(BlockWeights), _i, _i, _i, _i, _i, _p, _p, _p, _sz,
                          ctypes.POINTER(_i), _p]),
+    "h3b_workspace_bytes_ex": (_sz, [ctypes.POINTER(Dims), _i, ctypes.POINTER(StackOpts)]),
+    "h3b_stack_forward_ex": (_i, [ctypes.POINTER(Dims), ctypes.POINTER(BlockWeights), _i, ctypes.POINTER(StackOpts),
+                                  _p, _p, _sz, _p]),
+    "h3b_denoise_ex": (_i, [ctypes.POINTER(Dims), ctypes.POINTER(BlockWeights), _i, ctypes.POINTER(StackOpts), _i, _i,
+                            _i, _p, _p, _p, _sz, ctypes.POINTER(_i), ctypes.POINTER(_i), _p]),
     "h3b_quantize_weights": (_i, [_p, _i, _i, _p, _p, _p]),
     "h3b_token_merge": (_i, [ctypes.POINTER(Dims), _p, _p, _p]),
     "h3b_token_unmerge": (_i, [ctypes.POINTER(Dims), _p, _p, _p]),
@@ -250,6 +260,38 @@ def denoise(dims: Dims, blocks: Sequence[Block], x: torch.Tensor, v: torch.Tenso
                            _ptr(x, torch.float32, "x"), _ptr(v, torch.float32, "v"), _ptr(ws, None, "ws"),
                            ws.numel(), ctypes.byref(nf), _stream()), "h3b_denoise")
     return nf.value
+
+
+def stack_opts(merge_first: int = -1, merge_last: int = -1, unmerge_delta: bool = False, core_first: int = -1,
+               core_last: int = -1) -> StackOpts:
+    return StackOpts(merge_first, merge_last, int(unmerge_delta), core_first, core_last)
+
+
+def workspace_ex(dims: Dims, opts: StackOpts, dtype: int = BF16, device="cuda") -> torch.Tensor:
+    n = lib.h3b_workspace_bytes_ex(ctypes.byref(dims), dtype, ctypes.byref(opts))
+    if n == 0:
+        raise ValueError("invalid dims / options for workspace")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def stack_forward_ex(dims: Dims, blocks: Sequence[Block], x: torch.Tensor, ws: torch.Tensor,
+                     opts: StackOpts) -> torch.Tensor:
+    arr = _blocks_array(blocks)
+    _check(lib.h3b_stack_forward_ex(ctypes.byref(dims), arr, len(blocks), ctypes.byref(opts),
+                                    _ptr(x, torch.float32, "x"), _ptr(ws, None, "ws"), ws.numel(), _stream()),
+           "h3b_stack_forward_ex")
+    return x
+
+
+def denoise_ex(dims: Dims, blocks: Sequence[Block], x: torch.Tensor, v: torch.Tensor, ws: torch.Tensor, n_steps: int,
+               opts: StackOpts, reuse: int = 1, core_reuse: int = 1):
+    """Returns (stack evaluations, core evaluations)."""
+    arr = _blocks_array(blocks)
+    nf, nc = ctypes.c_int(0), ctypes.c_int(0)
+    _check(lib.h3b_denoise_ex(ctypes.byref(dims), arr, len(blocks), ctypes.byref(opts), n_steps, reuse, core_reuse,
+                              _ptr(x, torch.float32, "x"), _ptr(v, torch.float32, "v"), _ptr(ws, None, "ws"),
+                              ws.numel(), ctypes.byref(nf), ctypes.byref(nc), _stream()), "h3b_denoise_ex")
+    return nf.value, nc.value
 
 
 def quantize_weights(w: torch.Tensor):

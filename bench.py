@@ -216,8 +216,22 @@ def run_ours(args, wl):
     dm, blocks, x, ws = build_workload(wl, dev)
     loop = wl.steps > 0
     v = torch.empty_like(x) if loop else None
+    core = loop and args.core_reuse > 0
+    n_core = 0
 
-    if loop:
+    if loop and (core or args.unmerge_delta):
+        opts = h3b.stack_opts(wl.merge_first, wl.merge_last, args.unmerge_delta,
+                              wl.merge_first if core else -1, wl.merge_last if core else -1)
+        ws = h3b.workspace_ex(dm, opts, wl.dtype)
+        reuse = 1 if core else wl.reuse
+
+        def step():
+            h3b.denoise_ex(dm, blocks, x, v, ws, wl.steps, opts, reuse=reuse,
+                           core_reuse=args.core_reuse if core else 1)
+        n_fresh = len([i for i in range(wl.steps) if i % reuse == 0 or i == wl.steps - 1])
+        n_core = len([i for i in range(wl.steps) if i % args.core_reuse == 0 or i == wl.steps - 1]) if core else 0
+        units = 1.0
+    elif loop:
         def step():
             h3b.denoise(dm, blocks, x, v, ws, wl.steps, wl.reuse, wl.merge_first, wl.merge_last)
         n_fresh = len([i for i in range(wl.steps) if i % wl.reuse == 0 or i == wl.steps - 1])
@@ -296,8 +310,13 @@ def run_ours(args, wl):
     flops_step = wl.block_flops() * (len(blocks) if not loop else 0)
     if loop:
         fm, fr = wl.merge_first, wl.merge_last
-        per_eval = sum(wl.block_flops(merged=(fm >= 0 and fm <= l <= fr)) for l in range(len(blocks)))
-        flops_step = per_eval * n_fresh
+        if core:
+            outer = sum(wl.block_flops() for l in range(len(blocks)) if not fm <= l <= fr)
+            inner = sum(wl.block_flops(merged=True) for l in range(fm, fr + 1))
+            flops_step = outer * n_fresh + inner * n_core
+        else:
+            per_eval = sum(wl.block_flops(merged=(fm >= 0 and fm <= l <= fr)) for l in range(len(blocks)))
+            flops_step = per_eval * n_fresh
 
     # end-to-end through the public API with the tokens in pinned host memory:
     # every step copies its input in and its result out inside the timed
@@ -344,8 +363,12 @@ def run_ours(args, wl):
         "roofline": roof, "gpu_launches": my_launches, "clocks": clocks, "kernels": kernels,
     }
     if loop:
-        line["config"].update({"steps": wl.steps, "reuse": wl.reuse, "fresh_evals": n_fresh,
-                               "token_reduction": [wl.merge_first, wl.merge_last]})
+        line["config"].update({"steps": wl.steps, "reuse": 1 if core else wl.reuse, "fresh_evals": n_fresh,
+                               "token_reduction": [wl.merge_first, wl.merge_last],
+                               "unmerge": "delta" if args.unmerge_delta else "broadcast"})
+        if core:
+            line["config"].update({"core_reuse": args.core_reuse, "core_blocks": [wl.merge_first, wl.merge_last],
+                                   "core_evals": n_core})
         line["ms_per_loop"] = round(ms / args.steps, 3)
     if e2e:
         line["e2e"] = e2e
@@ -464,6 +487,9 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--core-reuse", type=int, default=0,
+                    help="loop workload: core residual reuse over the reduction window (replaces velocity reuse)")
+    ap.add_argument("--unmerge-delta", action="store_true", help="loop workload: delta-broadcast unmerge")
     ap.add_argument("--cpu-budget", type=float, default=30.0)
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # never fewer than 3 warm-up steps

@@ -68,7 +68,7 @@ extern "C" {
 #define H3B_INT8 1
 
 /* Sizes of one DiT block.  d = n_heads * head_dim; head_dim is 64 or 128;
- * ffn = 4 * d; d and ffn are multiples of 128; eps is the RMSNorm epsilon
+ * ffn a multiple of 128 (4 * d in the workloads); d a multiple of 128; eps the RMSNorm epsilon
  * (1e-6 in the workloads), rope_theta the RoPE base (10000). */
 typedef struct h3b_dims {
   int frames, rows, cols, n_audio;   /* video grid F x H x W, audio tokens A */
@@ -142,6 +142,43 @@ int h3b_stack_forward(const h3b_dims* dims, const h3b_block_weights* blocks, int
 int h3b_denoise(const h3b_dims* dims, const h3b_block_weights* blocks, int n_blocks,
                 int merge_first, int merge_last, int n_steps, int reuse,
                 float* x, float* v, void* ws, size_t ws_bytes, int* n_fresh, void* stream);
+
+/* Options of the extended stack / loop entry points ("next" rows of the
+ * survey: delta-broadcast unmerge and core residual reuse; the pages name the
+ * core-reuse knob, --core-reuse 1/4/6, exclusive with whole-velocity reuse,
+ * in the control table, but not its arithmetic; see the readings below).
+ *   merge_first, merge_last: token-reduction window (inclusive, 0-indexed),
+ *     merge_first = -1 turns it off.
+ *   unmerge_delta: 0 = broadcast each merged token back to both columns;
+ *     1 = pre-merge tokens plus the merged blocks' update broadcast:
+ *     x(f,r,c) = x_pre(f,r,c) + (y - m)(f,r,c/2); audio rows take y.
+ *   core_first, core_last: core window for h3b_denoise_ex (-1 = off); the
+ *     reduction window must lie inside it or outside it.  Ignored by
+ *     h3b_stack_forward_ex. */
+typedef struct h3b_stack_opts {
+  int merge_first, merge_last;
+  int unmerge_delta;
+  int core_first, core_last;
+} h3b_stack_opts;
+
+/* Workspace bytes for the extended entry points (adds the saved merged input
+ * for unmerge_delta and the cached core update [S, d] fp32 for core reuse). */
+size_t h3b_workspace_bytes_ex(const h3b_dims* dims, int dtype, const h3b_stack_opts* opts);
+
+/* h3b_stack_forward with the options above. */
+int h3b_stack_forward_ex(const h3b_dims* dims, const h3b_block_weights* blocks, int n_blocks,
+                         const h3b_stack_opts* opts, float* x, void* ws, size_t ws_bytes, void* stream);
+
+/* h3b_denoise with the options above and core residual reuse: with
+ * core_first >= 0 (then reuse must be 1) every step evaluates the stack, but
+ * the core blocks run only on steps i with i % core_reuse == 0 or
+ * i == n_steps-1, where their update (core output - core input) is cached in
+ * the workspace; on the other steps that update is added instead of running
+ * them.  n_fresh / n_core_fresh (host, may be NULL) receive the numbers of
+ * stack evaluations and of core evaluations. */
+int h3b_denoise_ex(const h3b_dims* dims, const h3b_block_weights* blocks, int n_blocks,
+                   const h3b_stack_opts* opts, int n_steps, int reuse, int core_reuse, float* x, float* v,
+                   void* ws, size_t ws_bytes, int* n_fresh, int* n_core_fresh, void* stream);
 
 /* Per-row symmetric int8 quantisation [int8]: s[r] = max_k |w[r,k]| / 127
  * (fp32), q[r,k] = rint(w[r,k] / s[r]) (IEEE fp32 divide, half-even),

@@ -101,3 +101,26 @@ def test_gemm_argument_errors():
     assert g(fake, fake, 128, 128, 128, 1, 0, fake, None, None, None, None, None, None, 0, None) == -1   # scales
     assert g(fake, fake, 128, 128, 128, 0, 9, fake, None, None, None, None, None, None, 0, None) == -4
     assert g(fake, fake + 8, 128, 128, 128, 0, 0, fake, None, None, None, None, None, None, 0, None) == -2
+
+
+def test_extended_options_argument_errors():
+    dm = h3b.dims_of(wlmod.WORKLOADS["block_d256_s288"])
+    fake = 1 << 20
+    arr = (h3b.BlockWeights * 4)(*[_weights(fake) for _ in range(4)])
+    dn = h3b.lib.h3b_denoise_ex
+    o = h3b.stack_opts(core_first=1, core_last=2)
+    need = h3b.lib.h3b_workspace_bytes_ex(ctypes.byref(dm), 0, ctypes.byref(o))
+    assert need > h3b.workspace_bytes(dm)                                       # + cached core update
+    # core reuse excludes whole-velocity reuse
+    assert dn(ctypes.byref(dm), arr, 4, ctypes.byref(o), 20, 2, 4, fake, fake, fake, need, None, None, None) == -3
+    # the reduction window partly overlapping the core window
+    o2 = h3b.stack_opts(0, 1, core_first=1, core_last=2)
+    need2 = h3b.lib.h3b_workspace_bytes_ex(ctypes.byref(dm), 0, ctypes.byref(o2))
+    assert dn(ctypes.byref(dm), arr, 4, ctypes.byref(o2), 20, 1, 4, fake, fake, fake, need2, None, None, None) == -3
+    # core window past the stack
+    o3 = h3b.stack_opts(core_first=2, core_last=4)
+    assert dn(ctypes.byref(dm), arr, 4, ctypes.byref(o3), 20, 1, 4, fake, fake, fake, need, None, None, None) == -3
+    # workspace without room for the cached update
+    small = h3b.workspace_bytes(dm)
+    assert dn(ctypes.byref(dm), arr, 4, ctypes.byref(o), 20, 1, 4, fake, fake, fake, small, None, None, None) == -5
+    assert h3b.lib.h3b_stack_forward_ex(ctypes.byref(dm), arr, 4, None, fake, fake, need, None) == -1

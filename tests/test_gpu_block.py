@@ -247,3 +247,79 @@ def test_host_pipeline_matches_device_calls(cuda_dev):
         h3b.block_forward(dm, blk, ref, ws)
         torch.cuda.synchronize()
         assert torch.equal(o, ref.cpu())
+
+
+# ----------------------------------------------------------------------------- next rows: delta unmerge, core reuse
+def _identity_blocks(wl, n, dev):
+    out = []
+    for l in range(n):
+        w = wlmod.block_weights(wl, l, dev)
+        w["w_o"] = torch.zeros_like(w["w_o"])
+        w["w_fc2"] = torch.zeros_like(w["w_fc2"])
+        out.append(h3b.Block.from_dict(w))
+    return out
+
+
+def test_unmerge_delta_identity_blocks_bitexact(cuda_dev):
+    """Blocks that change nothing: the delta unmerge returns x exactly, the
+    plain unmerge returns the pair means."""
+    wl = TINY.with_(n_blocks=3)
+    dm = h3b.dims_of(wl)
+    blocks = _identity_blocks(wl, 3, cuda_dev)
+    x0 = wlmod.initial_tokens(wl, cuda_dev)
+    for delta in (True, False):
+        o = h3b.stack_opts(0, 1, unmerge_delta=delta)
+        x = x0.clone()
+        h3b.stack_forward_ex(dm, blocks, x, h3b.workspace_ex(dm, o), o)
+        torch.cuda.synchronize()
+        if delta:
+            assert torch.equal(x, x0)
+        else:
+            ref = oracle.token_unmerge(oracle.token_merge(np64(x0), wl), wl).astype(np.float32)
+            assert np.array_equal(x.cpu().numpy(), ref)
+
+
+def test_stack_unmerge_delta_vs_oracle(cuda_dev):
+    wl = TINY.with_(n_blocks=5, depth_scaled_init=True, seed=8)
+    ws_ = [wlmod.block_weights(wl, l, cuda_dev) for l in range(5)]
+    blocks = [h3b.Block.from_dict(w) for w in ws_]
+    dm = h3b.dims_of(wl)
+    o = h3b.stack_opts(1, 3, unmerge_delta=True)
+    x0 = wlmod.initial_tokens(wl, cuda_dev)
+    x = x0.clone()
+    h3b.stack_forward_ex(dm, blocks, x, h3b.workspace_ex(dm, o), o)
+    torch.cuda.synchronize()
+    ref = oracle.stack_forward_ex(np64(x0), [host_weights(w) for w in ws_], wl, 1, 3, unmerge_delta=True)
+    check_bf16(np64(x0), np64(x), ref)
+
+
+@pytest.mark.parametrize("core_reuse,delta", [(2, False), (4, True), (1, True)])
+def test_denoise_core_reuse_vs_oracle(cuda_dev, core_reuse, delta):
+    wl = TINY.with_(n_blocks=5, depth_scaled_init=True, seed=9)
+    ws_ = [wlmod.block_weights(wl, l, cuda_dev) for l in range(5)]
+    blocks = [h3b.Block.from_dict(w) for w in ws_]
+    dm = h3b.dims_of(wl)
+    o = h3b.stack_opts(2, 3, unmerge_delta=delta, core_first=1, core_last=3)
+    x0 = wlmod.initial_tokens(wl, cuda_dev)
+    x = x0.clone()
+    v = torch.empty_like(x)
+    nf, nc = h3b.denoise_ex(dm, blocks, x, v, h3b.workspace_ex(dm, o), 6, o, reuse=1, core_reuse=core_reuse)
+    torch.cuda.synchronize()
+    assert h3b.device_error() == 0
+    ref, nc_ref = oracle.denoise_core(np64(x0), [host_weights(w) for w in ws_], wl, 6, core_reuse, 1, 3, 2, 3,
+                                      unmerge_delta=delta)
+    assert nf == 6 and nc == nc_ref
+    assert rel_l2(x, ref) <= 1e-2 and max_abs(x, ref) <= 5e-2
+
+
+def test_denoise_core_counts(cuda_dev):
+    wl = TINY.with_(n_blocks=3)
+    blocks = [h3b.Block.from_dict(wlmod.block_weights(wl, l, cuda_dev)) for l in range(3)]
+    dm = h3b.dims_of(wl)
+    o = h3b.stack_opts(core_first=1, core_last=1)
+    ws = h3b.workspace_ex(dm, o)
+    x = wlmod.initial_tokens(wl, cuda_dev)
+    v = torch.empty_like(x)
+    got = [h3b.denoise_ex(dm, blocks, x, v, ws, 20, o, core_reuse=r) for r in (1, 4, 6)]
+    assert got == [(20, 20), (20, 6), (20, 5)]
+    assert [len(oracle.fresh_steps(20, r)) for r in (1, 4, 6)] == [20, 6, 5]
