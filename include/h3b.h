@@ -143,10 +143,11 @@ int h3b_denoise(const h3b_dims* dims, const h3b_block_weights* blocks, int n_blo
                 int merge_first, int merge_last, int n_steps, int reuse,
                 float* x, float* v, void* ws, size_t ws_bytes, int* n_fresh, void* stream);
 
-/* Options of the extended stack / loop entry points ("next" rows of the
- * survey: delta-broadcast unmerge and core residual reuse; the pages name the
- * core-reuse knob, --core-reuse 1/4/6, exclusive with whole-velocity reuse,
- * in the control table, but not its arithmetic; see the readings below).
+/* Options of the extended stack / loop entry points: a delta-broadcast
+ * unmerge and core residual reuse.  The siami.tw article's control table names
+ * the core-reuse knob (--core-reuse 1/4/6, exclusive with whole-velocity
+ * reuse) but not its arithmetic, and no page gives an unmerge rule; the forms
+ * below are the plainest readings.
  *   merge_first, merge_last: token-reduction window (inclusive, 0-indexed),
  *     merge_first = -1 turns it off.
  *   unmerge_delta: 0 = broadcast each merged token back to both columns;
