@@ -45,7 +45,8 @@ DEFAULT_WORKLOAD = "block_d3072_s6400"
 METRIC = "DiT block tokens/s"
 # default timed steps per workload: about 1-30 s of device time each
 DEFAULT_STEPS = {"block_d256_s288": 2000, "block_d3072_s6400": 300, "stack8_d5120_s6528": 30,
-                 "block_int8_d5120_s20640": 60, "loop45_d5120_s6528": 2}
+                 "block_int8_d5120_s20640": 60, "loop45_d5120_s6528": 2,
+                 "preview40_d5120_s2784": 4}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -490,10 +491,20 @@ def main():
     ap.add_argument("--core-reuse", type=int, default=0,
                     help="loop workload: core residual reuse over the reduction window (replaces velocity reuse)")
     ap.add_argument("--unmerge-delta", action="store_true", help="loop workload: delta-broadcast unmerge")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="loop workload: run only the first L blocks (the pages' --layers 40/45/50)")
+    ap.add_argument("--denoise-steps", type=int, default=0,
+                    help="loop workload: denoising steps (the pages' 4..7-step presets; default: the workload's)")
     ap.add_argument("--cpu-budget", type=float, default=30.0)
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # never fewer than 3 warm-up steps
     wl = W.WORKLOADS[args.workload]
+    if args.layers or args.denoise_steps:
+        if wl.steps == 0:
+            ap.error("--layers / --denoise-steps apply to the denoising-loop workloads")
+        if args.layers and not (0 < args.layers and (wl.merge_last < args.layers)):
+            ap.error("--layers must keep the token-reduction window inside the active blocks")
+        wl = wl.with_(n_blocks=args.layers or wl.n_blocks, steps=args.denoise_steps or wl.steps)
     if args.steps is None:
         args.steps = DEFAULT_STEPS[args.workload] if args.impl == "ours" else 10
     if args.impl == "reference":

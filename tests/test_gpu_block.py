@@ -183,6 +183,24 @@ def test_denoise_small_vs_oracle(cuda_dev, steps, reuse, mf, ml):
     assert max_abs(x, ref) <= 5e-2
 
 
+@pytest.mark.parametrize("steps,reuse", [(4, 1), (5, 2), (7, 3)])
+def test_denoise_few_steps_layer_subset_vs_oracle(cuda_dev, steps, reuse):
+    """The 4..7-step presets on the first L = 3 of a 5-block model (--layers):
+    the loop is given only the active blocks."""
+    wl = TINY.with_(n_blocks=5, depth_scaled_init=True, seed=11, frames=2, rows=6, cols=10, n_audio=24)
+    ws_ = [wlmod.block_weights(wl, l, cuda_dev) for l in range(3)]
+    blocks = [h3b.Block.from_dict(w) for w in ws_]
+    dm = h3b.dims_of(wl)
+    x0 = wlmod.initial_tokens(wl, cuda_dev)
+    x = x0.clone()
+    v = torch.empty_like(x)
+    nf = h3b.denoise(dm, blocks, x, v, h3b.workspace(dm), steps, reuse)
+    torch.cuda.synchronize()
+    ref, nf_ref = oracle.denoise(np64(x0), [host_weights(w) for w in ws_], wl, steps, reuse)
+    assert nf == nf_ref
+    assert rel_l2(x, ref) <= 1e-2 and max_abs(x, ref) <= 5e-2
+
+
 def test_denoise_fresh_counts(cuda_dev):
     wl = TINY.with_(n_blocks=1)
     blocks = [h3b.Block.from_dict(wlmod.block_weights(wl, 0, cuda_dev))]

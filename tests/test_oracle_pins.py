@@ -374,6 +374,21 @@ def test_fresh_counts_golden():
         assert len(oracle.fresh_steps(g["n_steps"], int(r))) == n
 
 
+def test_fresh_counts_closed_form_few_steps():
+    """The 4..7-step presets and every other (N, r): the fresh steps are the
+    multiples of r below N plus the last step, so their number is
+    ceil((N-1)/r) + 1 for N >= 2 (and 1 for N = 1); the last step is always
+    fresh and step 0 always is."""
+    for n in range(1, 51):
+        for r in range(1, 8):
+            f = oracle.fresh_steps(n, r)
+            assert len(f) == (1 if n == 1 else -(-(n - 1) // r) + 1)
+            assert f[0] == 0 and f[-1] == n - 1
+    # the presets with the control table's reuse levels
+    assert [len(oracle.fresh_steps(n, 1)) for n in (4, 5, 6, 7)] == [4, 5, 6, 7]
+    assert [len(oracle.fresh_steps(n, 3)) for n in (4, 5, 6, 7)] == [2, 3, 3, 3]
+
+
 def test_sigmas_grid():
     s = oracle.sigmas(20)
     assert s.dtype == np.float32 and len(s) == 21

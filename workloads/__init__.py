@@ -89,6 +89,10 @@ WORKLOADS = {
     # 20-step flow-matching loop, reuse 2, 45 blocks, token reduction in blocks 15..29.
     "loop45_d5120_s6528": Workload("loop45_d5120_s6528", 6, 32, 32, 384, 5120, 40, 128, 20480, 45, BF16, 4, True,
                                    steps=20, reuse=2, merge_first=15, merge_last=29),
+    # The pages' aggressive preview: 320x320 internal canvas (6x20x20 latent video + 384 audio),
+    # 40 active blocks, reuse 3, 20 steps, no token reduction.
+    "preview40_d5120_s2784": Workload("preview40_d5120_s2784", 6, 20, 20, 384, 5120, 40, 128, 20480, 40, BF16, 5,
+                                      True, steps=20, reuse=3),
 }
 
 
