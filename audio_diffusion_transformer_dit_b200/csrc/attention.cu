@@ -10,8 +10,8 @@
 //               MMA reads it as its A operand.  O is rescaled in TMEM only when
 //               the running max grows by more than 2^8 (lazy rescale: o = O/l
 //               is exact for any reference max, the threshold bounds P <= 256).
-//   warp 8      TMA producer: Q_A, Q_B once; K and V tiles of 128 keys through
-//               two-stage rings.
+//   warp 8      TMA producer: Q_A, Q_B once; K tiles of 128 keys through a
+//               three-stage ring, V tiles through a two-stage ring.
 //   warp 9      MMA issuer: per key tile j, PV_A(j), S_A(j+1), PV_B(j),
 //               S_B(j+1).  MMAs from one thread execute in issue order, so
 //               S_A(j+1) may overwrite the columns PV_A(j) reads P from.
@@ -32,7 +32,7 @@ namespace h3b {
 
 namespace {
 
-constexpr int BQ = 128, BKV = 128, THREADS = 384, KS = 2, VS = 2;
+constexpr int BQ = 128, BKV = 128, THREADS = 384, KS = 3, VS = 2;
 // Register split (setmaxnreg): launch 384 x 168 = 64512; softmax warpgroups
 // 2 x 128 x 216 = 55296 plus control warpgroup 128 x 56 = 7168 -> 62464.
 constexpr int REG_SOFTMAX = 216, REG_CONTROL = 56;
@@ -42,7 +42,8 @@ constexpr int POLY_OF_8 = 0;   // key pairs (of every 8) that take the FMA-pipe 
 __host__ __device__ constexpr uint32_t s_col(int t) { return t * 256u; }
 __host__ __device__ constexpr uint32_t o_col(int t) { return t * 256u + 128u; }
 constexpr int TMEM_COLS = 512;
-constexpr int NUM_BARS = 18;
+// q_full, k_full/k_empty per K stage, v_full/v_empty per V stage, s_full x2, p_full x2x2, o_final x2, mma_done
+constexpr int NUM_BARS = 1 + 2 * KS + 2 * VS + 2 + 4 + 2 + 1;
 
 struct AttnArgs {
   int S, n_heads;
