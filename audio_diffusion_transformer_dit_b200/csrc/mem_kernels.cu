@@ -140,33 +140,45 @@ __global__ void k_unmerge_delta(float4* __restrict__ x, const float4* __restrict
 // ------------------------------------------------------------------ RoPE table
 // table[s][j] = (cos, sin) of pos * theta^(-2 jl / n) for pair j of token s,
 // jl the pair's index inside its section of width n (fp64 angle, fp32 store).
+// The D/2 frequencies of the video sections and of the audio section are
+// computed once per block (fp64) into shared memory; each element then costs
+// one fp64 product and a fp64 reduction modulo 2 pi before the fp32 sincos.
+constexpr int kMaxHalfHead = 64;  // head_dim <= 128
 __global__ void k_rope_table(float2* __restrict__ table, int F, int H, int Wc, int A, int D, float theta,
                              int merged) {
+  __shared__ double f_video[kMaxHalfHead], f_audio[kMaxHalfHead];
   const int half = D / 2;
+  const int nf = D / 4, nr = 3 * D / 8, nc = D - nf - nr;
+  const double l2t = log2(static_cast<double>(theta));
+  for (int j = threadIdx.x; j < half; j += blockDim.x) {
+    int jl, n;
+    if (j < nf / 2) {
+      jl = j; n = nf;
+    } else if (j < (nf + nr) / 2) {
+      jl = j - nf / 2; n = nr;
+    } else {
+      jl = j - (nf + nr) / 2; n = nc;
+    }
+    f_video[j] = exp2(-2.0 * jl / n * l2t);
+    f_audio[j] = exp2(-2.0 * j / D * l2t);
+  }
+  __syncthreads();
   const int n_video = F * H * Wc;
   const size_t total = static_cast<size_t>(n_video + A) * half;
-  const int nf = D / 4, nr = 3 * D / 8, nc = D - nf - nr;
   for (size_t e = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < total;
        e += static_cast<size_t>(gridDim.x) * blockDim.x) {
     const int s = static_cast<int>(e / half), j = static_cast<int>(e % half);
-    double pos;
-    int jl, n;
+    double ang;
     if (s < n_video) {
       const int f = s / (H * Wc), rem = s % (H * Wc), r = rem / Wc, c = rem % Wc;
-      if (j < nf / 2) {
-        pos = f; jl = j; n = nf;
-      } else if (j < (nf + nr) / 2) {
-        pos = r; jl = j - nf / 2; n = nr;
-      } else {
-        pos = merged ? 2.0 * c + 0.5 : static_cast<double>(c); jl = j - (nf + nr) / 2; n = nc;
-      }
+      const double pos = j < nf / 2 ? f : j < (nf + nr) / 2 ? r : (merged ? 2.0 * c + 0.5 : static_cast<double>(c));
+      ang = pos * f_video[j];
     } else {
-      pos = s - n_video; jl = j; n = D;
+      ang = static_cast<double>(s - n_video) * f_audio[j];
     }
-    // fp64 angle, reduced to [-pi, pi] in fp64, then fp32 sin/cos of the remainder
-    const double ang = pos * exp2(-2.0 * jl / n * log2(static_cast<double>(theta)));
-    const double two_pi = 6.283185307179586;
-    const float red = static_cast<float>(fma(-rint(ang / two_pi), two_pi, ang));
+    // reduce to about [-pi, pi] in fp64, then fp32 sin/cos of the remainder
+    const double two_pi = 6.283185307179586, inv_two_pi = 0.15915494309189535;
+    const float red = static_cast<float>(fma(-rint(ang * inv_two_pi), two_pi, ang));
     float sn, cs;
     sincosf(red, &sn, &cs);
     table[e] = make_float2(cs, sn);
@@ -386,7 +398,7 @@ cudaError_t launch_rope_table(const Ctx& c, const h3b_dims& dm, int merged, floa
   const int wc = merged ? dm.cols / 2 : dm.cols;
   const size_t total = static_cast<size_t>(dm.frames * dm.rows * wc + dm.n_audio) * (dm.head_dim / 2);
   if (total == 0) return cudaSuccess;
-  k_rope_table<<<grid_for(total, c.num_sms, 64), kThreads, 0, c.stream>>>(
+  k_rope_table<<<grid_for(total, c.num_sms, 8), kThreads, 0, c.stream>>>(
       reinterpret_cast<float2*>(table), dm.frames, dm.rows, wc, dm.n_audio, dm.head_dim, dm.rope_theta, merged);
   return cudaGetLastError();
 }
