@@ -37,7 +37,7 @@ import numpy as np
 from scipy.special import erf as _erf
 
 __all__ = [
-    "READINGS", "PINS",
+    "READINGS", "PINS", "MOD_FIELDS", "block_forward_cond", "stack_forward_cond", "denoise_cond",
     "linear", "rmsnorm", "gelu", "rope_sections", "token_positions", "rope_angles", "apply_rope",
     "attention", "block_forward", "stack_forward", "token_merge", "token_unmerge",
     "quantize_rows", "dequantize_rows", "int8_matmul", "dequant_weights", "block_forward_w8a8",
@@ -70,6 +70,14 @@ READINGS = {
                   "but the core blocks run only on fresh-core steps (i % r == 0 or the last step); their update "
                   "(output - input of the core) is cached and added on the other steps",
     "layers": "--layers L: the stack is given the active blocks (the first L of the model in the workloads)",
+    "modulation": "timestep conditioning as adaLN-style modulation (the pages give no form): per block and row "
+                  "class, u = RMSNorm(x)*(1+scale)+shift before the QKV and FC1 GEMMs and x += gate*update "
+                  "after the O-proj and FC2 GEMMs; class 0 = generated (video + audio) rows, class 1 = "
+                  "condition rows",
+    "condition_rows": "fixed condition rows (siami.tw file list: 0.999 condition augmentation + fixed condition "
+                      "rows in native DiT): C rows appended after the audio tokens, given already augmented; "
+                      "they take part in every block (joint attention) with no rotary embedding, every "
+                      "evaluation starts them from the given values, and the Euler update leaves them out",
 }
 
 # What pins each function to something other than itself (tests/test_oracle_*.py).
@@ -91,6 +99,12 @@ PINS = {
                            "identity when the merged blocks change nothing",
     "denoise_core": "core_reuse = 1 equals the plain loop; a core that adds a constant gives the closed form; "
                     "hand-computed 3-step case",
+    "block_forward_cond": "identity modulation without condition rows equals block_forward; zero gates give the "
+                          "identity; scale = -1 makes every normed row equal to the shift (closed form without "
+                          "RoPE); condition rows are permutation-equivariant among themselves (no rotation); a "
+                          "class-1 zero gate leaves condition rows unchanged",
+    "denoise_cond": "no condition rows and no modulation equals denoise / denoise_core; a toy block gives the "
+                    "closed form that needs the condition rows refilled every evaluation",
 }
 
 
@@ -228,37 +242,39 @@ def block_forward(x, w, dims, merged=False, rows=None, rope=True):
 
 def token_merge(x, dims):
     """Token reduction: the merged video token (f, r, c') is the mean of the
-    horizontally adjacent pair (f, r, 2c') and (f, r, 2c'+1); audio rows are
-    carried unchanged after the merged video rows."""
+    horizontally adjacent pair (f, r, 2c') and (f, r, 2c'+1); the rows after
+    the video rows (audio, then any condition rows) are carried unchanged after
+    the merged video rows."""
     x = _f64(x)
-    F, H, W, A = dims.frames, dims.rows, dims.cols, dims.n_audio
+    F, H, W = dims.frames, dims.rows, dims.cols
     V = F * H * W
     vid = x[:V].reshape(F, H, W, -1)
     m = (vid[:, :, 0::2, :] + vid[:, :, 1::2, :]) * 0.5
-    return np.concatenate([m.reshape(V // 2, -1), x[V:V + A]], axis=0)
+    return np.concatenate([m.reshape(V // 2, -1), x[V:]], axis=0)
 
 
 def token_unmerge(xm, dims):
     """Inverse of the reduction: each merged token is broadcast back to both
-    columns it came from; audio rows are carried unchanged."""
+    columns it came from; the rows after the video rows are carried unchanged."""
     xm = _f64(xm)
-    F, H, W, A = dims.frames, dims.rows, dims.cols, dims.n_audio
+    F, H, W = dims.frames, dims.rows, dims.cols
     V = F * H * W
     vid = xm[:V // 2].reshape(F, H, W // 2, -1)
     full = np.repeat(vid, 2, axis=2)
-    return np.concatenate([full.reshape(V, -1), xm[V // 2:V // 2 + A]], axis=0)
+    return np.concatenate([full.reshape(V, -1), xm[V // 2:]], axis=0)
 
 
 def token_unmerge_delta(x_pre, ym, xm0, dims):
     """Delta-broadcast unmerge: full token (f, r, c) = x_pre(f, r, c) +
     (ym - xm0)(f, r, c // 2), where xm0 is the merged sequence that entered
-    the merged blocks and ym what they returned; audio rows take ym."""
+    the merged blocks and ym what they returned; the rows after the video rows
+    (audio, condition) take ym."""
     x_pre, ym, xm0 = _f64(x_pre), _f64(ym), _f64(xm0)
-    F, H, W, A = dims.frames, dims.rows, dims.cols, dims.n_audio
+    F, H, W = dims.frames, dims.rows, dims.cols
     V = F * H * W
     dv = (ym[:V // 2] - xm0[:V // 2]).reshape(F, H, W // 2, -1)
     full = x_pre[:V].reshape(F, H, W, -1) + np.repeat(dv, 2, axis=2)
-    return np.concatenate([full.reshape(V, -1), ym[V // 2:V // 2 + A]], axis=0)
+    return np.concatenate([full.reshape(V, -1), ym[V // 2:]], axis=0)
 
 
 def stack_forward_ex(x, blocks, dims, merge_first=-1, merge_last=-1, unmerge_delta=False, block_fn=None):
@@ -387,6 +403,135 @@ def block_forward_w8a8(x, w, dims, merged=False, rope=True):
     x1 = x + _w8a8_linear(o, *qw["w_o"])
     g = gelu(_w8a8_linear(rmsnorm(x1, w["g_mlp"], dims.eps), *qw["w_fc1"]))
     return x1 + _w8a8_linear(g, *qw["w_fc2"])
+
+
+# ----------------------------------------------------------------------------- modulation and condition rows
+MOD_FIELDS = ("shift_attn", "scale_attn", "gate_attn", "shift_mlp", "scale_mlp", "gate_mlp")
+
+
+def _mod_rows(mod, n_rows, n_cond, field):
+    """[rows, d] view of one modulation field: class 0 for the generated rows,
+    class 1 for the last n_cond (condition) rows."""
+    mod = _f64(mod)
+    i = MOD_FIELDS.index(field)
+    cls = np.zeros(n_rows, dtype=np.int64)
+    cls[n_rows - n_cond:] = 1
+    return mod[cls, i, :]
+
+
+def block_forward_cond(x, w, dims, mod=None, n_cond=0, merged=False, rows=None, rope=True):
+    """block_forward over [generated rows ; n_cond condition rows] with
+    adaLN-style modulation.  ``mod``: [2, 6, d] (row class, MOD_FIELDS) or
+    None (scale 0, shift 0, gate 1):
+
+        u  = RMSNorm(x; g_attn) * (1 + scale_attn) + shift_attn
+        x1 = x + gate_attn * (Attn(RoPE(u W_qkv^T)) W_o^T)
+        x2 = x1 + gate_mlp * (GELU((RMSNorm(x1; g_mlp) * (1 + scale_mlp) + shift_mlp) W_fc1^T) W_fc2^T)
+
+    Condition rows carry no rotary embedding; every row attends to every row.
+    ``rows`` returns x2 only at those rows (keys/values still cover all)."""
+    x = _f64(x)
+    S, d = x.shape
+    Sg = S - n_cond
+    H = dims.n_heads
+    rows = np.arange(S) if rows is None else np.asarray(rows)
+    if mod is None:
+        mod = np.zeros((2, 6, d))
+        mod[:, 2, :] = 1.0
+        mod[:, 5, :] = 1.0
+    f = {k: _mod_rows(mod, S, n_cond, k) for k in MOD_FIELDS}
+    wqkv = _f64(w["w_qkv"])
+    u = rmsnorm(x, w["g_attn"], dims.eps) * (1.0 + f["scale_attn"]) + f["shift_attn"]
+    k = u @ wqkv[d:2 * d].T
+    v = u @ wqkv[2 * d:3 * d].T
+    q = u[rows] @ wqkv[:d].T
+    if rope:
+        ang = np.zeros((S, d // H // 2))
+        ang[:Sg] = rope_angles(dims, merged)
+        q = apply_rope(q, ang[rows], H)
+        k = apply_rope(k, ang, H)
+    o = attention(q, k, v, H)
+    x1 = x[rows] + f["gate_attn"][rows] * (o @ _f64(w["w_o"]).T)
+    h2 = rmsnorm(x1, w["g_mlp"], dims.eps) * (1.0 + f["scale_mlp"][rows]) + f["shift_mlp"][rows]
+    return x1 + f["gate_mlp"][rows] * (gelu(h2 @ _f64(w["w_fc1"]).T) @ _f64(w["w_fc2"]).T)
+
+
+def stack_forward_cond(x, blocks, dims, mods=None, n_cond=0, merge_first=-1, merge_last=-1, unmerge_delta=False,
+                       block_fn=None):
+    """Blocks in order on [generated ; condition] rows; block l takes
+    ``mods[l]`` ([2, 6, d]) when ``mods`` is given.  Token reduction as in
+    stack_forward_ex (condition rows are carried like the audio rows)."""
+    fn = block_forward_cond if block_fn is None else block_fn
+    on = merge_first >= 0
+    x = _f64(x)
+    x_pre = xm0 = None
+    for layer, w in enumerate(blocks):
+        if on and layer == merge_first:
+            x_pre = x
+            xm0 = token_merge(x, dims)
+            x = xm0
+        x = fn(x, w, dims, None if mods is None else mods[layer], n_cond,
+               merged=on and merge_first <= layer <= merge_last)
+        if on and layer == merge_last:
+            x = token_unmerge_delta(x_pre, x, xm0, dims) if unmerge_delta else token_unmerge(x, dims)
+    return x
+
+
+def denoise_cond(x0, blocks, dims, n_steps, cond_rows=None, mods=None, reuse=1, merge_first=-1, merge_last=-1,
+                 unmerge_delta=False, core_reuse=1, core_first=-1, core_last=-1, block_fn=None):
+    """The flow-matching loop with fixed condition rows and per-step
+    modulation.  x0: generated rows [S, d]; cond_rows: [C, d] (every
+    evaluation starts from them; the Euler update covers the S generated rows
+    only); mods: None, [n_blocks, 2, 6, d] for every step or
+    [n_steps, n_blocks, 2, 6, d].  Velocity reuse (reuse) or, with
+    core_first >= 0 and reuse = 1, core residual reuse as in denoise_core.
+    Returns (x_N, stack evaluations, core evaluations)."""
+    x = _f64(x0)
+    S = x.shape[0]
+    C = 0 if cond_rows is None else len(cond_rows)
+    cond = np.zeros((0, x.shape[1])) if cond_rows is None else _f64(cond_rows)
+    L = len(blocks)
+    if core_first >= 0:
+        if reuse != 1:
+            raise ValueError("core reuse excludes whole-velocity reuse")
+        inside = merge_first >= 0 and core_first <= merge_first and merge_last <= core_last
+        if not (inside or merge_first < 0 or merge_last < core_first or merge_first > core_last):
+            raise ValueError("the token-reduction window must lie inside the core window or outside it")
+
+    def mods_at(i):
+        if mods is None:
+            return None
+        m = _f64(mods)
+        return m[i] if m.ndim == 5 else m
+
+    def run(e, lo, hi, i):  # blocks lo..hi, the reduction window re-based when it lies in them
+        if lo > hi:
+            return e
+        mf, ml = (merge_first - lo, merge_last - lo) if merge_first >= 0 and lo <= merge_first <= hi else (-1, -1)
+        m = mods_at(i)
+        return stack_forward_cond(e, blocks[lo:hi + 1], dims, None if m is None else m[lo:hi + 1], C, mf, ml,
+                                  unmerge_delta, block_fn)
+
+    sig = sigmas(n_steps)
+    vel = delta = None
+    n_fresh = n_core = 0
+    for i in range(n_steps):
+        if core_first >= 0:
+            e = run(np.concatenate([x, cond], axis=0), 0, core_first - 1, i)
+            if is_fresh(i, n_steps, core_reuse):
+                out = run(e, core_first, core_last, i)
+                delta = out - e
+                e = out
+                n_core += 1
+            else:
+                e = e + delta
+            vel = run(e, core_last + 1, L - 1, i)[:S]
+            n_fresh += 1
+        elif is_fresh(i, n_steps, reuse):
+            vel = run(np.concatenate([x, cond], axis=0), 0, L - 1, i)[:S]
+            n_fresh += 1
+        x = flow_step(x, vel, sig[i], sig[i + 1])
+    return x, n_fresh, n_core
 
 
 # ----------------------------------------------------------------------------- flow-matching loop

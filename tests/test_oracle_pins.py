@@ -166,10 +166,20 @@ def test_attention_uniform_and_convex():
 
 
 # ----------------------------------------------------------------------------- block
-def brute_block(x, w, dm, merged=False):
+def brute_block(x, w, dm, merged=False, mod=None, n_cond=0):
     """Pure-Python loops: RMSNorm, QKV, RoPE by explicit (f,r,c)/audio
-    positions, softmax attention, output projection, RMSNorm, GELU MLP."""
+    positions, softmax attention, output projection, RMSNorm, GELU MLP.
+    With ``mod`` ([2][6][d] nested lists: shift/scale/gate for attention, then
+    for the MLP; class 1 = the last n_cond rows) each normed row becomes
+    u*(1+scale)+shift and each residual update is multiplied by its gate;
+    the n_cond condition rows get no rotation."""
     S, d, H, D, f = len(x), dm.d, dm.n_heads, dm.head_dim, dm.ffn
+    if mod is None:
+        ident = [[0.0] * d, [0.0] * d, [1.0] * d]
+        mod = [ident + ident, ident + ident]
+
+    def cls(i):
+        return 1 if i >= S - n_cond else 0
     wqkv, wo, w1, w2 = (w[k].tolist() for k in ("w_qkv", "w_o", "w_fc1", "w_fc2"))
 
     def norm(row, g):
@@ -189,9 +199,13 @@ def brute_block(x, w, dm, merged=False):
                 pos.append(("v", fi, ri, 2 * ci + 0.5 if merged else ci))
     for a in range(A):
         pos.append(("a", a))
+    for _ in range(n_cond):
+        pos.append(("c",))
 
     def rot(vec, p):
         out = list(vec)
+        if p[0] == "c":
+            return out
         for h in range(H):
             for j in range(D // 2):
                 if p[0] == "a":
@@ -208,18 +222,22 @@ def brute_block(x, w, dm, merged=False):
                 out[h * D + 2 * j + 1] = a0 * math.sin(ang) + a1 * math.cos(ang)
         return out
 
-    u = [norm(row, w["g_attn"].tolist()) for row in x]
+    def modulate(row, i, first):
+        sh, sc = mod[cls(i)][first], mod[cls(i)][first + 1]
+        return [a * (1.0 + sc[e]) + sh[e] for e, a in enumerate(row)]
+
+    u = [modulate(norm(row, w["g_attn"].tolist()), i, 0) for i, row in enumerate(x)]
     qkv = [mv(wqkv, row) for row in u]
     q = [rot(r[:d], pos[i]) for i, r in enumerate(qkv)]
     k = [rot(r[d:2 * d], pos[i]) for i, r in enumerate(qkv)]
     v = [r[2 * d:] for r in qkv]
     o = brute_attention(q, k, v, H).tolist()
-    x1 = [[a + b for a, b in zip(x[i], mv(wo, o[i]))] for i in range(S)]
+    x1 = [[a + gt * b for a, b, gt in zip(x[i], mv(wo, o[i]), mod[cls(i)][2])] for i in range(S)]
     out = []
     for i in range(S):
-        hvec = mv(w1, norm(x1[i], w["g_mlp"].tolist()))
+        hvec = mv(w1, modulate(norm(x1[i], w["g_mlp"].tolist()), i, 3))
         g = [0.5 * a * (1 + math.erf(a / math.sqrt(2))) for a in hvec]
-        out.append([a + b for a, b in zip(x1[i], mv(w2, g))])
+        out.append([a + gt * b for a, b, gt in zip(x1[i], mv(w2, g), mod[cls(i)][5])])
     return np.array(out)
 
 
@@ -275,6 +293,117 @@ def test_block_row_sampling_matches_full():
     rows = np.array([0, 5, 31, 32, 36])
     full = oracle.block_forward(x, w, dm)
     assert np.allclose(oracle.block_forward(x, w, dm, rows=rows), full[rows], rtol=1e-13, atol=1e-14)
+
+
+# ----------------------------------------------------------------------------- modulation and condition rows
+def rand_mod(rng, d, scale=0.3):
+    m = rng.normal(size=(2, 6, d)) * scale
+    m[:, 2, :] += 1.0   # gates around 1
+    m[:, 5, :] += 1.0
+    return m
+
+
+@pytest.mark.parametrize("merged,n_cond", [(False, 0), (False, 3), (True, 2)])
+def test_cond_block_vs_bruteforce(merged, n_cond):
+    dm = dims_of(1, 2, 4, 2, 32, 2, 64)
+    rng = np.random.default_rng(30 + n_cond)
+    S = (4 if merged else 8) + 2 + n_cond
+    x = rng.normal(size=(S, 32))
+    w = rand_block(rng, 32, 64)
+    mod = rand_mod(rng, 32)
+    ref = brute_block(x.tolist(), w, dm, merged, mod.tolist(), n_cond)
+    got = oracle.block_forward_cond(x, w, dm, mod, n_cond, merged=merged)
+    assert np.allclose(got, ref, rtol=1e-11, atol=1e-12)
+
+
+def test_cond_block_identity_modulation_and_zero_gates():
+    dm = dims_of(2, 2, 2, 3, 64, 4, 128)
+    rng = np.random.default_rng(31)
+    x = rng.normal(size=(11, 64))
+    w = rand_block(rng, 64, 128)
+    ident = np.zeros((2, 6, 64))
+    ident[:, 2] = ident[:, 5] = 1.0
+    assert np.allclose(oracle.block_forward_cond(x, w, dm, ident), oracle.block_forward(x, w, dm), rtol=1e-14)
+    assert np.allclose(oracle.block_forward_cond(x, w, dm, None), oracle.block_forward(x, w, dm), rtol=1e-14)
+    # zero gates: the block adds nothing, whatever the shifts and scales
+    m = rand_mod(rng, 64)
+    m[:, 2] = m[:, 5] = 0.0
+    xc = rng.normal(size=(14, 64))
+    assert np.array_equal(oracle.block_forward_cond(xc, w, dm, m, n_cond=3), xc)
+
+
+def test_cond_block_scale_minus_one_closed_form():
+    """scale_attn = -1 replaces every normed row by its class's shift, so the
+    attention input holds two distinct rows (generated: s0, condition: s1);
+    without RoPE each head's output is the softmax mix of the two value rows
+    weighted by their counts.  MLP gate 0 isolates the attention branch."""
+    dm = dims_of(2, 2, 2, 1, 16, 2, 32)
+    rng = np.random.default_rng(32)
+    Sg, C, d, H, D = 9, 4, 16, 2, 8
+    x = rng.normal(size=(Sg + C, d))
+    w = rand_block(rng, d, 32, scale=0.5)
+    m = rand_mod(rng, d)
+    m[:, 1] = -1.0
+    m[:, 5] = 0.0
+    got = oracle.block_forward_cond(x, w, dm, m, n_cond=C, rope=False)
+    wq, wk, wv = w["w_qkv"][:d], w["w_qkv"][d:2 * d], w["w_qkv"][2 * d:]
+    s0, s1 = m[0, 0], m[1, 0]
+    k0, k1, v0, v1 = wk @ s0, wk @ s1, wv @ s0, wv @ s1
+    for i in range(Sg + C):
+        cl = 1 if i >= Sg else 0
+        q = wq @ (s1 if cl else s0)
+        o = np.zeros(d)
+        for h in range(H):
+            sl = slice(h * D, h * D + D)
+            a0 = math.exp(float(q[sl] @ k0[sl]) / math.sqrt(D)) * Sg
+            a1 = math.exp(float(q[sl] @ k1[sl]) / math.sqrt(D)) * C
+            o[sl] = (a0 * v0[sl] + a1 * v1[sl]) / (a0 + a1)
+        ref = x[i] + m[cl, 2] * (w["w_o"] @ o)
+        assert np.allclose(got[i], ref, rtol=1e-12, atol=1e-13)
+
+
+def test_cond_rows_unrotated_and_gated_by_their_class():
+    dm = dims_of(2, 2, 4, 3, 32, 2, 64)
+    rng = np.random.default_rng(33)
+    Sg, C = 19, 5
+    x = rng.normal(size=(Sg + C, 32))
+    w = rand_block(rng, 32, 64)
+    m = rand_mod(rng, 32)
+    # condition rows carry no position: permuting them permutes their outputs
+    # and leaves the generated rows unchanged (RoPE on)
+    perm = np.concatenate([np.arange(Sg), Sg + rng.permutation(C)])
+    a = oracle.block_forward_cond(x, w, dm, m, n_cond=C)
+    b = oracle.block_forward_cond(x[perm], w, dm, m, n_cond=C)
+    assert np.allclose(a[perm], b, rtol=1e-12, atol=1e-13)
+    # class-1 gates 0: condition rows pass through, generated rows still see them
+    m1 = m.copy()
+    m1[1, 2] = m1[1, 5] = 0.0
+    c = oracle.block_forward_cond(x, w, dm, m1, n_cond=C)
+    assert np.array_equal(c[Sg:], x[Sg:])
+    x2 = x.copy()
+    x2[Sg:] += 1.0
+    c2 = oracle.block_forward_cond(x2, w, dm, m1, n_cond=C)
+    assert not np.allclose(c2[:Sg], c[:Sg], rtol=1e-6)
+
+
+def test_cond_stack_merge_carries_condition_rows():
+    dm = dims_of(1, 2, 4, 2, 32, 2, 64)
+    rng = np.random.default_rng(34)
+    C = 3
+    x = rng.normal(size=(10 + C, 32))
+    m = oracle.token_merge(x, dm)
+    assert m.shape == (4 + 2 + C, 32) and np.array_equal(m[4:], x[8:])
+    assert np.array_equal(oracle.token_unmerge(m, dm)[8:], x[8:])
+    blocks = [rand_block(rng, 32, 64) for _ in range(3)]
+    mods = [rand_mod(rng, 32) for _ in range(3)]
+    for delta in (False, True):
+        got = oracle.stack_forward_cond(x, blocks, dm, mods, C, 1, 1, unmerge_delta=delta)
+        xm0 = oracle.token_merge(oracle.block_forward_cond(x, blocks[0], dm, mods[0], C), dm)
+        ym = oracle.block_forward_cond(xm0, blocks[1], dm, mods[1], C, merged=True)
+        x1 = oracle.block_forward_cond(x, blocks[0], dm, mods[0], C)
+        mid = oracle.token_unmerge_delta(x1, ym, xm0, dm) if delta else oracle.token_unmerge(ym, dm)
+        ref = oracle.block_forward_cond(mid, blocks[2], dm, mods[2], C)
+        assert np.allclose(got, ref, rtol=1e-13, atol=1e-14)
 
 
 # ----------------------------------------------------------------------------- token reduction
@@ -485,3 +614,41 @@ def test_denoise_core_hand_computed():
     assert nc == 2 and np.allclose(got, x3, rtol=1e-14)
     with pytest.raises(ValueError):
         oracle.denoise_core(x0, [a, b, c], dm, 3, 2, 1, 1, merge_first=0, merge_last=1, block_fn=fn)
+
+
+def test_denoise_cond_reduces_to_plain_loops():
+    dm = dims_of(1, 1, 2, 1, 4, 1, 4)
+    x0 = np.random.default_rng(35).normal(size=(3, 4))
+    fn = lambda x, w, d, merged: np.tanh(x * w)  # noqa: E731
+    fc = lambda x, w, d, mod, n_cond, merged: np.tanh(x * w)  # noqa: E731
+    ws = [0.9, 1.1, 0.7, 1.3]
+    a, na = oracle.denoise(x0, ws, dm, 7, 3, block_fn=fn)
+    b, nb, _ = oracle.denoise_cond(x0, ws, dm, 7, reuse=3, block_fn=fc)
+    assert na == nb and np.allclose(a, b, rtol=1e-15)
+    a, nc = oracle.denoise_core(x0, ws, dm, 6, 4, 1, 2, block_fn=fn)
+    b, nf, nc2 = oracle.denoise_cond(x0, ws, dm, 6, core_reuse=4, core_first=1, core_last=2, block_fn=fc)
+    assert nf == 6 and nc == nc2 and np.allclose(a, b, rtol=1e-15)
+
+
+def test_denoise_cond_rows_refilled_each_evaluation():
+    """A toy block that adds the mean of the condition rows to every row: the
+    condition rows grow inside an evaluation, but each evaluation starts from
+    the given values, so the velocity of the generated rows is
+    L * x + (sum over blocks of the running condition mean) at every step."""
+    dm = dims_of(1, 1, 2, 1, 4, 1, 4)
+    rng = np.random.default_rng(36)
+    x0, cond = rng.normal(size=(3, 4)), rng.normal(size=(2, 4))
+
+    def fc(x, w, d, mod, n_cond, merged):
+        return x + x[len(x) - n_cond:].mean(axis=0)
+
+    got, nf, _ = oracle.denoise_cond(x0, [0, 0], dm, 4, cond_rows=cond, reuse=1, block_fn=fc)
+    s = oracle.sigmas(4).astype(np.float64)
+    c = cond.mean(axis=0)
+    x = x0.copy()
+    for i in range(4):
+        # block 1: rows + c; block 2: rows + (c + c) -> generated rows x + 3c
+        x = x + (s[i + 1] - s[i]) * (x + 3.0 * c)
+    assert nf == 4 and np.allclose(got, x, rtol=1e-14)
+    with pytest.raises(ValueError):
+        oracle.denoise_cond(x0, [0, 0], dm, 4, reuse=2, core_first=0, core_last=0, block_fn=fc)
