@@ -118,11 +118,15 @@ struct Plan {
   size_t rope, rope_m, xm;            // RoPE tables, merged-sequence buffer
   size_t xm0, delta;                  // merged input (delta unmerge), cached core update
   size_t total;
+  int n_cond;                         // condition rows after the audio tokens
 };
 
-Plan plan(const h3b_dims& dm, int dtype, int reduction, int keep_merged_input = 0, int core = 0) {
+// Activations cover the generated rows plus n_cond condition rows; the RoPE
+// tables cover the generated rows only (condition rows are not rotated).
+Plan plan(const h3b_dims& dm, int dtype, int reduction, int keep_merged_input = 0, int core = 0, int n_cond = 0) {
   Plan p{};
-  const size_t S = seq_len(dm, 0), d = dm.d, f = dm.ffn;
+  p.n_cond = n_cond;
+  const size_t S = seq_len(dm, 0) + n_cond, d = dm.d, f = dm.ffn;
   if (dtype == H3B_INT8) {
     p.qkv = 0;
     p.o = al256(6 * d * S);
@@ -155,11 +159,11 @@ Plan plan(const h3b_dims& dm, int dtype, int reduction, int keep_merged_input = 
   p.amax = off;
   off += al256(S * 4);
   p.rope = off;
-  off += al256(S * (dm.head_dim / 2) * 8);
+  off += al256(static_cast<size_t>(seq_len(dm, 0)) * (dm.head_dim / 2) * 8);
   if (reduction) {
-    const size_t Sm = seq_len(dm, 1);
+    const size_t Sm = seq_len(dm, 1) + n_cond;
     p.rope_m = off;
-    off += al256(Sm * (dm.head_dim / 2) * 8);
+    off += al256(static_cast<size_t>(seq_len(dm, 1)) * (dm.head_dim / 2) * 8);
     p.xm = off;
     off += al256(Sm * d * 4);
   } else {
@@ -168,7 +172,7 @@ Plan plan(const h3b_dims& dm, int dtype, int reduction, int keep_merged_input = 
   p.xm0 = p.delta = 0;
   if (reduction && keep_merged_input) {
     p.xm0 = off;
-    off += al256(static_cast<size_t>(seq_len(dm, 1)) * d * 4);
+    off += al256(static_cast<size_t>(seq_len(dm, 1) + n_cond) * d * 4);
   }
   if (core) {
     p.delta = off;
@@ -221,13 +225,37 @@ GemmArgs gemm_args(int M, int N, int K, void* C, const float* sa, const float* s
   a.full_tiles = 0;
   a.split = 1;
   a.partial = nullptr;
+  a.gate = nullptr;
+  a.gate_split = 0;
+  a.gate_stride = 0;
+  a.rope_rows = M;
   return a;
 }
 
-// One block on x [S_eff, d]; rope = table of this geometry (already filled).
+GemmArgs gated(GemmArgs a, const float* gate, int split, int stride) {
+  a.gate = gate;
+  a.gate_split = split;
+  a.gate_stride = stride;
+  return a;
+}
+
+// One block on x [S_eff + n_cond, d]; rope = table of this geometry (already
+// filled).  mod (nullable): this block's modulation [2][6][d] fp32 -- row class
+// (generated, condition) x (shift, scale, gate of the attention half, then of
+// the MLP half).
 int block_impl(const Ctx& c, const h3b_dims& dm, const h3b_block_weights& w, float* x, int merged, uint8_t* ws,
-               const Plan& p, const float* rope) {
-  const int S = seq_len(dm, merged), d = dm.d, f = dm.ffn;
+               const Plan& p, const float* rope, const float* mod = nullptr) {
+  const int Sg = seq_len(dm, merged), S = Sg + p.n_cond, d = dm.d, f = dm.ffn;
+  Mod m1, m2;
+  const float *gate1 = nullptr, *gate2 = nullptr;
+  if (mod) {
+    m1 = Mod{mod, mod + d, Sg, 6 * d};
+    m2 = Mod{mod + 3 * d, mod + 4 * d, Sg, 6 * d};
+    gate1 = mod + 2 * d;
+    gate2 = mod + 5 * d;
+  }
+  GemmArgs qkv_args = gemm_args(S, 3 * d, d, nullptr, nullptr, nullptr, rope, dm, nullptr, c.err);
+  qkv_args.rope_rows = Sg;
   uint8_t* A = ws;
   void* qkv = A + p.qkv;
   void* o = A + p.o;
@@ -236,43 +264,49 @@ int block_impl(const Ctx& c, const h3b_dims& dm, const h3b_block_weights& w, flo
   void* g = A + p.g;
   float* s_act = reinterpret_cast<float*>(ws + p.s_act);
   if (w.dtype == H3B_BF16) {
-    H3B_CU(KID_RMSNORM, launch_rmsnorm(c, x, w.g_attn, S, d, dm.eps, u1, nullptr, 0));
-    H3B_CU(KID_GEMM_QKV, launch_gemm(c, u1, w.w_qkv, 0, H3B_EPI_QKV_ROPE,
-                                     gemm_args(S, 3 * d, d, qkv, nullptr, nullptr, rope, dm, nullptr, c.err)));
+    H3B_CU(KID_RMSNORM, launch_rmsnorm(c, x, w.g_attn, S, d, dm.eps, u1, nullptr, 0, m1));
+    qkv_args.C = qkv;
+    H3B_CU(KID_GEMM_QKV, launch_gemm(c, u1, w.w_qkv, 0, H3B_EPI_QKV_ROPE, qkv_args));
     // the norm-1 arena is dead once the QKV GEMM has run: key-split attention partials
     H3B_CU(KID_ATTN, launch_attention(c, qkv, S, dm.n_heads, dm.head_dim, o, reinterpret_cast<float*>(u1),
                                       2 * static_cast<size_t>(d) * S));
     // O-proj: the dead QKV arena holds split-K partials; FC2: the dead MLP-input arena
     H3B_CU(KID_GEMM_O, launch_gemm(c, o, w.w_o, 0, H3B_EPI_RESID,
-                                   gemm_args(S, d, d, x, nullptr, nullptr, nullptr, dm, nullptr, c.err),
+                                   gated(gemm_args(S, d, d, x, nullptr, nullptr, nullptr, dm, nullptr, c.err), gate1,
+                                         Sg, 6 * d),
                                    reinterpret_cast<float*>(A + p.qkv), p.o - p.qkv));
-    H3B_CU(KID_RMSNORM, launch_rmsnorm(c, x, w.g_mlp, S, d, dm.eps, u2, nullptr, 0));
+    H3B_CU(KID_RMSNORM, launch_rmsnorm(c, x, w.g_mlp, S, d, dm.eps, u2, nullptr, 0, m2));
     H3B_CU(KID_GEMM_FC1, launch_gemm(c, u2, w.w_fc1, 0, H3B_EPI_GELU,
                                      gemm_args(S, f, d, g, nullptr, nullptr, nullptr, dm, nullptr, c.err)));
     H3B_CU(KID_GEMM_FC2, launch_gemm(c, g, w.w_fc2, 0, H3B_EPI_RESID,
-                                     gemm_args(S, d, f, x, nullptr, nullptr, nullptr, dm, nullptr, c.err),
+                                     gated(gemm_args(S, d, f, x, nullptr, nullptr, nullptr, dm, nullptr, c.err),
+                                           gate2, Sg, 6 * d),
                                      reinterpret_cast<float*>(A + p.u2), p.g - p.u2));
   } else {
     int8_t* oq = reinterpret_cast<int8_t*>(A + p.oq);
     int8_t* gq = reinterpret_cast<int8_t*>(A + p.gq);
     float* s_g = reinterpret_cast<float*>(ws + p.s_g);
     float* amax = reinterpret_cast<float*>(ws + p.amax);
-    H3B_CU(KID_RMSNORM, launch_rmsnorm(c, x, w.g_attn, S, d, dm.eps, u1, s_act, 1));
-    H3B_CU(KID_GEMM_QKV, launch_gemm(c, u1, w.w_qkv, 1, H3B_EPI_QKV_ROPE,
-                                     gemm_args(S, 3 * d, d, qkv, s_act, w.s_qkv, rope, dm, nullptr, c.err)));
+    H3B_CU(KID_RMSNORM, launch_rmsnorm(c, x, w.g_attn, S, d, dm.eps, u1, s_act, 1, m1));
+    qkv_args.C = qkv;
+    qkv_args.sa = s_act;
+    qkv_args.sb = w.s_qkv;
+    H3B_CU(KID_GEMM_QKV, launch_gemm(c, u1, w.w_qkv, 1, H3B_EPI_QKV_ROPE, qkv_args));
     H3B_CU(KID_ATTN, launch_attention(c, qkv, S, dm.n_heads, dm.head_dim, o, reinterpret_cast<float*>(u1),
                                       static_cast<size_t>(d) * S));
     H3B_CU(KID_QUANT_ROWS, launch_quant_rows(c, o, S, d, oq, s_act));
     H3B_CU(KID_GEMM_O, launch_gemm(c, oq, w.w_o, 1, H3B_EPI_RESID,
-                                   gemm_args(S, d, d, x, s_act, w.s_o, nullptr, dm, nullptr, c.err),
+                                   gated(gemm_args(S, d, d, x, s_act, w.s_o, nullptr, dm, nullptr, c.err), gate1, Sg,
+                                         6 * d),
                                    reinterpret_cast<float*>(A + p.qkv), p.o - p.qkv));
-    H3B_CU(KID_RMSNORM, launch_rmsnorm(c, x, w.g_mlp, S, d, dm.eps, u2, s_act, 1));
+    H3B_CU(KID_RMSNORM, launch_rmsnorm(c, x, w.g_mlp, S, d, dm.eps, u2, s_act, 1, m2));
     H3B_CU(KID_MEMSET, cudaMemsetAsync(amax, 0, sizeof(float) * S, c.stream));
     H3B_CU(KID_GEMM_FC1, launch_gemm(c, u2, w.w_fc1, 1, H3B_EPI_GELU,
                                      gemm_args(S, f, d, g, s_act, w.s_fc1, nullptr, dm, amax, c.err)));
     H3B_CU(KID_QUANT_ABSMAX, launch_quant_absmax(c, g, amax, S, f, gq, s_g));
     H3B_CU(KID_GEMM_FC2, launch_gemm(c, gq, w.w_fc2, 1, H3B_EPI_RESID,
-                                     gemm_args(S, d, f, x, s_g, w.s_fc2, nullptr, dm, nullptr, c.err),
+                                     gated(gemm_args(S, d, f, x, s_g, w.s_fc2, nullptr, dm, nullptr, c.err), gate2,
+                                           Sg, 6 * d),
                                      reinterpret_cast<float*>(A + p.u2), p.g - p.u2));
   }
   return H3B_OK;
@@ -287,37 +321,41 @@ int fill_rope(const Ctx& c, const h3b_dims& dm, uint8_t* ws, const Plan& p, int 
 // Blocks lo..hi on x; the token-reduction window [mf, ml] is applied when it
 // lies inside [lo, hi] (merge before mf, unmerge after ml; udelta selects the
 // delta-broadcast unmerge).  RoPE tables must be filled.
+// mod (nullable): [n_blocks][2][6][d] for blocks 0.. of the whole stack.
 int run_blocks(const Ctx& c, const h3b_dims& dm, const h3b_block_weights* blocks, int lo, int hi, int mf, int ml,
-               int udelta, float* x, uint8_t* ws, const Plan& p) {
+               int udelta, float* x, uint8_t* ws, const Plan& p, const float* mod = nullptr) {
   const bool on = mf >= 0 && lo <= mf && ml <= hi;
   float* rope = reinterpret_cast<float*>(ws + p.rope);
   float* rope_m = on ? reinterpret_cast<float*>(ws + p.rope_m) : nullptr;
   float* xm = on ? reinterpret_cast<float*>(ws + p.xm) : nullptr;
   float* xm0 = on && udelta ? reinterpret_cast<float*>(ws + p.xm0) : nullptr;
   const int V = dm.frames * dm.rows * dm.cols;
+  const int tail = dm.n_audio + p.n_cond;  // rows after the video rows, carried through the reduction
   for (int l = lo; l <= hi; ++l) {
-    if (on && l == mf) H3B_CU(KID_MERGE, launch_merge(c, x, xm, V, dm.n_audio, dm.d, xm0));
+    if (on && l == mf) H3B_CU(KID_MERGE, launch_merge(c, x, xm, V, tail, dm.d, xm0));
     const bool merged = on && l >= mf && l <= ml;
-    H3B_TRY(block_impl(c, dm, blocks[l], merged ? xm : x, merged, ws, p, merged ? rope_m : rope));
+    H3B_TRY(block_impl(c, dm, blocks[l], merged ? xm : x, merged, ws, p, merged ? rope_m : rope,
+                       mod ? mod + static_cast<size_t>(l) * 12 * dm.d : nullptr));
     if (on && l == ml) {
       if (udelta)
-        H3B_CU(KID_UNMERGE_DELTA, launch_unmerge_delta(c, x, xm, xm0, V, dm.n_audio, dm.d));
+        H3B_CU(KID_UNMERGE_DELTA, launch_unmerge_delta(c, x, xm, xm0, V, tail, dm.d));
       else
-        H3B_CU(KID_UNMERGE, launch_unmerge(c, xm, x, V, dm.n_audio, dm.d));
+        H3B_CU(KID_UNMERGE, launch_unmerge(c, xm, x, V, tail, dm.d));
     }
   }
   return H3B_OK;
 }
 
 int stack_impl(const Ctx& c, const h3b_dims& dm, const h3b_block_weights* blocks, int n_blocks, int mf, int ml,
-               float* x, uint8_t* ws, const Plan& p, int udelta = 0) {
+               float* x, uint8_t* ws, const Plan& p, int udelta = 0, const float* mod = nullptr) {
   H3B_TRY(fill_rope(c, dm, ws, p, mf >= 0));
-  return run_blocks(c, dm, blocks, 0, n_blocks - 1, mf, ml, udelta, x, ws, p);
+  return run_blocks(c, dm, blocks, 0, n_blocks - 1, mf, ml, udelta, x, ws, p, mod);
 }
 
 int check_stack_args(const h3b_dims* dims, const h3b_block_weights* blocks, int n_blocks, int mf, int ml, float* x,
-                     void* ws, size_t ws_bytes, Plan* out, int udelta = 0, int cf = -1, int cl = -1) {
+                     void* ws, size_t ws_bytes, Plan* out, int udelta = 0, int cf = -1, int cl = -1, int n_cond = 0) {
   H3B_TRY(check_dims(dims));
+  if (n_cond < 0 || seq_len(*dims, 0) + static_cast<long long>(n_cond) > (1LL << 24)) return H3B_ERR_DIMS;
   if (!blocks || !x || !ws) return H3B_ERR_NULL;
   if (!aligned16(x) || !aligned16(ws)) return H3B_ERR_ALIGN;
   if (n_blocks < 0) return H3B_ERR_DIMS;
@@ -332,7 +370,7 @@ int check_stack_args(const h3b_dims* dims, const h3b_block_weights* blocks, int 
     // the reduction window lies inside the core window or outside it
     if (mf >= 0 && !(cf <= mf && ml <= cl) && !(ml < cf || mf > cl)) return H3B_ERR_DIMS;
   }
-  *out = plan(*dims, dtype, mf >= 0, mf >= 0 && udelta, cf >= 0);
+  *out = plan(*dims, dtype, mf >= 0, mf >= 0 && udelta, cf >= 0, n_cond);
   if (ws_bytes < out->total) return H3B_ERR_WORKSPACE;
   return H3B_OK;
 }
@@ -341,30 +379,40 @@ int check_stack_args(const h3b_dims* dims, const h3b_block_weights* blocks, int 
 // i % reuse == 0 or the last one.  Core reuse (cf >= 0, reuse == 1): the core
 // blocks run on steps with i % core_reuse == 0 or the last one; their update
 // is cached (as its negative, in ws at p.delta) and added on the other steps.
+// Condition rows (p.n_cond): v holds [generated ; condition] rows; every
+// evaluation refills the condition rows from cond, the Euler update covers
+// the generated rows only.  mod: [mod_steps][n_blocks][2][6][d] or NULL.
 int denoise_impl(const Ctx& c, const h3b_dims& dm, const h3b_block_weights* blocks, int n_blocks, int mf, int ml,
                  int udelta, int cf, int cl, int n_steps, int reuse, int core_reuse, float* x, float* v, uint8_t* ws,
-                 const Plan& p, int* n_fresh, int* n_core) {
-  const size_t n = static_cast<size_t>(seq_len(dm, 0)) * dm.d;
+                 const Plan& p, int* n_fresh, int* n_core, const float* cond = nullptr, const float* mod = nullptr,
+                 int mod_steps = 1) {
+  const size_t n = static_cast<size_t>(seq_len(dm, 0)) * dm.d;    // generated rows
+  const size_t n_all = n + static_cast<size_t>(p.n_cond) * dm.d;  // + condition rows
   auto fresh = [&](int i, int r) { return i % r == 0 || i == n_steps - 1; };
   float* neg_delta = cf >= 0 ? reinterpret_cast<float*>(ws + p.delta) : nullptr;
+  const size_t mod_step = static_cast<size_t>(n_blocks) * 12 * dm.d;
   int count = 0, core_count = 0;
   H3B_TRY(fill_rope(c, dm, ws, p, mf >= 0));
   H3B_CU(KID_COPY, cudaMemcpyAsync(v, x, n * sizeof(float), cudaMemcpyDeviceToDevice, c.stream));
   for (int i = 0; i < n_steps; ++i) {
+    const float* m = mod ? mod + (mod_steps > 1 ? static_cast<size_t>(i) * mod_step : 0) : nullptr;
     if (fresh(i, reuse)) {
+      if (p.n_cond)
+        H3B_CU(KID_COPY,
+               cudaMemcpyAsync(v + n, cond, (n_all - n) * sizeof(float), cudaMemcpyDeviceToDevice, c.stream));
       if (cf < 0) {
-        H3B_TRY(run_blocks(c, dm, blocks, 0, n_blocks - 1, mf, ml, udelta, v, ws, p));
+        H3B_TRY(run_blocks(c, dm, blocks, 0, n_blocks - 1, mf, ml, udelta, v, ws, p, m));
       } else {
-        H3B_TRY(run_blocks(c, dm, blocks, 0, cf - 1, mf, ml, udelta, v, ws, p));
+        H3B_TRY(run_blocks(c, dm, blocks, 0, cf - 1, mf, ml, udelta, v, ws, p, m));
         if (fresh(i, core_reuse)) {
-          H3B_CU(KID_COPY, cudaMemcpyAsync(neg_delta, v, n * sizeof(float), cudaMemcpyDeviceToDevice, c.stream));
-          H3B_TRY(run_blocks(c, dm, blocks, cf, cl, mf, ml, udelta, v, ws, p));
-          H3B_CU(KID_FLOW, launch_flow_step(c, neg_delta, v, -1.0f, n, nullptr));  // input - output
+          H3B_CU(KID_COPY, cudaMemcpyAsync(neg_delta, v, n_all * sizeof(float), cudaMemcpyDeviceToDevice, c.stream));
+          H3B_TRY(run_blocks(c, dm, blocks, cf, cl, mf, ml, udelta, v, ws, p, m));
+          H3B_CU(KID_FLOW, launch_flow_step(c, neg_delta, v, -1.0f, n_all, nullptr));  // input - output
           ++core_count;
         } else {
-          H3B_CU(KID_FLOW, launch_flow_step(c, v, neg_delta, -1.0f, n, nullptr));  // + cached update
+          H3B_CU(KID_FLOW, launch_flow_step(c, v, neg_delta, -1.0f, n_all, nullptr));  // + cached update
         }
-        H3B_TRY(run_blocks(c, dm, blocks, cl + 1, n_blocks - 1, mf, ml, udelta, v, ws, p));
+        H3B_TRY(run_blocks(c, dm, blocks, cl + 1, n_blocks - 1, mf, ml, udelta, v, ws, p, m));
       }
       ++count;
     }
@@ -411,6 +459,18 @@ bool encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, int elem_bytes,
 }  // namespace h3b
 
 using namespace h3b;
+
+// Options of the extended entry points: the condition-row count and the
+// modulation array (16-byte aligned; mod_steps >= 1 slices of [n_blocks][2][6][d]).
+static int check_opts(const h3b_stack_opts* o) {
+  if (!o) return H3B_ERR_NULL;
+  if (o->n_cond < 0) return H3B_ERR_DIMS;
+  if (o->modulation) {
+    if (!aligned16(o->modulation)) return H3B_ERR_ALIGN;
+    if (o->mod_steps < 1) return H3B_ERR_DIMS;
+  }
+  return H3B_OK;
+}
 
 // ====================================================================== C ABI
 extern "C" {
@@ -491,39 +551,47 @@ int h3b_denoise(const h3b_dims* dims, const h3b_block_weights* blocks, int n_blo
 
 size_t h3b_workspace_bytes_ex(const h3b_dims* dims, int dtype, const h3b_stack_opts* o) {
   if (!o || check_dims(dims) != H3B_OK || (dtype != H3B_BF16 && dtype != H3B_INT8)) return 0;
+  if (check_opts(o) != H3B_OK) return 0;
   const int red = o->merge_first >= 0;
   if (red && (dims->cols & 1)) return 0;
-  return plan(*dims, dtype, red, red && o->unmerge_delta, o->core_first >= 0).total;
+  return plan(*dims, dtype, red, red && o->unmerge_delta, o->core_first >= 0, o->n_cond).total;
 }
 
 int h3b_stack_forward_ex(const h3b_dims* dims, const h3b_block_weights* blocks, int n_blocks,
                          const h3b_stack_opts* o, float* x, void* ws, size_t ws_bytes, void* stream) {
   if (!o) return H3B_ERR_NULL;
+  H3B_TRY(check_opts(o));
   Plan p;
   H3B_TRY(check_stack_args(dims, blocks, n_blocks, o->merge_first, o->merge_last, x, ws, ws_bytes, &p,
-                           o->unmerge_delta));
+                           o->unmerge_delta, -1, -1, o->n_cond));
   Ctx c;
   H3B_TRY(device_ctx(static_cast<cudaStream_t>(stream), &c));
   return stack_impl(c, *dims, blocks, n_blocks, o->merge_first, o->merge_last, x, static_cast<uint8_t*>(ws), p,
-                    o->unmerge_delta);
+                    o->unmerge_delta, o->modulation);
 }
 
 int h3b_denoise_ex(const h3b_dims* dims, const h3b_block_weights* blocks, int n_blocks, const h3b_stack_opts* o,
                    int n_steps, int reuse, int core_reuse, float* x, float* v, void* ws, size_t ws_bytes,
                    int* n_fresh, int* n_core_fresh, void* stream) {
   if (!o) return H3B_ERR_NULL;
+  H3B_TRY(check_opts(o));
   Plan p;
   H3B_TRY(check_stack_args(dims, blocks, n_blocks, o->merge_first, o->merge_last, x, ws, ws_bytes, &p,
-                           o->unmerge_delta, o->core_first, o->core_last));
+                           o->unmerge_delta, o->core_first, o->core_last, o->n_cond));
   if (!v) return H3B_ERR_NULL;
   if (!aligned16(v)) return H3B_ERR_ALIGN;
   if (n_steps <= 0 || reuse <= 0 || core_reuse <= 0) return H3B_ERR_DIMS;
   if (o->core_first >= 0 && reuse != 1) return H3B_ERR_DIMS;  // core reuse excludes whole-velocity reuse
+  if (o->modulation && o->mod_steps != 1 && o->mod_steps != n_steps) return H3B_ERR_DIMS;
+  if (o->n_cond > 0) {
+    if (!o->cond_rows) return H3B_ERR_NULL;
+    if (!aligned16(o->cond_rows)) return H3B_ERR_ALIGN;
+  }
   Ctx c;
   H3B_TRY(device_ctx(static_cast<cudaStream_t>(stream), &c));
   return denoise_impl(c, *dims, blocks, n_blocks, o->merge_first, o->merge_last, o->unmerge_delta, o->core_first,
                       o->core_last, n_steps, reuse, core_reuse, x, v, static_cast<uint8_t*>(ws), p, n_fresh,
-                      n_core_fresh);
+                      n_core_fresh, o->cond_rows, o->modulation, o->modulation ? o->mod_steps : 1);
 }
 
 int h3b_quantize_weights(const void* w, int rows, int k, int8_t* q, float* scale, void* stream) {

@@ -106,6 +106,21 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& p, int m, int n, 
   }
   if (EPI == H3B_EPI_RESID) {
     float4* c = reinterpret_cast<float4*>(static_cast<float*>(p.C) + off);
+    if (p.gate) {  // gated residual update
+      const float4* g4 =
+          reinterpret_cast<const float4*>(p.gate + (m >= p.gate_split ? static_cast<size_t>(p.gate_stride) : 0) + n);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float4 g = __ldg(g4 + i);
+        float4 a = c[i];
+        a.x = fmaf(g.x, v[4 * i], a.x);
+        a.y = fmaf(g.y, v[4 * i + 1], a.y);
+        a.z = fmaf(g.z, v[4 * i + 2], a.z);
+        a.w = fmaf(g.w, v[4 * i + 3], a.w);
+        c[i] = a;
+      }
+      return;
+    }
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       float4 a = c[i];
@@ -118,7 +133,7 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& p, int m, int n, 
     return;
   }
   if (EPI == H3B_EPI_QKV_ROPE) {
-    if (n < 2 * p.d) {  // Q or K column block: rotate its 16 interleaved pairs
+    if (n < 2 * p.d && m < p.rope_rows) {  // Q or K column block: rotate its 16 interleaved pairs
       const int j0 = (n % p.head_dim) >> 1;
       const float4* t4 = reinterpret_cast<const float4*>(p.rope + static_cast<size_t>(m) * (p.head_dim >> 1) + j0);
 #pragma unroll
@@ -335,7 +350,8 @@ __global__ void __launch_bounds__(THREADS, 1)
 // (deterministic).  One CTA per (tail tile, row), one thread per column.
 template <int TM>
 __global__ void __launch_bounds__(BN) k_splitk_add(float* __restrict__ C, const float* __restrict__ partial, int M,
-                                                   int N, int full_tiles, int split, int num_m, int num_n) {
+                                                   int N, int full_tiles, int split, int num_m, int num_n,
+                                                   const float* __restrict__ gate, int gate_split, int gate_stride) {
   const int i = blockIdx.x / TM, r = blockIdx.x % TM, col = threadIdx.x;
   int mb, nb;
   tile_coords(full_tiles + i, num_m, num_n, mb, nb);
@@ -344,7 +360,11 @@ __global__ void __launch_bounds__(BN) k_splitk_add(float* __restrict__ C, const 
   const float* src = partial + static_cast<size_t>(i) * split * (TM * BN) + r * BN + col;
   float acc = 0.f;
   for (int q = 0; q < split; ++q) acc += src[static_cast<size_t>(q) * (TM * BN)];
-  C[static_cast<size_t>(m) * N + n] += acc;
+  if (gate)
+    C[static_cast<size_t>(m) * N + n] =
+        fmaf(gate[(m >= gate_split ? static_cast<size_t>(gate_stride) : 0) + n], acc, C[static_cast<size_t>(m) * N + n]);
+  else
+    C[static_cast<size_t>(m) * N + n] += acc;
 }
 
 // ---------------------------------------------------------------------------
@@ -711,10 +731,12 @@ cudaError_t launch_gemm(const Ctx& c, const void* A, const void* B, int ab_int8,
   if (e != cudaSuccess || args.split <= 1) return e;
   if (pair)
     k_splitk_add<BM2><<<rem * BM2, BN, 0, c.stream>>>(static_cast<float*>(args.C), args.partial, args.M, args.N,
-                                                      args.full_tiles, args.split, num_m, num_n);
+                                                      args.full_tiles, args.split, num_m, num_n, args.gate,
+                                                      args.gate_split, args.gate_stride);
   else
     k_splitk_add<BM><<<rem * BM, BN, 0, c.stream>>>(static_cast<float*>(args.C), args.partial, args.M, args.N,
-                                                    args.full_tiles, args.split, num_m, num_n);
+                                                    args.full_tiles, args.split, num_m, num_n, args.gate,
+                                                    args.gate_split, args.gate_stride);
   return cudaGetLastError();
 }
 

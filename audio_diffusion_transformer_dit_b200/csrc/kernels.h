@@ -45,8 +45,16 @@ cudaError_t launch_unmerge_delta(const Ctx& c, float* x, const float* ym, const 
                                  int d);
 cudaError_t launch_unmerge(const Ctx& c, const float* xm, float* x, int n_video, int n_audio, int d);
 cudaError_t launch_rope_table(const Ctx& c, const h3b_dims& dm, int merged, float* table);
+// adaLN-style modulation of a normed row, y <- y * (1 + scale[k]) + shift[k]
+// for k < d; rows >= split (the condition rows) read their vectors at +stride.
+// shift == nullptr: no modulation.
+struct Mod {
+  const float* shift = nullptr;
+  const float* scale = nullptr;
+  int split = 0, stride = 0;
+};
 cudaError_t launch_rmsnorm(const Ctx& c, const float* x, const float* g, int rows, int d, float eps, void* out,
-                           float* out_scale, int out_int8);
+                           float* out_scale, int out_int8, const Mod& mod = Mod{});
 cudaError_t launch_quant_rows(const Ctx& c, const void* a, int rows, int k, int8_t* q, float* s);
 cudaError_t launch_quant_absmax(const Ctx& c, const void* a, const float* absmax, int rows, int k, int8_t* q,
                                 float* s);
@@ -63,6 +71,11 @@ struct GemmArgs {
   // split-K of the tail tiles (residual epilogue only; set by launch_gemm)
   int full_tiles, split;
   float* partial;
+  // residual epilogue: C += gate[n] * acc when gate is set (rows >= gate_split
+  // read the gate at +gate_stride); QKV epilogue: rows >= rope_rows are not rotated
+  const float* gate;
+  int gate_split, gate_stride;
+  int rope_rows;
 };
 
 // A [M,K], B [N,K] K-major (bf16 or int8); C per epilogue.  scratch (may be

@@ -190,7 +190,8 @@ __global__ void k_rope_table(float2* __restrict__ table, int F, int H, int Wc, i
 // the output pass (x is read from HBM exactly once).
 template <int VPT, bool INT8>
 __global__ void __launch_bounds__(kThreads) k_rmsnorm(const float* __restrict__ x, const float* __restrict__ g, int d,
-                                                      float eps, void* __restrict__ out, float* __restrict__ out_scale) {
+                                                      float eps, void* __restrict__ out, float* __restrict__ out_scale,
+                                                      const Mod mod) {
   __shared__ float red[32];
   const int row = blockIdx.x, d4 = d >> 2;
   const float4* xr = reinterpret_cast<const float4*>(x + static_cast<size_t>(row) * d);
@@ -209,6 +210,9 @@ __global__ void __launch_bounds__(kThreads) k_rmsnorm(const float* __restrict__ 
   }
   ss = block_reduce<false>(ss, red);
   const float r = 1.0f / sqrtf(ss / static_cast<float>(d) + eps);
+  const size_t cls = mod.shift && row >= mod.split ? static_cast<size_t>(mod.stride) : 0;
+  const float4* sh4 = reinterpret_cast<const float4*>(mod.shift + cls);
+  const float4* sc4 = reinterpret_cast<const float4*>(mod.scale + cls);
   float amax = 0.f;
 #pragma unroll
   for (int i = 0; i < VPT; ++i) {
@@ -219,6 +223,13 @@ __global__ void __launch_bounds__(kThreads) k_rmsnorm(const float* __restrict__ 
       v[i].y = v[i].y * r * gg.y;
       v[i].z = v[i].z * r * gg.z;
       v[i].w = v[i].w * r * gg.w;
+      if (mod.shift) {
+        const float4 sh = __ldg(sh4 + c), sc = __ldg(sc4 + c);
+        v[i].x = fmaf(v[i].x, 1.0f + sc.x, sh.x);
+        v[i].y = fmaf(v[i].y, 1.0f + sc.y, sh.y);
+        v[i].z = fmaf(v[i].z, 1.0f + sc.z, sh.z);
+        v[i].w = fmaf(v[i].w, 1.0f + sc.w, sh.w);
+      }
       if (INT8) amax = fmaxf(amax, fmaxf(fmaxf(fabsf(v[i].x), fabsf(v[i].y)), fmaxf(fabsf(v[i].z), fabsf(v[i].w))));
       else {
         uint2 p;
@@ -404,7 +415,7 @@ cudaError_t launch_rope_table(const Ctx& c, const h3b_dims& dm, int merged, floa
 }
 
 cudaError_t launch_rmsnorm(const Ctx& c, const float* x, const float* g, int rows, int d, float eps, void* out,
-                           float* out_scale, int out_int8) {
+                           float* out_scale, int out_int8, const Mod& mod) {
   if (rows == 0) return cudaSuccess;
   const int d4 = d / 4;
   int threads = d4 >= kThreads ? kThreads : ((d4 + 31) / 32) * 32;
@@ -412,9 +423,9 @@ cudaError_t launch_rmsnorm(const Ctx& c, const float* x, const float* g, int row
 #define H3B_NORM_CASE(V)                                                                                  \
   case V:                                                                                                 \
     if (out_int8)                                                                                         \
-      k_rmsnorm<V, true><<<rows, threads, 0, c.stream>>>(x, g, d, eps, out, out_scale);                   \
+      k_rmsnorm<V, true><<<rows, threads, 0, c.stream>>>(x, g, d, eps, out, out_scale, mod);              \
     else                                                                                                  \
-      k_rmsnorm<V, false><<<rows, threads, 0, c.stream>>>(x, g, d, eps, out, out_scale);                  \
+      k_rmsnorm<V, false><<<rows, threads, 0, c.stream>>>(x, g, d, eps, out, out_scale, mod);             \
     break;
   switch (vpt) {
     H3B_NORM_CASE(1) H3B_NORM_CASE(2) H3B_NORM_CASE(3) H3B_NORM_CASE(4)

@@ -41,7 +41,7 @@ class BlockWeights(ctypes.Structure):
 
 class StackOpts(ctypes.Structure):
     _fields_ = [("merge_first", _i), ("merge_last", _i), ("unmerge_delta", _i), ("core_first", _i),
-                ("core_last", _i)]
+                ("core_last", _i), ("n_cond", _i), ("mod_steps", _i), ("cond_rows", _p), ("modulation", _p)]
 
 
 _SIGS = {
@@ -263,8 +263,23 @@ def denoise(dims: Dims, blocks: Sequence[Block], x: torch.Tensor, v: torch.Tenso
 
 
 def stack_opts(merge_first: int = -1, merge_last: int = -1, unmerge_delta: bool = False, core_first: int = -1,
-               core_last: int = -1) -> StackOpts:
-    return StackOpts(merge_first, merge_last, int(unmerge_delta), core_first, core_last)
+               core_last: int = -1, n_cond: int = 0, cond_rows: Optional[torch.Tensor] = None,
+               modulation: Optional[torch.Tensor] = None) -> StackOpts:
+    """Options of the extended entry points.  cond_rows: fp32 [n_cond, d]
+    (the loop's fixed condition rows); modulation: fp32 [n_blocks, 2, 6, d]
+    (every step) or [n_steps, n_blocks, 2, 6, d] (one slice per step).  The
+    tensors are kept referenced by the returned object."""
+    if cond_rows is not None and n_cond == 0:
+        n_cond = cond_rows.shape[0]
+    mod_steps = 0
+    if modulation is not None:
+        if modulation.dim() not in (4, 5) or tuple(modulation.shape[-3:-1]) != (2, 6):
+            raise ValueError("modulation must be [n_blocks, 2, 6, d] or [n_steps, n_blocks, 2, 6, d]")
+        mod_steps = modulation.shape[0] if modulation.dim() == 5 else 1
+    o = StackOpts(merge_first, merge_last, int(unmerge_delta), core_first, core_last, n_cond, mod_steps,
+                  _ptr(cond_rows, torch.float32, "cond_rows"), _ptr(modulation, torch.float32, "modulation"))
+    o._keep = (cond_rows, modulation)
+    return o
 
 
 def workspace_ex(dims: Dims, opts: StackOpts, dtype: int = BF16, device="cuda") -> torch.Tensor:

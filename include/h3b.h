@@ -144,26 +144,53 @@ int h3b_denoise(const h3b_dims* dims, const h3b_block_weights* blocks, int n_blo
                 float* x, float* v, void* ws, size_t ws_bytes, int* n_fresh, void* stream);
 
 /* Options of the extended stack / loop entry points: a delta-broadcast
- * unmerge and core residual reuse.  The siami.tw article's control table names
- * the core-reuse knob (--core-reuse 1/4/6, exclusive with whole-velocity
- * reuse) but not its arithmetic, and no page gives an unmerge rule; the forms
- * below are the plainest readings.
+ * unmerge, core residual reuse, fixed condition rows and timestep
+ * modulation.  The siami.tw article's control table names the core-reuse knob
+ * (--core-reuse 1/4/6, exclusive with whole-velocity reuse) but not its
+ * arithmetic, its file list names "0.999 condition augmentation + fixed
+ * condition rows" without a form, and no page gives an unmerge rule; the
+ * forms below are the plainest readings.  Zero-initialise the struct: every
+ * field's zero (with merge_first = core_first = -1) is "off".
  *   merge_first, merge_last: token-reduction window (inclusive, 0-indexed),
  *     merge_first = -1 turns it off.
  *   unmerge_delta: 0 = broadcast each merged token back to both columns;
  *     1 = pre-merge tokens plus the merged blocks' update broadcast:
- *     x(f,r,c) = x_pre(f,r,c) + (y - m)(f,r,c/2); audio rows take y.
+ *     x(f,r,c) = x_pre(f,r,c) + (y - m)(f,r,c/2); the rows after the
+ *     video rows (audio, condition) take y.
  *   core_first, core_last: core window for h3b_denoise_ex (-1 = off); the
  *     reduction window must lie inside it or outside it.  Ignored by
- *     h3b_stack_forward_ex. */
+ *     h3b_stack_forward_ex.
+ *   n_cond: condition rows appended after the audio tokens (0 = none).  They
+ *     take part in every block (joint attention) without rotary embedding.
+ *     h3b_stack_forward_ex: x is [S + n_cond, d] (S = h3b_seq_len).
+ *     h3b_denoise_ex: x is [S, d] (the generated rows), v is [S + n_cond, d],
+ *     and cond_rows [n_cond, d] fp32 (device, 16-byte aligned; already
+ *     augmented) are copied into v before every evaluation; the Euler update
+ *     covers the S generated rows only.
+ *   modulation (NULL = none): fp32 device array, 16-byte aligned, of
+ *     mod_steps slices of [n_blocks][2][6][d]: per block, per row class
+ *     (0 = generated rows, 1 = condition rows), the vectors shift_attn,
+ *     scale_attn, gate_attn, shift_mlp, scale_mlp, gate_mlp.  The block becomes
+ *       u  = RMSNorm(x) * (1 + scale_attn) + shift_attn  (QKV GEMM input)
+ *       x += gate_attn * (O-proj output)
+ *       u2 = RMSNorm(x) * (1 + scale_mlp) + shift_mlp    (FC1 GEMM input)
+ *       x += gate_mlp * (FC2 output).
+ *     h3b_stack_forward_ex reads slice 0; h3b_denoise_ex reads slice i at
+ *     step i when mod_steps == n_steps, slice 0 at every step when it is 1
+ *     (any other value: H3B_ERR_DIMS). */
 typedef struct h3b_stack_opts {
   int merge_first, merge_last;
   int unmerge_delta;
   int core_first, core_last;
+  int n_cond;
+  int mod_steps;
+  const float* cond_rows;
+  const float* modulation;
 } h3b_stack_opts;
 
-/* Workspace bytes for the extended entry points (adds the saved merged input
- * for unmerge_delta and the cached core update [S, d] fp32 for core reuse). */
+/* Workspace bytes for the extended entry points (sized for S + n_cond rows;
+ * adds the saved merged input for unmerge_delta and the cached core update
+ * [S + n_cond, d] fp32 for core reuse). */
 size_t h3b_workspace_bytes_ex(const h3b_dims* dims, int dtype, const h3b_stack_opts* opts);
 
 /* h3b_stack_forward with the options above. */

@@ -124,3 +124,35 @@ def test_extended_options_argument_errors():
     small = h3b.workspace_bytes(dm)
     assert dn(ctypes.byref(dm), arr, 4, ctypes.byref(o), 20, 1, 4, fake, fake, fake, small, None, None, None) == -5
     assert h3b.lib.h3b_stack_forward_ex(ctypes.byref(dm), arr, 4, None, fake, fake, need, None) == -1
+
+
+def test_condition_rows_and_modulation_argument_errors():
+    """Every case here fails validation before anything is launched."""
+    dm = h3b.dims_of(wlmod.WORKLOADS["block_d256_s288"])
+    fake = 1 << 20
+    arr = (h3b.BlockWeights * 4)(*[_weights(fake) for _ in range(4)])
+    dn, sf = h3b.lib.h3b_denoise_ex, h3b.lib.h3b_stack_forward_ex
+    wsx = h3b.lib.h3b_workspace_bytes_ex
+
+    def opts(**kw):
+        o = h3b.StackOpts(-1, -1, 0, -1, -1, 0, 0, None, None)
+        for k, v in kw.items():
+            setattr(o, k, v)
+        return ctypes.byref(o)
+
+    D = ctypes.byref(dm)
+    need = wsx(D, 0, opts(n_cond=8))
+    assert need > h3b.workspace_bytes(dm)                            # room for the condition rows
+    assert wsx(D, 0, opts(n_cond=-1)) == 0
+    assert sf(D, arr, 4, opts(n_cond=-1), fake, fake, need, None) == -3
+    assert sf(D, arr, 4, opts(modulation=fake + 4, mod_steps=1), fake, fake, need, None) == -2
+    assert sf(D, arr, 4, opts(modulation=fake, mod_steps=0), fake, fake, need, None) == -3
+    # per-step slices must number 1 or n_steps
+    assert dn(D, arr, 4, opts(modulation=fake, mod_steps=3), 20, 1, 1, fake, fake, fake, need, None, None,
+              None) == -3
+    # condition rows without their values, or misaligned
+    assert dn(D, arr, 4, opts(n_cond=8), 20, 1, 1, fake, fake, fake, need, None, None, None) == -1
+    assert dn(D, arr, 4, opts(n_cond=8, cond_rows=fake + 8), 20, 1, 1, fake, fake, fake, need, None, None,
+              None) == -2
+    # workspace sized without the condition rows
+    assert sf(D, arr, 4, opts(n_cond=8), fake, fake, h3b.workspace_bytes(dm), None) == -5

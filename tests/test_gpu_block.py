@@ -341,3 +341,89 @@ def test_denoise_core_counts(cuda_dev):
     got = [h3b.denoise_ex(dm, blocks, x, v, ws, 20, o, core_reuse=r) for r in (1, 4, 6)]
     assert got == [(20, 20), (20, 6), (20, 5)]
     assert [len(oracle.fresh_steps(20, r)) for r in (1, 4, 6)] == [20, 6, 5]
+
+
+# ----------------------------------------------------------------------------- modulation and condition rows
+def rand_mod(shape, seed, dev):
+    """Modulation vectors [..., 2, 6, d]: shifts and scales ~ N(0, 0.1), gates ~ 1 + N(0, 0.1)."""
+    m = wlmod.normal_tensor(shape, seed, dev, std=0.1)
+    m[..., 2, :] += 1.0
+    m[..., 5, :] += 1.0
+    return m.contiguous()
+
+
+@pytest.mark.parametrize("int8", [False, True])
+def test_modulated_block_with_condition_rows_vs_oracle(cuda_dev, int8):
+    wl = TINY
+    C = 16
+    w, blk = make_block(wl, 0, cuda_dev, int8)
+    dm = h3b.dims_of(wl)
+    mod = rand_mod((1, 2, 6, wl.d), 40, cuda_dev)
+    x0 = wlmod.initial_tokens(wl, cuda_dev, seq=wl.seq + C)
+    x = x0.clone()
+    o = h3b.stack_opts(n_cond=C, modulation=mod)
+    h3b.stack_forward_ex(dm, [blk], x, h3b.workspace_ex(dm, o, h3b.INT8 if int8 else h3b.BF16), o)
+    torch.cuda.synchronize()
+    hw = host_weights(w)
+    ref = oracle.block_forward_cond(np64(x0), oracle.dequant_weights(hw) if int8 else hw, wl, np64(mod[0]), C)
+    (check_int8 if int8 else check_bf16)(np64(x0), np64(x), ref)
+
+
+def test_identity_modulation_is_bitexact(cuda_dev):
+    wl = TINY.with_(n_blocks=3, depth_scaled_init=True, seed=12)
+    blocks = [h3b.Block.from_dict(wlmod.block_weights(wl, l, cuda_dev)) for l in range(3)]
+    dm = h3b.dims_of(wl)
+    ident = torch.zeros((3, 2, 6, wl.d), device=cuda_dev)
+    ident[..., 2, :] = 1.0
+    ident[..., 5, :] = 1.0
+    x = wlmod.initial_tokens(wl, cuda_dev)
+    y = x.clone()
+    o = h3b.stack_opts(0, 1, modulation=ident)
+    h3b.stack_forward_ex(dm, blocks, x, h3b.workspace_ex(dm, o), o)
+    h3b.stack_forward(dm, blocks, y, h3b.workspace(dm, h3b.BF16, True), 0, 1)
+    torch.cuda.synchronize()
+    assert torch.equal(x, y)
+
+
+@pytest.mark.parametrize("delta", [False, True])
+def test_condition_stack_with_reduction_vs_oracle(cuda_dev, delta):
+    wl = TINY.with_(n_blocks=5, depth_scaled_init=True, seed=13)
+    C = 24
+    ws_ = [wlmod.block_weights(wl, l, cuda_dev) for l in range(5)]
+    blocks = [h3b.Block.from_dict(w) for w in ws_]
+    dm = h3b.dims_of(wl)
+    mod = rand_mod((5, 2, 6, wl.d), 41, cuda_dev)
+    x0 = wlmod.initial_tokens(wl, cuda_dev, seq=wl.seq + C)
+    x = x0.clone()
+    o = h3b.stack_opts(1, 3, unmerge_delta=delta, n_cond=C, modulation=mod)
+    h3b.stack_forward_ex(dm, blocks, x, h3b.workspace_ex(dm, o), o)
+    torch.cuda.synchronize()
+    assert h3b.device_error() == 0
+    ref = oracle.stack_forward_cond(np64(x0), [host_weights(w) for w in ws_], wl, np64(mod), C, 1, 3,
+                                    unmerge_delta=delta)
+    check_bf16(np64(x0), np64(x), ref)
+
+
+@pytest.mark.parametrize("reuse,core_reuse,per_step", [(2, 1, True), (1, 3, True), (3, 1, False)])
+def test_denoise_with_condition_rows_and_modulation_vs_oracle(cuda_dev, reuse, core_reuse, per_step):
+    wl = TINY.with_(n_blocks=4, depth_scaled_init=True, seed=14)
+    C, steps = 12, 5
+    ws_ = [wlmod.block_weights(wl, l, cuda_dev) for l in range(4)]
+    blocks = [h3b.Block.from_dict(w) for w in ws_]
+    dm = h3b.dims_of(wl)
+    mod = rand_mod(((steps,) if per_step else ()) + (4, 2, 6, wl.d), 42, cuda_dev)
+    cond = wlmod.normal_tensor((C, wl.d), 43, cuda_dev)
+    core = core_reuse > 1
+    o = h3b.stack_opts(1, 2, core_first=1 if core else -1, core_last=2 if core else -1, cond_rows=cond,
+                       modulation=mod)
+    x0 = wlmod.initial_tokens(wl, cuda_dev)
+    x = x0.clone()
+    v = torch.empty((wl.seq + C, wl.d), device=cuda_dev)
+    nf, nc = h3b.denoise_ex(dm, blocks, x, v, h3b.workspace_ex(dm, o), steps, o, reuse=reuse, core_reuse=core_reuse)
+    torch.cuda.synchronize()
+    assert h3b.device_error() == 0
+    ref, nf_ref, nc_ref = oracle.denoise_cond(np64(x0), [host_weights(w) for w in ws_], wl, steps, np64(cond),
+                                              np64(mod), reuse, 1, 2, core_reuse=core_reuse,
+                                              core_first=1 if core else -1, core_last=2 if core else -1)
+    assert nf == nf_ref and (not core or nc == nc_ref)
+    assert rel_l2(x, ref) <= 1e-2 and max_abs(x, ref) <= 5e-2
