@@ -220,9 +220,18 @@ def run_ours(args, wl):
     core = loop and args.core_reuse > 0
     n_core = 0
 
-    if loop and (core or args.unmerge_delta):
+    if loop and (core or args.unmerge_delta or args.cond_rows or args.modulation):
+        cond = mod = None
+        if args.cond_rows:
+            cond = W.normal_tensor((args.cond_rows, wl.d), wl.seed * 7 + 1, dev)
+            v = torch.empty((wl.seq + args.cond_rows, wl.d), dtype=torch.float32, device=dev)
+        if args.modulation:
+            mod = W.normal_tensor((wl.steps, len(blocks), 2, 6, wl.d), wl.seed * 7 + 2, dev, std=0.1)
+            mod[..., 2, :] += 1.0
+            mod[..., 5, :] += 1.0
         opts = h3b.stack_opts(wl.merge_first, wl.merge_last, args.unmerge_delta,
-                              wl.merge_first if core else -1, wl.merge_last if core else -1)
+                              wl.merge_first if core else -1, wl.merge_last if core else -1,
+                              cond_rows=cond, modulation=mod)
         ws = h3b.workspace_ex(dm, opts, wl.dtype)
         reuse = 1 if core else wl.reuse
 
@@ -311,12 +320,13 @@ def run_ours(args, wl):
     flops_step = wl.block_flops() * (len(blocks) if not loop else 0)
     if loop:
         fm, fr = wl.merge_first, wl.merge_last
+        fl = wl.with_(n_audio=wl.n_audio + args.cond_rows)  # condition rows add to every block's sequence
         if core:
-            outer = sum(wl.block_flops() for l in range(len(blocks)) if not fm <= l <= fr)
-            inner = sum(wl.block_flops(merged=True) for l in range(fm, fr + 1))
+            outer = sum(fl.block_flops() for l in range(len(blocks)) if not fm <= l <= fr)
+            inner = sum(fl.block_flops(merged=True) for l in range(fm, fr + 1))
             flops_step = outer * n_fresh + inner * n_core
         else:
-            per_eval = sum(wl.block_flops(merged=(fm >= 0 and fm <= l <= fr)) for l in range(len(blocks)))
+            per_eval = sum(fl.block_flops(merged=(fm >= 0 and fm <= l <= fr)) for l in range(len(blocks)))
             flops_step = per_eval * n_fresh
 
     # end-to-end through the public API with the tokens in pinned host memory:
@@ -370,6 +380,8 @@ def run_ours(args, wl):
         if core:
             line["config"].update({"core_reuse": args.core_reuse, "core_blocks": [wl.merge_first, wl.merge_last],
                                    "core_evals": n_core})
+        if args.cond_rows or args.modulation:
+            line["config"].update({"cond_rows": args.cond_rows, "modulation": "per step" if args.modulation else None})
         line["ms_per_loop"] = round(ms / args.steps, 3)
     if e2e:
         line["e2e"] = e2e
@@ -495,13 +507,19 @@ def main():
                     help="loop workload: run only the first L blocks (the pages' --layers 40/45/50)")
     ap.add_argument("--denoise-steps", type=int, default=0,
                     help="loop workload: denoising steps (the pages' 4..7-step presets; default: the workload's)")
+    ap.add_argument("--cond-rows", type=int, default=0,
+                    help="loop workload: fixed condition rows appended after the audio tokens")
+    ap.add_argument("--modulation", action="store_true",
+                    help="loop workload: per-step, per-block timestep modulation (shift/scale/gate)")
     ap.add_argument("--cpu-budget", type=float, default=30.0)
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # never fewer than 3 warm-up steps
     wl = W.WORKLOADS[args.workload]
+    if (args.layers or args.denoise_steps or args.cond_rows or args.modulation or args.core_reuse
+            or args.unmerge_delta) and wl.steps == 0:
+        ap.error("--layers, --denoise-steps, --cond-rows, --modulation, --core-reuse and --unmerge-delta apply to "
+                 "the denoising-loop workloads")
     if args.layers or args.denoise_steps:
-        if wl.steps == 0:
-            ap.error("--layers / --denoise-steps apply to the denoising-loop workloads")
         if args.layers and not (0 < args.layers and (wl.merge_last < args.layers)):
             ap.error("--layers must keep the token-reduction window inside the active blocks")
         wl = wl.with_(n_blocks=args.layers or wl.n_blocks, steps=args.denoise_steps or wl.steps)
