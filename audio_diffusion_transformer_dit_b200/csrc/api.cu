@@ -68,7 +68,7 @@ struct Trace {
 const char* kKernelNames[KID_COUNT] = {"flow_step", "token_merge", "token_unmerge", "rope_table", "rmsnorm",
                                        "quant_rows", "quant_absmax", "gemm_qkv_rope", "gemm_o_resid",
                                        "gemm_fc1_gelu", "gemm_fc2_resid", "gemm", "attention", "memset",
-                                       "token_unmerge_delta", "copy"};
+                                       "token_unmerge_delta", "copy", "gelu"};
 
 struct TraceScope {
   TraceRec* rec = nullptr;
@@ -722,6 +722,15 @@ int h3b_exp2_poly(const float* x, float* y, int n, void* stream) {
   Ctx c;
   H3B_TRY(device_ctx(static_cast<cudaStream_t>(stream), &c));
   H3B_CU(KID_ATTN, launch_exp2_poly(c, x, y, n));
+  return H3B_OK;
+}
+
+int h3b_gelu(const float* x, float* y, size_t n, void* stream) {
+  if (n == 0) return H3B_OK;
+  if (!x || !y) return H3B_ERR_NULL;
+  Ctx c;
+  H3B_TRY(device_ctx(static_cast<cudaStream_t>(stream), &c));
+  H3B_CU(KID_GELU, launch_gelu(c, x, y, n));
   return H3B_OK;
 }
 

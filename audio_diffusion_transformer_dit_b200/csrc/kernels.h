@@ -28,6 +28,7 @@ enum KernelId {
   KID_MEMSET,
   KID_UNMERGE_DELTA,
   KID_COPY,
+  KID_GELU,
   KID_COUNT
 };
 
@@ -53,6 +54,7 @@ struct Mod {
   const float* scale = nullptr;
   int split = 0, stride = 0;
 };
+cudaError_t launch_gelu(const Ctx& c, const float* x, float* y, size_t n);
 cudaError_t launch_rmsnorm(const Ctx& c, const float* x, const float* g, int rows, int d, float eps, void* out,
                            float* out_scale, int out_int8, const Mod& mod = Mod{});
 cudaError_t launch_quant_rows(const Ctx& c, const void* a, int rows, int k, int8_t* q, float* s);

@@ -185,6 +185,13 @@ __global__ void k_rope_table(float2* __restrict__ table, int F, int H, int Wc, i
   }
 }
 
+// ------------------------------------------------------------------ GELU (the FC1 epilogue's function)
+__global__ void k_gelu(const float* __restrict__ x, float* __restrict__ y, size_t n) {
+  for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x)
+    y[i] = gelu_erf(x[i]);
+}
+
 // ------------------------------------------------------------------ RMSNorm (+ quant)
 // One CTA per token row; the row stays in registers between the statistics and
 // the output pass (x is read from HBM exactly once).
@@ -411,6 +418,12 @@ cudaError_t launch_rope_table(const Ctx& c, const h3b_dims& dm, int merged, floa
   if (total == 0) return cudaSuccess;
   k_rope_table<<<grid_for(total, c.num_sms, 8), kThreads, 0, c.stream>>>(
       reinterpret_cast<float2*>(table), dm.frames, dm.rows, wc, dm.n_audio, dm.head_dim, dm.rope_theta, merged);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gelu(const Ctx& c, const float* x, float* y, size_t n) {
+  if (n == 0) return cudaSuccess;
+  k_gelu<<<grid_for(n, c.num_sms), kThreads, 0, c.stream>>>(x, y, n);
   return cudaGetLastError();
 }
 

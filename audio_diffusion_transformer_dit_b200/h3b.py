@@ -68,6 +68,7 @@ _SIGS = {
     "h3b_quantize_rows_absmax": (_i, [_p, _p, _i, _i, _p, _p, _p]),
     "h3b_attention": (_i, [_p, _i, _i, _i, _p, _p, _sz, _p]),
     "h3b_exp2_poly": (_i, [_p, _p, _i, _p]),
+    "h3b_gelu": (_i, [_p, _p, _sz, _p]),
     "h3b_device_error": (_i, [_p]),
     "h3b_selftest_wait_timeout": (_i, [_i, _p]),
     "h3b_trace_start": (_i, [_i]),
@@ -205,9 +206,13 @@ class HostPipeline:
     ``submit(x_in, x_out)`` enqueues one step: x_in (pinned host, [S, d] fp32)
     is copied in, processed, and the result copied to x_out (pinned host).
     The call returns at once; x_in must stay untouched and x_out is valid only
-    after ``synchronize()`` (or once a later submit has reused its buffer)."""
+    after ``synchronize()`` (or once a later submit has reused its buffer).
 
-    def __init__(self, dims: Dims, blocks, ws: torch.Tensor, shape, depth: int = 2, merge_first: int = -1,
+    Three buffers (the default) let step i+1's copy-in start while step i-1's
+    copy-out is still running; with two, that copy-in waits for it and the
+    loop runs at compute + copy-out + copy-in per two steps."""
+
+    def __init__(self, dims: Dims, blocks, ws: torch.Tensor, shape, depth: int = 3, merge_first: int = -1,
                  merge_last: int = -1):
         self.dims, self.ws = dims, ws
         self.blocks = list(blocks) if isinstance(blocks, (list, tuple)) else [blocks]
@@ -396,6 +401,12 @@ def attention(qkv: torch.Tensor, n_heads: int, head_dim: int, o: Optional[torch.
 def exp2_poly(x: torch.Tensor) -> torch.Tensor:
     y = torch.empty_like(x)
     _check(lib.h3b_exp2_poly(_ptr(x, torch.float32, "x"), y.data_ptr(), x.numel(), _stream()), "h3b_exp2_poly")
+    return y
+
+
+def gelu(x: torch.Tensor) -> torch.Tensor:
+    y = torch.empty_like(x)
+    _check(lib.h3b_gelu(_ptr(x, torch.float32, "x"), y.data_ptr(), x.numel(), _stream()), "h3b_gelu")
     return y
 
 

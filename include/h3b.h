@@ -322,6 +322,13 @@ int h3b_attention(const void* qkv, int S, int n_heads, int head_dim, void* o, vo
  * x, y: fp32 [n] device buffers.  For accuracy tests of that approximation. */
 int h3b_exp2_poly(const float* x, float* y, int n, void* stream);
 
+/* The FC1 epilogue's GELU, y[i] = x[i] * Phi(x[i]) in fp32 for i < n, for
+ * accuracy tests: Phi from the complementary error function of Abramowitz &
+ * Stegun formula 7.1.26 (absolute error <= 1.5e-7), never forming 1 + erf on
+ * the negative side.  x, y: fp32 device buffers (any alignment); n == 0 is a
+ * no-op. */
+int h3b_gelu(const float* x, float* y, size_t n, void* stream);
+
 /* ---------------------------------------------------------------------------
  * Device error word and tracing
  * ------------------------------------------------------------------------- */

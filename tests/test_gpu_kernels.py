@@ -284,6 +284,22 @@ def test_attention_large_scores(cuda_dev):
     assert rel_l2(o, ref) < 1e-2
 
 
+def test_gelu_accuracy(cuda_dev):
+    """The GEMM epilogue's GELU against the exact-erf form in fp64.  Budget:
+    Abramowitz & Stegun 7.1.26 is within 1.5e-7 of erfc, i.e. 0.75e-7 * |x| in
+    GELU; the fp32 evaluation adds a few ulp of erfc/2 (< 0.5) and of the
+    result -- together below 2e-7 * |x| + 1e-6 * |GELU(x)|."""
+    x = torch.cat([torch.linspace(-12.0, 12.0, 200001), wlmod.normal_tensor((100000,), 50, "cpu") * 4.0,
+                   torch.tensor([0.0, -0.0, 1e-30, -1e-30, 30.0, -30.0, 3e4, -3e4])]).float().to(cuda_dev)
+    y = h3b.gelu(x)
+    torch.cuda.synchronize()
+    xr = np64(x)
+    ref = oracle.gelu(xr)
+    err = np.abs(np64(y) - ref)
+    assert np.all(err <= 2e-7 * np.abs(xr) + 1e-6 * np.abs(ref))
+    assert np.all(np64(y)[xr >= 0] >= 0) and np.all(np64(y)[xr < 0] <= 0)
+
+
 def test_exp2_poly_error_bound(cuda_dev):
     """The FMA-pipe exp2 of the attention kernel against 2^x in fp64."""
     x = torch.cat([torch.linspace(-125.0, 8.0, 1_000_001), torch.tensor([0.0, -0.5, 0.5, 1.0, -1.0, 7.5])])
