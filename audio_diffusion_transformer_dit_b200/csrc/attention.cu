@@ -153,6 +153,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   constexpr int KB = D / 64;         // 128-byte column blocks per head row
   constexpr int TILE = 128 * D * 2;  // bytes of a 128-row Q/K/V tile
   constexpr int BLK = 128 * 128;     // bytes of one 128-row x 128-byte block
+  pdl_trigger();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;               // tiles A, B
@@ -211,6 +212,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  pdl_wait();
   const uint32_t tmem = *tmem_slot;
   if (warp >= 8) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REG_CONTROL));
@@ -453,6 +455,8 @@ __global__ void __launch_bounds__(THREADS, 1)
 // o = sum_c O_c 2^(m_c - M) / sum_c l_c 2^(m_c - M), parts in fixed order.
 template <int D>
 __global__ void __launch_bounds__(D) k_attn_combine(const AttnArgs a) {
+  pdl_trigger();
+  pdl_wait();
   const int ti = blockIdx.x / 256, r = blockIdx.x % 256, col = threadIdx.x;
   const int item = a.n_full + ti;
   const int grow = (item % a.pairs) * 2 * BQ + r, h = item / a.pairs;
@@ -471,6 +475,8 @@ __global__ void __launch_bounds__(D) k_attn_combine(const AttnArgs a) {
 }
 
 __global__ void k_exp2_poly(const float* __restrict__ x, float* __restrict__ y, int n) {
+  pdl_trigger();
+  pdl_wait();
   const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
   if (i + 1 < n) {
     const uint64_t r = ex2_poly2(f2_pack(x[i], x[i + 1]));
@@ -486,7 +492,8 @@ __global__ void k_exp2_poly(const float* __restrict__ x, float* __restrict__ y, 
 cudaError_t launch_exp2_poly(const Ctx& c, const float* x, float* y, int n) {
   if (n <= 0) return cudaSuccess;
   const int threads = 256, blocks = (n / 2 + threads) / threads;
-  k_exp2_poly<<<blocks, threads, 0, c.stream>>>(x, y, n);
+  const cudaError_t e = launch_pdl(c.stream, k_exp2_poly, dim3(blocks), dim3(threads), 0, 1u, x, y, n);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
@@ -529,13 +536,14 @@ cudaError_t launch_attention(const Ctx& c, const void* qkv, int S, int n_heads, 
     }
   }
   const int grid = a.n_full + (items - a.n_full) * a.ks;
-  kern<<<grid, THREADS, smem, c.stream>>>(tm, a);
+  e = launch_pdl(c.stream, kern, dim3(grid), dim3(THREADS), smem, 1u, tm, a);
+  if (e != cudaSuccess) return e;
   e = cudaGetLastError();
   if (e != cudaSuccess || a.ks == 1) return e;
   if (d128)
-    k_attn_combine<128><<<(items - a.n_full) * 256, 128, 0, c.stream>>>(a);
+    e = launch_pdl(c.stream, k_attn_combine<128>, dim3((items - a.n_full) * 256), dim3(128), 0, 1u, a);
   else
-    k_attn_combine<64><<<(items - a.n_full) * 256, 64, 0, c.stream>>>(a);
+    e = launch_pdl(c.stream, k_attn_combine<64>, dim3((items - a.n_full) * 256), dim3(64), 0, 1u, a);
   return cudaGetLastError();
 }
 

@@ -39,6 +39,19 @@ __device__ __forceinline__ uint64_t global_ns() {
   return t;
 }
 
+// ------------------------------------------------------------------ dependent launch
+// Every kernel is launched with programmatic stream serialization: it may be
+// scheduled while its predecessor in the stream is still running.  Each
+// kernel lets its own successor be scheduled at once (pdl_trigger; a
+// successor is only scheduled after every CTA of this grid has started, so a
+// waiting successor never holds resources this grid still needs) and calls
+// pdl_wait -- which returns once every prerequisite grid has completed and its
+// memory is visible -- before its first access to global memory a predecessor
+// may read or write.  Work before the wait is confined to shared memory,
+// TMEM, barriers and kernel parameters.
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ------------------------------------------------------------------ mbarrier
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");

@@ -170,6 +170,7 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& p, int m, int n, 
 template <bool INT8, int EPI>
 __global__ void __launch_bounds__(THREADS, 1)
     k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const GemmArgs p) {
+  pdl_trigger();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
@@ -206,6 +207,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  pdl_wait();
   const uint32_t tmem_base = *tmem_slot;
 
   const int num_m = (p.M + BM - 1) / BM, num_n = (p.N + BN - 1) / BN, num_tiles = num_m * num_n;
@@ -352,6 +354,8 @@ template <int TM>
 __global__ void __launch_bounds__(BN) k_splitk_add(float* __restrict__ C, const float* __restrict__ partial, int M,
                                                    int N, int full_tiles, int split, int num_m, int num_n,
                                                    const float* __restrict__ gate, int gate_split, int gate_stride) {
+  pdl_trigger();
+  pdl_wait();
   const int i = blockIdx.x / TM, r = blockIdx.x % TM, col = threadIdx.x;
   int mb, nb;
   tile_coords(full_tiles + i, num_m, num_n, mb, nb);
@@ -436,6 +440,7 @@ __device__ __forceinline__ void commit2_local(uint32_t bar) {
 template <bool INT8, int EPI>
 __global__ void __launch_bounds__(THREADS, 1)
     k_gemm2(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const GemmArgs p) {
+  pdl_trigger();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
@@ -478,6 +483,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncthreads();
   cluster_sync();  // both ranks' barriers exist before any cross-rank arrival
   tc_fence_after();
+  pdl_wait();
   const uint32_t tmem_base = *tmem_slot;
 
   const int num_m = (p.M + BM2 - 1) / BM2, num_n = (p.N + BN - 1) / BN, num_tiles = num_m * num_n;
@@ -720,23 +726,19 @@ cudaError_t launch_gemm(const Ctx& c, const void* A, const void* B, int ab_int8,
       args.partial = scratch;
     }
   }
-  if (pair) {
-    cfg.gridDim = dim3(2 * grid);
-    e = cudaLaunchKernelEx(&cfg, kern, ta, tb, args);
-    if (e != cudaSuccess) return e;
-  } else {
-    kern<<<grid, THREADS, smem, c.stream>>>(ta, tb, args);
-  }
+  e = launch_pdl(c.stream, kern, dim3(pair ? 2 * grid : grid), dim3(THREADS), smem, pair ? 2u : 1u, ta, tb, args);
+  if (e != cudaSuccess) return e;
   e = cudaGetLastError();
   if (e != cudaSuccess || args.split <= 1) return e;
   if (pair)
-    k_splitk_add<BM2><<<rem * BM2, BN, 0, c.stream>>>(static_cast<float*>(args.C), args.partial, args.M, args.N,
-                                                      args.full_tiles, args.split, num_m, num_n, args.gate,
-                                                      args.gate_split, args.gate_stride);
+    e = launch_pdl(c.stream, k_splitk_add<BM2>, dim3(rem * BM2), dim3(BN), 0, 1u, static_cast<float*>(args.C),
+                   static_cast<const float*>(args.partial), args.M, args.N, args.full_tiles, args.split, num_m, num_n,
+                   args.gate, args.gate_split, args.gate_stride);
   else
-    k_splitk_add<BM><<<rem * BM, BN, 0, c.stream>>>(static_cast<float*>(args.C), args.partial, args.M, args.N,
-                                                    args.full_tiles, args.split, num_m, num_n, args.gate,
-                                                    args.gate_split, args.gate_stride);
+    e = launch_pdl(c.stream, k_splitk_add<BM>, dim3(rem * BM), dim3(BN), 0, 1u, static_cast<float*>(args.C),
+                   static_cast<const float*>(args.partial), args.M, args.N, args.full_tiles, args.split, num_m, num_n,
+                   args.gate, args.gate_split, args.gate_stride);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -10,6 +10,33 @@
 
 namespace h3b {
 
+// Launch with programmatic stream serialization (the kernel overlaps its
+// prologue with its predecessor's tail; see pdl_wait in common.cuh).
+// cluster_x > 1 adds a thread-block-cluster dimension.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(cudaStream_t stream, void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       unsigned cluster_x, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute at[2];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  unsigned n = 1;
+  if (cluster_x > 1) {
+    at[1].id = cudaLaunchAttributeClusterDimension;
+    at[1].val.clusterDim.x = cluster_x;
+    at[1].val.clusterDim.y = 1;
+    at[1].val.clusterDim.z = 1;
+    n = 2;
+  }
+  cfg.attrs = at;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 // kernel ids for tracing (names in h3b_kernel_name)
 enum KernelId {
   KID_FLOW = 0,

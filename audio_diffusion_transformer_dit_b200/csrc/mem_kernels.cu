@@ -55,6 +55,8 @@ __device__ __forceinline__ int8_t quant1(float v, float s, float rs) {
 // ------------------------------------------------------------------ Euler step
 __global__ void k_flow(float* __restrict__ x, const float* __restrict__ v, float dt, size_t n,
                        float* __restrict__ xc) {
+  pdl_trigger();
+  pdl_wait();
   const size_t n4 = n >> 2;
   const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
   float4* x4 = reinterpret_cast<float4*>(x);
@@ -82,6 +84,8 @@ __global__ void k_flow(float* __restrict__ x, const float* __restrict__ v, float
 // sequence, so merged row i averages full rows 2i and 2i+1; audio rows follow.
 __global__ void k_merge(const float4* __restrict__ x, float4* __restrict__ xm, float4* __restrict__ xm_copy,
                         int half_video, int n_audio, int d4) {
+  pdl_trigger();
+  pdl_wait();
   const size_t total = static_cast<size_t>(half_video + n_audio) * d4;
   const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
   for (size_t e = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < total; e += stride) {
@@ -103,6 +107,8 @@ __global__ void k_merge(const float4* __restrict__ x, float4* __restrict__ xm, f
 }
 
 __global__ void k_unmerge(const float4* __restrict__ xm, float4* __restrict__ x, int n_video, int n_audio, int d4) {
+  pdl_trigger();
+  pdl_wait();
   const size_t total = static_cast<size_t>(n_video + n_audio) * d4;
   const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
   const int half = n_video / 2;
@@ -117,6 +123,8 @@ __global__ void k_unmerge(const float4* __restrict__ xm, float4* __restrict__ x,
 // merged blocks' update); audio rows take ym.
 __global__ void k_unmerge_delta(float4* __restrict__ x, const float4* __restrict__ ym,
                                 const float4* __restrict__ xm0, int n_video, int n_audio, int d4) {
+  pdl_trigger();
+  pdl_wait();
   const size_t total = static_cast<size_t>(n_video + n_audio) * d4;
   const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
   const int half = n_video / 2;
@@ -146,6 +154,7 @@ __global__ void k_unmerge_delta(float4* __restrict__ x, const float4* __restrict
 constexpr int kMaxHalfHead = 64;  // head_dim <= 128
 __global__ void k_rope_table(float2* __restrict__ table, int F, int H, int Wc, int A, int D, float theta,
                              int merged) {
+  pdl_trigger();
   __shared__ double f_video[kMaxHalfHead], f_audio[kMaxHalfHead];
   const int half = D / 2;
   const int nf = D / 4, nr = 3 * D / 8, nc = D - nf - nr;
@@ -163,6 +172,7 @@ __global__ void k_rope_table(float2* __restrict__ table, int F, int H, int Wc, i
     f_audio[j] = exp2(-2.0 * j / D * l2t);
   }
   __syncthreads();
+  pdl_wait();  // the table may still be read by the previous block's QKV GEMM
   const int n_video = F * H * Wc;
   const size_t total = static_cast<size_t>(n_video + A) * half;
   for (size_t e = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < total;
@@ -187,6 +197,8 @@ __global__ void k_rope_table(float2* __restrict__ table, int F, int H, int Wc, i
 
 // ------------------------------------------------------------------ GELU (the FC1 epilogue's function)
 __global__ void k_gelu(const float* __restrict__ x, float* __restrict__ y, size_t n) {
+  pdl_trigger();
+  pdl_wait();
   for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
        i += static_cast<size_t>(gridDim.x) * blockDim.x)
     y[i] = gelu_erf(x[i]);
@@ -199,6 +211,8 @@ template <int VPT, bool INT8>
 __global__ void __launch_bounds__(kThreads) k_rmsnorm(const float* __restrict__ x, const float* __restrict__ g, int d,
                                                       float eps, void* __restrict__ out, float* __restrict__ out_scale,
                                                       const Mod mod) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ float red[32];
   const int row = blockIdx.x, d4 = d >> 2;
   const float4* xr = reinterpret_cast<const float4*>(x + static_cast<size_t>(row) * d);
@@ -289,6 +303,8 @@ __device__ __forceinline__ uint2 quant8(const float (&f)[8], float s, float rs) 
 template <int VPT>
 __global__ void __launch_bounds__(kThreads) k_quant_rows(const uint4* __restrict__ a, int k8, int8_t* __restrict__ q,
                                                          float* __restrict__ scale) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ float red[32];
   const int row = blockIdx.x;
   const uint4* ar = a + static_cast<size_t>(row) * k8;
@@ -322,6 +338,8 @@ __global__ void __launch_bounds__(kThreads) k_quant_rows(const uint4* __restrict
 // turns 16 bf16 (two 16-byte loads) into 16 codes (one 16-byte store).
 __global__ void k_quant_absmax(const uint4* __restrict__ a, const float* __restrict__ absmax, int k16,
                                int8_t* __restrict__ q, float* __restrict__ scale) {
+  pdl_trigger();
+  pdl_wait();
   const int row = blockIdx.y;
   const float s = absmax[row] / 127.0f, rs = 1.0f / s;
   const uint4* ar = a + static_cast<size_t>(row) * k16 * 2;
@@ -339,6 +357,8 @@ __global__ void k_quant_absmax(const uint4* __restrict__ a, const float* __restr
 // Same with 8 elements per thread (k a multiple of 8 but not of 16).
 __global__ void k_quant_absmax8(const uint4* __restrict__ a, const float* __restrict__ absmax, int k8,
                                 int8_t* __restrict__ q, float* __restrict__ scale) {
+  pdl_trigger();
+  pdl_wait();
   const int row = blockIdx.y;
   const float s = absmax[row] / 127.0f, rs = 1.0f / s;
   const uint4* ar = a + static_cast<size_t>(row) * k8;
@@ -355,6 +375,8 @@ __global__ void k_quant_absmax8(const uint4* __restrict__ a, const float* __rest
 // with a short limit; the bounded wait must give up, record its code in the
 // device error word and let the kernel exit normally.
 __global__ void k_selftest_wait(int* err, unsigned long long timeout_ns) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ uint64_t bar;
   __shared__ int abort_flag;
   if (threadIdx.x == 0) {
@@ -377,18 +399,17 @@ int grid_for(size_t work_items, int num_sms, int per_sm = 8) {
 
 cudaError_t launch_flow_step(const Ctx& c, float* x, const float* v, float dt, size_t n, float* x_copy) {
   if (n == 0) return cudaSuccess;
-  k_flow<<<grid_for((n + 3) / 4, c.num_sms), kThreads, 0, c.stream>>>(x, v, dt, n, x_copy);
-  return cudaGetLastError();
+  return launch_pdl(c.stream, k_flow, dim3(grid_for((n + 3) / 4, c.num_sms)), dim3(kThreads), 0, 1u, x, v, dt, n,
+                    x_copy);
 }
 
 cudaError_t launch_merge(const Ctx& c, const float* x, float* xm, int n_video, int n_audio, int d, float* xm_copy) {
   const int d4 = d / 4;
   const size_t total = static_cast<size_t>(n_video / 2 + n_audio) * d4;
   if (total == 0) return cudaSuccess;
-  k_merge<<<grid_for(total, c.num_sms), kThreads, 0, c.stream>>>(
-      reinterpret_cast<const float4*>(x), reinterpret_cast<float4*>(xm), reinterpret_cast<float4*>(xm_copy),
-      n_video / 2, n_audio, d4);
-  return cudaGetLastError();
+  return launch_pdl(c.stream, k_merge, dim3(grid_for(total, c.num_sms)), dim3(kThreads), 0, 1u,
+                    reinterpret_cast<const float4*>(x), reinterpret_cast<float4*>(xm),
+                    reinterpret_cast<float4*>(xm_copy), n_video / 2, n_audio, d4);
 }
 
 cudaError_t launch_unmerge_delta(const Ctx& c, float* x, const float* ym, const float* xm0, int n_video, int n_audio,
@@ -396,35 +417,31 @@ cudaError_t launch_unmerge_delta(const Ctx& c, float* x, const float* ym, const 
   const int d4 = d / 4;
   const size_t total = static_cast<size_t>(n_video + n_audio) * d4;
   if (total == 0) return cudaSuccess;
-  k_unmerge_delta<<<grid_for(total, c.num_sms), kThreads, 0, c.stream>>>(
-      reinterpret_cast<float4*>(x), reinterpret_cast<const float4*>(ym), reinterpret_cast<const float4*>(xm0),
-      n_video, n_audio, d4);
-  return cudaGetLastError();
+  return launch_pdl(c.stream, k_unmerge_delta, dim3(grid_for(total, c.num_sms)), dim3(kThreads), 0, 1u,
+                    reinterpret_cast<float4*>(x), reinterpret_cast<const float4*>(ym),
+                    reinterpret_cast<const float4*>(xm0), n_video, n_audio, d4);
 }
 
 cudaError_t launch_unmerge(const Ctx& c, const float* xm, float* x, int n_video, int n_audio, int d) {
   const int d4 = d / 4;
   const size_t total = static_cast<size_t>(n_video + n_audio) * d4;
   if (total == 0) return cudaSuccess;
-  k_unmerge<<<grid_for(total, c.num_sms), kThreads, 0, c.stream>>>(reinterpret_cast<const float4*>(xm),
-                                                                    reinterpret_cast<float4*>(x), n_video, n_audio,
-                                                                    d4);
-  return cudaGetLastError();
+  return launch_pdl(c.stream, k_unmerge, dim3(grid_for(total, c.num_sms)), dim3(kThreads), 0, 1u,
+                    reinterpret_cast<const float4*>(xm), reinterpret_cast<float4*>(x), n_video, n_audio, d4);
 }
 
 cudaError_t launch_rope_table(const Ctx& c, const h3b_dims& dm, int merged, float* table) {
   const int wc = merged ? dm.cols / 2 : dm.cols;
   const size_t total = static_cast<size_t>(dm.frames * dm.rows * wc + dm.n_audio) * (dm.head_dim / 2);
   if (total == 0) return cudaSuccess;
-  k_rope_table<<<grid_for(total, c.num_sms, 8), kThreads, 0, c.stream>>>(
-      reinterpret_cast<float2*>(table), dm.frames, dm.rows, wc, dm.n_audio, dm.head_dim, dm.rope_theta, merged);
-  return cudaGetLastError();
+  return launch_pdl(c.stream, k_rope_table, dim3(grid_for(total, c.num_sms, 8)), dim3(kThreads), 0, 1u,
+                    reinterpret_cast<float2*>(table), dm.frames, dm.rows, wc, dm.n_audio, dm.head_dim, dm.rope_theta,
+                    merged);
 }
 
 cudaError_t launch_gelu(const Ctx& c, const float* x, float* y, size_t n) {
   if (n == 0) return cudaSuccess;
-  k_gelu<<<grid_for(n, c.num_sms), kThreads, 0, c.stream>>>(x, y, n);
-  return cudaGetLastError();
+  return launch_pdl(c.stream, k_gelu, dim3(grid_for(n, c.num_sms)), dim3(kThreads), 0, 1u, x, y, n);
 }
 
 cudaError_t launch_rmsnorm(const Ctx& c, const float* x, const float* g, int rows, int d, float eps, void* out,
@@ -433,12 +450,13 @@ cudaError_t launch_rmsnorm(const Ctx& c, const float* x, const float* g, int row
   const int d4 = d / 4;
   int threads = d4 >= kThreads ? kThreads : ((d4 + 31) / 32) * 32;
   const int vpt = (d4 + threads - 1) / threads;
-#define H3B_NORM_CASE(V)                                                                                  \
-  case V:                                                                                                 \
-    if (out_int8)                                                                                         \
-      k_rmsnorm<V, true><<<rows, threads, 0, c.stream>>>(x, g, d, eps, out, out_scale, mod);              \
-    else                                                                                                  \
-      k_rmsnorm<V, false><<<rows, threads, 0, c.stream>>>(x, g, d, eps, out, out_scale, mod);             \
+  cudaError_t e;
+#define H3B_NORM_CASE(V)                                                                                       \
+  case V:                                                                                                      \
+    e = out_int8 ? launch_pdl(c.stream, k_rmsnorm<V, true>, dim3(rows), dim3(threads), 0, 1u, x, g, d, eps, out,  \
+                              out_scale, mod)                                                                  \
+                 : launch_pdl(c.stream, k_rmsnorm<V, false>, dim3(rows), dim3(threads), 0, 1u, x, g, d, eps, out, \
+                              out_scale, mod);                                                                 \
     break;
   switch (vpt) {
     H3B_NORM_CASE(1) H3B_NORM_CASE(2) H3B_NORM_CASE(3) H3B_NORM_CASE(4)
@@ -446,7 +464,7 @@ cudaError_t launch_rmsnorm(const Ctx& c, const float* x, const float* g, int row
     default: return cudaErrorInvalidValue;
   }
 #undef H3B_NORM_CASE
-  return cudaGetLastError();
+  return e;
 }
 
 cudaError_t launch_quant_rows(const Ctx& c, const void* a, int rows, int k, int8_t* q, float* s) {
@@ -455,8 +473,9 @@ cudaError_t launch_quant_rows(const Ctx& c, const void* a, int rows, int k, int8
   const int threads = k8 >= kThreads ? kThreads : ((k8 + 31) / 32) * 32;
   const int vpt = (k8 + threads - 1) / threads;
   const uint4* a4 = reinterpret_cast<const uint4*>(a);
+  cudaError_t e;
 #define H3B_Q_CASE(V) \
-  case V: k_quant_rows<V><<<rows, threads, 0, c.stream>>>(a4, k8, q, s); break;
+  case V: e = launch_pdl(c.stream, k_quant_rows<V>, dim3(rows), dim3(threads), 0, 1u, a4, k8, q, s); break;
   switch (vpt) {
     H3B_Q_CASE(1) H3B_Q_CASE(2) H3B_Q_CASE(3) H3B_Q_CASE(4) H3B_Q_CASE(5) H3B_Q_CASE(6)
     H3B_Q_CASE(7) H3B_Q_CASE(8) H3B_Q_CASE(9) H3B_Q_CASE(10) H3B_Q_CASE(11) H3B_Q_CASE(12)
@@ -464,7 +483,7 @@ cudaError_t launch_quant_rows(const Ctx& c, const void* a, int rows, int k, int8
     default: return cudaErrorInvalidValue;
   }
 #undef H3B_Q_CASE
-  return cudaGetLastError();
+  return e;
 }
 
 cudaError_t launch_quant_absmax(const Ctx& c, const void* a, const float* absmax, int rows, int k, int8_t* q,
@@ -477,17 +496,16 @@ cudaError_t launch_quant_absmax(const Ctx& c, const void* a, const float* absmax
     const int nr = rows - r0 < 65535 ? rows - r0 : 65535;
     const dim3 grid(bx, nr);
     const uint4* a4 = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(a) + static_cast<size_t>(r0) * k);
-    if (per_thread == 16)
-      k_quant_absmax<<<grid, kThreads, 0, c.stream>>>(a4, absmax + r0, chunks, q + static_cast<size_t>(r0) * k, s + r0);
-    else
-      k_quant_absmax8<<<grid, kThreads, 0, c.stream>>>(a4, absmax + r0, chunks, q + static_cast<size_t>(r0) * k, s + r0);
+    const cudaError_t e =
+        launch_pdl(c.stream, per_thread == 16 ? k_quant_absmax : k_quant_absmax8, grid, dim3(kThreads), 0, 1u, a4,
+                   absmax + r0, chunks, q + static_cast<size_t>(r0) * k, s + r0);
+    if (e != cudaSuccess) return e;
   }
   return cudaGetLastError();
 }
 
 cudaError_t launch_selftest_wait(const Ctx& c, unsigned long long timeout_ns) {
-  k_selftest_wait<<<1, 32, 0, c.stream>>>(c.err, timeout_ns);
-  return cudaGetLastError();
+  return launch_pdl(c.stream, k_selftest_wait, dim3(1), dim3(32), 0, 1u, c.err, timeout_ns);
 }
 
 }  // namespace h3b

@@ -48,6 +48,12 @@ def test_invalid_dims_rejected():
         dm = h3b.Dims(**{**base, **bad})
         assert h3b.lib.h3b_seq_len(ctypes.byref(dm), 0) == -1
         assert h3b.lib.h3b_workspace_bytes(ctypes.byref(dm), 0, 0) == 0
+    # the largest accepted sizes, and one past each
+    for ok, bad in ((dict(d=8192, n_heads=64), dict(d=8320, n_heads=65)),
+                    (dict(ffn=32768), dict(ffn=32896)),
+                    (dict(frames=1, rows=1, cols=1 << 24, n_audio=0), dict(frames=1, rows=1, cols=1 << 24, n_audio=1))):
+        assert h3b.lib.h3b_seq_len(ctypes.byref(h3b.Dims(**{**base, **ok})), 0) > 0
+        assert h3b.lib.h3b_seq_len(ctypes.byref(h3b.Dims(**{**base, **bad})), 0) == -1
     odd = h3b.Dims(**{**base, "cols": 3})
     assert h3b.lib.h3b_seq_len(ctypes.byref(odd), 1) == -1
     assert h3b.lib.h3b_workspace_bytes(ctypes.byref(odd), 0, 1) == 0

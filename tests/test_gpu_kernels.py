@@ -459,3 +459,51 @@ def test_quantize_ties_and_near_ties_bitexact(cuda_dev):
     assert np.array_equal(s.cpu().numpy(), sr) and np.array_equal(q.cpu().numpy(), qr)
     assert np.array_equal(s2.cpu().numpy(), sr) and np.array_equal(q2.cpu().numpy(), qr)
     assert set(np.abs(qr[0, 1:255]).tolist()) >= {0, 2, 126}  # half-even ties really occurred
+
+
+# ----------------------------------------------------------------------------- maximum sizes
+@pytest.mark.parametrize("M,N,K", [(130, 24576, 256), (130, 2048, 32768)])
+def test_gemm_int8_max_sizes_extremes_bitexact(cuda_dev, M, N, K):
+    """The largest operands the API accepts: N = 3 d at d = 8192 (QKV) and
+    K = f = 32768 (FC2).  Codes of +-127 drive every int32 accumulator to
+    +-127^2 K = 528,482,304 at K = 32768, still inside int32."""
+    A = torch.full((M, K), 127, dtype=torch.int8, device=cuda_dev)
+    A[1::2] = -127
+    B = wlmod.int8_tensor((N, K), 60, cuda_dev)
+    B[:64] = 127
+    C = torch.zeros((M, N), dtype=torch.int32, device=cuda_dev)
+    h3b.gemm(A, B, h3b.EPI_I32, C)
+    torch.cuda.synchronize()
+    ref = oracle.int8_matmul(A.cpu().numpy(), B.cpu().numpy())
+    assert np.abs(ref).max() == 127 * 127 * K
+    assert np.array_equal(C.cpu().numpy().astype(np.int64), ref)
+
+
+def test_gemm_bf16_residual_max_k(cuda_dev):
+    """FC2 at the largest MLP width (K = 32768) with the residual epilogue.
+    The bf16 products are exact; the fp32 accumulation error grows like
+    sqrt(K) (the K <= 3072 cases hold 1e-5, i.e. ~3.3e-5 at 32768), so the bar
+    is 1e-4.  A lost or doubled 64-wide K block would show as ~sqrt(64/K) =
+    4e-2; the int8 case at the same K is bit-exact."""
+    M, N, K = 257, 2048, 32768
+    A = wlmod.normal_tensor((M, K), 61, cuda_dev, dtype=torch.bfloat16)
+    B = wlmod.normal_tensor((N, K), 62, cuda_dev, 0.01, dtype=torch.bfloat16)
+    X0 = wlmod.normal_tensor((M, N), 63, cuda_dev)
+    X = X0.clone()
+    h3b.gemm(A, B, h3b.EPI_RESID, X)
+    torch.cuda.synchronize()
+    acc = oracle.linear(np64(A), np64(B))
+    assert rel_l2(np64(X) - np64(X0), acc) < 1e-4
+
+
+def test_attention_max_heads(cuda_dev):
+    """d = 8192: 64 heads of 128, over a ragged 300-token sequence."""
+    S, H, D = 300, 64, 128
+    qkv = wlmod.normal_tensor((S, 3 * H * D), 64, cuda_dev, 1.5, dtype=torch.bfloat16)
+    o = h3b.attention(qkv, H, D)
+    torch.cuda.synchronize()
+    assert h3b.device_error() == 0
+    q = np64(qkv)
+    d = H * D
+    ref = oracle.attention(q[:, :d], q[:, d:2 * d], q[:, 2 * d:], H)
+    assert rel_l2(o, ref) < 1e-2 and max_abs(o, ref) < 3e-2
