@@ -233,15 +233,19 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // x < 0, z = |x| / sqrt(2), with erfc(z) from Abramowitz & Stegun, Handbook of
 // Mathematical Functions, formula 7.1.26: erfc(z) ~= (a1 t + a2 t^2 + a3 t^3 +
 // a4 t^4 + a5 t^5) exp(-z^2), t = 1 / (1 + p z), absolute error <= 1.5e-7.
-// The negative side never forms 1 + erf, so it does not cancel.
+// The negative side never forms 1 + erf, so it does not cancel.  t and
+// exp(-z^2) use the MUFU approximations (rcp.approx, ex2.approx: relative
+// errors near 2^-23 and 2^-22), which stay below the formula's own error.
 __device__ __forceinline__ float gelu_erf(float x) {
   const float z = fabsf(x) * 0.70710678118654752f;
-  const float t = __frcp_rn(fmaf(0.3275911f, z, 1.0f));
+  float t, e;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(t) : "f"(fmaf(0.3275911f, z, 1.0f)));
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(-1.4426950408889634f * z * z));
   float p = fmaf(1.061405429f, t, -1.453152027f);
   p = fmaf(p, t, 1.421413741f);
   p = fmaf(p, t, -0.284496736f);
   p = fmaf(p, t, 0.254829592f);
-  const float half_erfc = 0.5f * p * t * exp2f(-1.4426950408889634f * z * z);
+  const float half_erfc = 0.5f * p * t * e;
   return x >= 0.f ? fmaf(-x, half_erfc, x) : x * half_erfc;
 }
 
