@@ -69,9 +69,19 @@ __device__ __forceinline__ void unit_range(int u, int full_tiles, int split, int
   kb1 = (part + 1) * num_kb / split;
 }
 
-template <bool INT8, int EPI>
+// The 32 residual values C[m, n .. n+32) (fp32, n < N).
+__device__ __forceinline__ void load_resid8(const GemmArgs& p, int m, int n, float4 (&dst)[8]) {
+  const float4* src =
+      reinterpret_cast<const float4*>(static_cast<const float*>(p.C) + static_cast<size_t>(m) * p.N + n);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) dst[i] = src[i];
+}
+
+// One 32-column chunk of one row.  PRE (residual epilogue only): cur holds
+// C[m, n .. n+32), loaded ahead by the caller.
+template <bool INT8, int EPI, bool PRE = false>
 __device__ __forceinline__ void epilogue_chunk(const GemmArgs& p, int m, int n, const uint32_t (&r)[32],
-                                               float& row_amax) {
+                                               float& row_amax, const float4* cur = nullptr) {
   const size_t off = static_cast<size_t>(m) * p.N + n;
   if (EPI == H3B_EPI_I32) {
     int4* c = reinterpret_cast<int4*>(static_cast<int*>(p.C) + off);
@@ -112,7 +122,7 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& p, int m, int n, 
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const float4 g = __ldg(g4 + i);
-        float4 a = c[i];
+        float4 a = PRE ? cur[i] : c[i];
         a.x = fmaf(g.x, v[4 * i], a.x);
         a.y = fmaf(g.y, v[4 * i + 1], a.y);
         a.z = fmaf(g.z, v[4 * i + 2], a.z);
@@ -123,7 +133,7 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& p, int m, int n, 
     }
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      float4 a = c[i];
+      float4 a = PRE ? cur[i] : c[i];
       a.x += v[4 * i];
       a.y += v[4 * i + 1];
       a.z += v[4 * i + 2];
@@ -302,8 +312,13 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc_fence_after();
       const int m = mb * BM + q * 32 + lane;
       float row_amax = 0.f;
+      // residual tiles: the next chunk's C values are in flight while this chunk is processed
+      const int c0 = ch * (BN / 64), c1 = (ch + 1) * (BN / 64);
+      const bool pipe = EPI == H3B_EPI_RESID && part < 0 && m < p.M && nb * BN + c0 * 32 < p.N;
+      float4 cnext[8];
+      if (pipe) load_resid8(p, m, nb * BN + c0 * 32, cnext);
 #pragma unroll 1
-      for (int c = ch * (BN / 64); c < (ch + 1) * (BN / 64); ++c) {
+      for (int c = c0; c < c1; ++c) {
         const int n = nb * BN + c * 32;
         if (n >= p.N) break;
         uint32_t r[32];
@@ -326,6 +341,12 @@ __global__ void __launch_bounds__(THREADS, 1)
               dst[i] = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
                                    __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
           }
+        } else if (pipe) {
+          float4 cur[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) cur[i] = cnext[i];
+          if (c + 1 < c1 && n + 32 < p.N) load_resid8(p, m, n + 32, cnext);
+          epilogue_chunk<INT8, EPI, true>(p, m, n, r, row_amax, cur);
         } else if (m < p.M) {
           epilogue_chunk<INT8, EPI>(p, m, n, r, row_amax);
         }
@@ -581,8 +602,12 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int trow = 128 * rank + q * 32 + lane;  // row inside the 256-row tile
       const int m = mb * BM2 + trow;
       float row_amax = 0.f;
+      const int c0 = ch * (BN / 64), c1 = (ch + 1) * (BN / 64);
+      const bool pipe = EPI == H3B_EPI_RESID && part < 0 && m < p.M && nb * BN + c0 * 32 < p.N;
+      float4 cnext[8];
+      if (pipe) load_resid8(p, m, nb * BN + c0 * 32, cnext);
 #pragma unroll 1
-      for (int c = ch * (BN / 64); c < (ch + 1) * (BN / 64); ++c) {
+      for (int c = c0; c < c1; ++c) {
         const int n = nb * BN + c * 32;
         if (n >= p.N) break;
         uint32_t r[32];
@@ -604,6 +629,12 @@ __global__ void __launch_bounds__(THREADS, 1)
               dst[i] = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
                                    __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
           }
+        } else if (pipe) {
+          float4 cur[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) cur[i] = cnext[i];
+          if (c + 1 < c1 && n + 32 < p.N) load_resid8(p, m, n + 32, cnext);
+          epilogue_chunk<INT8, EPI, true>(p, m, n, r, row_amax, cur);
         } else if (m < p.M) {
           epilogue_chunk<INT8, EPI>(p, m, n, r, row_amax);
         }
