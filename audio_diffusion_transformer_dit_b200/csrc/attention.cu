@@ -65,22 +65,6 @@ constexpr int smem_bytes() {
   return 1024 + (2 + KS + VS) * 128 * D * 2 + NUM_BARS * 8 + 16;
 }
 
-// ---------------------------------------------------------------- packed fp32 helpers
-__device__ __forceinline__ uint64_t f2_pack(float a, float b) {
-  return (static_cast<uint64_t>(__float_as_uint(b)) << 32) | __float_as_uint(a);
-}
-__device__ __forceinline__ float f2_lo(uint64_t v) { return __uint_as_float(static_cast<uint32_t>(v)); }
-__device__ __forceinline__ float f2_hi(uint64_t v) { return __uint_as_float(static_cast<uint32_t>(v >> 32)); }
-__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
-}
-__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("add.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
 __device__ __forceinline__ float ex2_mufu(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));

@@ -229,6 +229,28 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// Packed fp32 pairs (f32x2 arithmetic: one instruction for two lanes' worth).
+__device__ __forceinline__ uint64_t f2_pack(float a, float b) {
+  return (static_cast<uint64_t>(__float_as_uint(b)) << 32) | __float_as_uint(a);
+}
+__device__ __forceinline__ float f2_lo(uint64_t v) { return __uint_as_float(static_cast<uint32_t>(v)); }
+__device__ __forceinline__ float f2_hi(uint64_t v) { return __uint_as_float(static_cast<uint32_t>(v >> 32)); }
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
 // GELU(x) = x * Phi(x): x * (1 - erfc(z)/2) for x >= 0 and x * erfc(z)/2 for
 // x < 0, z = |x| / sqrt(2), with erfc(z) from Abramowitz & Stegun, Handbook of
 // Mathematical Functions, formula 7.1.26: erfc(z) ~= (a1 t + a2 t^2 + a3 t^3 +
@@ -247,6 +269,25 @@ __device__ __forceinline__ float gelu_erf(float x) {
   p = fmaf(p, t, 0.254829592f);
   const float half_erfc = 0.5f * p * t * e;
   return x >= 0.f ? fmaf(-x, half_erfc, x) : x * half_erfc;
+}
+
+// gelu_erf of two values, the polynomial and products in packed f32x2 (the
+// same roundings as gelu_erf in each lane: one fma.rn per Horner step).
+__device__ __forceinline__ void gelu_erf2(float& x0, float& x1) {
+  const float z0 = fabsf(x0) * 0.70710678118654752f, z1 = fabsf(x1) * 0.70710678118654752f;
+  float t0, t1, e0, e1;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(t0) : "f"(fmaf(0.3275911f, z0, 1.0f)));
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(t1) : "f"(fmaf(0.3275911f, z1, 1.0f)));
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e0) : "f"(-1.4426950408889634f * z0 * z0));
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e1) : "f"(-1.4426950408889634f * z1 * z1));
+  const uint64_t t = f2_pack(t0, t1);
+  uint64_t p = f2_fma(f2_pack(1.061405429f, 1.061405429f), t, f2_pack(-1.453152027f, -1.453152027f));
+  p = f2_fma(p, t, f2_pack(1.421413741f, 1.421413741f));
+  p = f2_fma(p, t, f2_pack(-0.284496736f, -0.284496736f));
+  p = f2_fma(p, t, f2_pack(0.254829592f, 0.254829592f));
+  const uint64_t h = f2_mul(f2_mul(f2_mul(f2_pack(0.5f, 0.5f), p), t), f2_pack(e0, e1));  // erfc/2
+  x0 = x0 >= 0.f ? fmaf(-x0, f2_lo(h), x0) : x0 * f2_lo(h);
+  x1 = x1 >= 0.f ? fmaf(-x1, f2_hi(h), x1) : x1 * f2_hi(h);
 }
 
 }  // namespace h3b

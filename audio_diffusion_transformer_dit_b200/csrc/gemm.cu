@@ -159,7 +159,7 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& p, int m, int n, 
   }
   if (EPI == H3B_EPI_GELU) {
 #pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = gelu_erf(v[i]);
+    for (int i = 0; i < 32; i += 2) gelu_erf2(v[i], v[i + 1]);
   }
   // bf16 store (BF16, QKV_ROPE, GELU)
   uint32_t w[16];

@@ -199,9 +199,16 @@ __global__ void k_rope_table(float2* __restrict__ table, int F, int H, int Wc, i
 __global__ void k_gelu(const float* __restrict__ x, float* __restrict__ y, size_t n) {
   pdl_trigger();
   pdl_wait();
-  for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
-       i += static_cast<size_t>(gridDim.x) * blockDim.x)
-    y[i] = gelu_erf(x[i]);
+  // pairs through the same packed form the GEMM epilogue uses; an odd last element alone
+  const size_t pairs = n / 2;
+  for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < pairs;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    float a = x[2 * i], b = x[2 * i + 1];
+    gelu_erf2(a, b);
+    y[2 * i] = a;
+    y[2 * i + 1] = b;
+  }
+  if ((n & 1) && blockIdx.x == 0 && threadIdx.x == 0) y[n - 1] = gelu_erf(x[n - 1]);
 }
 
 // ------------------------------------------------------------------ RMSNorm (+ quant)
