@@ -217,7 +217,7 @@ def run_ours(args, wl):
     dev = torch.device("cuda", local)
     if world > 1:
         import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     dm, blocks, x, ws = build_workload(wl, dev)
     loop = wl.steps > 0
     v = torch.empty_like(x) if loop else None
