@@ -347,6 +347,28 @@ def run_ours(args, wl):
             per_eval = sum(fl.block_flops(merged=(fm >= 0 and fm <= l <= fr)) for l in range(len(blocks)))
             flops_step = per_eval * n_fresh
 
+    # Whole-step roofline: every launch's algorithmic work at its own bound's
+    # measured peak, summed over the step, against the untraced step time.
+    tensor_peak = pk.get("bf16_tflops_sustained", pk.get("bf16_tflops"))
+    if not loop:
+        t_ideal = 0.0
+        for k, (c, _) in per.items():
+            a, u, b = kernel_work(k, wl, wl.dtype)
+            if a is None:
+                continue
+            if b == "tensor":
+                t_ideal += c * a / (tensor_peak * (2.0 if u == "TOP/s" else 1.0) * 1e12)
+            else:
+                t_ideal += c * a / (pk.get("hbm_gbs") * 1e9)
+        t_ideal /= args.steps
+        basis = "every traced launch: GEMM/attention work at the sustained bf16 peak (int8 x2), memory kernels at HBM"
+    else:
+        t_ideal = flops_step / (tensor_peak * 1e12)
+        basis = "GEMM + attention work of the step at the sustained bf16 peak (memory-bound kernels < 2 %)"
+    t_step = ms / 1e3 / args.steps
+    step_roofline = {"t_ideal_ms": round(t_ideal * 1e3, 4), "t_ms": round(t_step * 1e3, 4),
+                     "frac": round(t_ideal / t_step, 4), "basis": basis}
+
     # end-to-end through the public API with the tokens in pinned host memory:
     # every step copies its input in and its result out inside the timed
     # region; HostPipeline overlaps those copies with the neighbouring steps'
@@ -413,9 +435,11 @@ def run_ours(args, wl):
                    "global_batch": 1, "parallelism": f"replicas x{world}",
                    "l2": "no flush: per-step working set (weights + activations + workspace) > 126 MB L2"},
         "tflops": round(flops_step * args.steps * world / (ms / 1e3) / 1e12, 2),
-        "roofline": roof, "gpu_launches": my_launches, "clocks": clocks, "kernels": kernels,
+        "roofline": roof, "step_roofline": step_roofline, "gpu_launches": my_launches, "clocks": clocks,
+        "kernels": kernels,
     }
     if loop:
+        line["s_per_fresh_eval"] = round(ms / 1e3 / args.steps / n_fresh, 6)
         line["config"].update({"steps": wl.steps, "reuse": 1 if core else wl.reuse, "fresh_evals": n_fresh,
                                "token_reduction": [wl.merge_first, wl.merge_last],
                                "unmerge": "delta" if args.unmerge_delta else "broadcast"})
@@ -468,6 +492,16 @@ def oracle_block_rate(wl, rows_a=64, rows_b=256, reps=1):
     return a, b, t_used
 
 
+def cpu_model():
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def cpu_threads():
     try:
         from threadpoolctl import threadpool_info
@@ -483,13 +517,15 @@ def cpu_baseline(wl, budget_s=30.0):
     if wl.steps > 0:
         n_fresh = len([i for i in range(wl.steps) if i % wl.reuse == 0 or i == wl.steps - 1])
         seconds = per_block * n_blocks * n_fresh / wl.steps
-        return {"value": round(seconds, 3), "unit": "s/step", "cores": cpu_threads(), "kind": "oracle",
+        return {"value": round(seconds, 3), "unit": "s/step", "cores": cpu_threads(), "cpu_model": cpu_model(),
+                "kind": "oracle",
                 "sample": f"oracle block forward on this host with 64 and 256 query rows (all {wl.seq} keys); "
                           f"full block {per_block:.2f} s extrapolated linearly in rows, x{n_blocks} blocks "
                           f"x{n_fresh} fresh evals / {wl.steps} steps (merged blocks counted at full S); "
                           f"{used:.1f} s of CPU time"}
     value = wl.seq / per_block
-    return {"value": round(value, 3), "unit": "tokens/s", "cores": cpu_threads(), "kind": "oracle",
+    return {"value": round(value, 3), "unit": "tokens/s", "cores": cpu_threads(), "cpu_model": cpu_model(),
+            "kind": "oracle",
             "sample": f"oracle block forward (fp64 numpy) with 64 and 256 sampled query rows, keys/values over "
                       f"all {wl.seq} tokens; full-block time {per_block:.2f} s = fixed + per-row cost x {wl.seq} "
                       f"rows, fitted from the two runs ({used:.1f} s of CPU time)"}
@@ -528,8 +564,8 @@ def run_reference(args, wl):
             "higher_is_better": hib, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (same seeded inputs)", "config": {"workload": wl.name, "seq_len": wl.seq,
                                                                  "d": wl.d, "blocks": blocks},
-            "cpu_baseline": {"value": round(value, 4), "unit": unit, "cores": cpu_threads(), "kind": "oracle",
-                             "sample": sample},
+            "cpu_baseline": {"value": round(value, 4), "unit": unit, "cores": cpu_threads(),
+                             "cpu_model": cpu_model(), "kind": "oracle", "sample": sample},
             "e2e": {"value": round(value, 4), "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
