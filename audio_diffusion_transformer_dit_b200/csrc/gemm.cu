@@ -69,19 +69,121 @@ __device__ __forceinline__ void unit_range(int u, int full_tiles, int split, int
   kb1 = (part + 1) * num_kb / split;
 }
 
-// The 32 residual values C[m, n .. n+32) (fp32, n < N).
-__device__ __forceinline__ void load_resid8(const GemmArgs& p, int m, int n, float4 (&dst)[8]) {
-  const float4* src =
-      reinterpret_cast<const float4*>(static_cast<const float*>(p.C) + static_cast<size_t>(m) * p.N + n);
+// Residual epilogue through shared memory.  TMEM hands each thread one row of
+// a 32x32 chunk; stored straight to global memory, every 16-byte access of a
+// warp would touch 32 rows (32 cache lines).  Each epilogue warp instead parks
+// the chunk in a 4 KB buffer of its own (16-byte groups XOR-swizzled by row:
+// conflict-free both ways) and reads it back four rows per instruction, eight
+// lanes covering one 128-byte row segment, so the residual read and write
+// touch 4 lines per instruction.
+constexpr int STG_FLOATS = 32 * 32;                   // one warp's buffer
+constexpr int STG_BYTES = EPI_WARPS * STG_FLOATS * 4;  // 32 KB per CTA
+
+__device__ __forceinline__ int stg_off(int row, int grp) { return row * 32 + ((grp ^ (row & 7)) << 2); }
+
+// Row-per-thread values -> the warp's buffer (all lanes).
+__device__ __forceinline__ void stage_put(float* stg, int lane, const float (&v)[32]) {
+  __syncwarp();  // the previous chunk has been read back
 #pragma unroll
-  for (int i = 0; i < 8; ++i) dst[i] = src[i];
+  for (int j = 0; j < 8; ++j)
+    *reinterpret_cast<float4*>(stg + stg_off(lane, j)) = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+  __syncwarp();
 }
 
-// One 32-column chunk of one row.  PRE (residual epilogue only): cur holds
-// C[m, n .. n+32), loaded ahead by the caller.
-template <bool INT8, int EPI, bool PRE = false>
+// Element group i of this lane: chunk row 4i + lane/8, columns 4(lane%8) .. +4.
+__device__ __forceinline__ float4 stage_get(const float* stg, int lane, int i) {
+  return *reinterpret_cast<const float4*>(stg + stg_off(4 * i + (lane >> 3), lane & 7));
+}
+
+// The residual values of a chunk in the same row-contiguous lane order
+// (rows row0 .. row0+32 of C, columns n .. n+32; rows >= M read as 0).
+__device__ __forceinline__ void load_resid_rows(const GemmArgs& p, int row0, int n, int lane, float4 (&dst)[8]) {
+  const float* C = static_cast<const float*>(p.C) + n + 4 * (lane & 7);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int m = row0 + 4 * i + (lane >> 3);
+    dst[i] = m < p.M ? *reinterpret_cast<const float4*>(C + static_cast<size_t>(m) * p.N) : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+}
+
+// Row-per-thread fp32 values of one chunk (dequantised for INT8; row m >= M gives 0 scale).
+template <bool INT8>
+__device__ __forceinline__ void chunk_values(const GemmArgs& p, int m, int n, const uint32_t (&r)[32], float (&v)[32]) {
+  if (INT8) {
+    const float sa = m < p.M ? p.sa[m] : 0.f;
+    const float4* sb4 = reinterpret_cast<const float4*>(p.sb + n);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float4 sb = __ldg(sb4 + i);
+      v[4 * i + 0] = static_cast<float>(static_cast<int>(r[4 * i + 0])) * sa * sb.x;
+      v[4 * i + 1] = static_cast<float>(static_cast<int>(r[4 * i + 1])) * sa * sb.y;
+      v[4 * i + 2] = static_cast<float>(static_cast<int>(r[4 * i + 2])) * sa * sb.z;
+      v[4 * i + 3] = static_cast<float>(static_cast<int>(r[4 * i + 3])) * sa * sb.w;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+  }
+}
+
+// C[m, n .. n+32) += gate[class(m), n ..] * staged values (gate 1 when absent;
+// fmaf(1, v, c) rounds exactly like c + v), res = the prefetched C values.
+__device__ __forceinline__ void resid_rows(const GemmArgs& p, const float* stg, int row0, int n, int lane,
+                                           const float4 (&res)[8]) {
+  const int col = n + 4 * (lane & 7);
+  float4 g0 = make_float4(1.f, 1.f, 1.f, 1.f), g1 = g0;
+  if (p.gate) {
+    g0 = __ldg(reinterpret_cast<const float4*>(p.gate + col));
+    if (p.gate_split < p.M) g1 = __ldg(reinterpret_cast<const float4*>(p.gate + static_cast<size_t>(p.gate_stride) + col));
+  }
+  float* C = static_cast<float*>(p.C) + col;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int m = row0 + 4 * i + (lane >> 3);
+    if (m < p.M) {
+      const float4 v = stage_get(stg, lane, i);
+      const float4 g = m >= p.gate_split ? g1 : g0;
+      float4 a = res[i];
+      a.x = fmaf(g.x, v.x, a.x);
+      a.y = fmaf(g.y, v.y, a.y);
+      a.z = fmaf(g.z, v.z, a.z);
+      a.w = fmaf(g.w, v.w, a.w);
+      *reinterpret_cast<float4*>(C + static_cast<size_t>(m) * p.N) = a;
+    }
+  }
+}
+
+// Staged chunk -> rows trow0 .. trow0+32 of a tile-shaped fp32 partial (row stride BN).
+__device__ __forceinline__ void partial_rows(float* part, const float* stg, int trow0, int ccol, int lane) {
+  float* dst = part + ccol + 4 * (lane & 7);
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    *reinterpret_cast<float4*>(dst + static_cast<size_t>(trow0 + 4 * i + (lane >> 3)) * BN) = stage_get(stg, lane, i);
+}
+
+// One chunk of a residual tile (whole tile or K-part), all lanes of the warp.
+template <bool INT8>
+__device__ __forceinline__ void resid_chunk(const GemmArgs& p, float* stg, int lane, int row0, int n, int ccol,
+                                            const uint32_t (&r)[32], float* part, int trow0, float4 (&cnext)[8],
+                                            bool more) {
+  float v[32];
+  chunk_values<INT8>(p, row0 + lane, n, r, v);
+  stage_put(stg, lane, v);
+  if (part) {
+    partial_rows(part, stg, trow0, ccol, lane);
+    return;
+  }
+  float4 cur[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) cur[i] = cnext[i];
+  if (more) load_resid_rows(p, row0, n + 32, lane, cnext);
+  resid_rows(p, stg, row0, n, lane, cur);
+}
+
+// One 32-column chunk of one row (every epilogue but the residual one).
+template <bool INT8, int EPI>
 __device__ __forceinline__ void epilogue_chunk(const GemmArgs& p, int m, int n, const uint32_t (&r)[32],
-                                               float& row_amax, const float4* cur = nullptr) {
+                                               float& row_amax) {
   const size_t off = static_cast<size_t>(m) * p.N + n;
   if (EPI == H3B_EPI_I32) {
     int4* c = reinterpret_cast<int4*>(static_cast<int*>(p.C) + off);
@@ -112,34 +214,6 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& p, int m, int n, 
     float4* c = reinterpret_cast<float4*>(static_cast<float*>(p.C) + off);
 #pragma unroll
     for (int i = 0; i < 8; ++i) c[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-    return;
-  }
-  if (EPI == H3B_EPI_RESID) {
-    float4* c = reinterpret_cast<float4*>(static_cast<float*>(p.C) + off);
-    if (p.gate) {  // gated residual update
-      const float4* g4 =
-          reinterpret_cast<const float4*>(p.gate + (m >= p.gate_split ? static_cast<size_t>(p.gate_stride) : 0) + n);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float4 g = __ldg(g4 + i);
-        float4 a = PRE ? cur[i] : c[i];
-        a.x = fmaf(g.x, v[4 * i], a.x);
-        a.y = fmaf(g.y, v[4 * i + 1], a.y);
-        a.z = fmaf(g.z, v[4 * i + 2], a.z);
-        a.w = fmaf(g.w, v[4 * i + 3], a.w);
-        c[i] = a;
-      }
-      return;
-    }
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      float4 a = PRE ? cur[i] : c[i];
-      a.x += v[4 * i];
-      a.y += v[4 * i + 1];
-      a.z += v[4 * i + 2];
-      a.w += v[4 * i + 3];
-      c[i] = a;
-    }
     return;
   }
   if (EPI == H3B_EPI_QKV_ROPE) {
@@ -185,7 +259,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * A_STAGE;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * B_STAGE);
+  float* stg_all = reinterpret_cast<float*>(sB + STAGES * B_STAGE);  // residual staging (RESID only)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * B_STAGE + (EPI == H3B_EPI_RESID ? STG_BYTES : 0));
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NUM_BARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -314,9 +389,14 @@ __global__ void __launch_bounds__(THREADS, 1)
       float row_amax = 0.f;
       // residual tiles: the next chunk's C values are in flight while this chunk is processed
       const int c0 = ch * (BN / 64), c1 = (ch + 1) * (BN / 64);
-      const bool pipe = EPI == H3B_EPI_RESID && part < 0 && m < p.M && nb * BN + c0 * 32 < p.N;
+      float* const stg = stg_all + (warp - 2) * STG_FLOATS;
+      float* const part_dst =
+          EPI == H3B_EPI_RESID && part >= 0
+              ? p.partial + (static_cast<size_t>(t - p.full_tiles) * p.split + part) * (BM * BN)
+              : nullptr;
       float4 cnext[8];
-      if (pipe) load_resid8(p, m, nb * BN + c0 * 32, cnext);
+      if (EPI == H3B_EPI_RESID && !part_dst && nb * BN + c0 * 32 < p.N)
+        load_resid_rows(p, m - lane, nb * BN + c0 * 32, lane, cnext);
 #pragma unroll 1
       for (int c = c0; c < c1; ++c) {
         const int n = nb * BN + c * 32;
@@ -324,29 +404,10 @@ __global__ void __launch_bounds__(THREADS, 1)
         uint32_t r[32];
         tmem_ld32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN + c * 32, r);
         tmem_ld_wait();
-        if (EPI == H3B_EPI_RESID && part >= 0) {
-          // K-part of a tail tile: fp32 partial into its scratch slot (added into C later, in part order)
-          float4* dst = reinterpret_cast<float4*>(p.partial + (static_cast<size_t>(t - p.full_tiles) * p.split + part) *
-                                                                  (BM * BN) + (q * 32 + lane) * BN + c * 32);
-          if (INT8) {
-            float v[32];
-            const float sa = m < p.M ? p.sa[m] : 0.f;
-#pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = static_cast<float>(static_cast<int>(r[i])) * sa * __ldg(p.sb + n + i);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-          } else {
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-              dst[i] = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
-                                   __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
-          }
-        } else if (pipe) {
-          float4 cur[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) cur[i] = cnext[i];
-          if (c + 1 < c1 && n + 32 < p.N) load_resid8(p, m, n + 32, cnext);
-          epilogue_chunk<INT8, EPI, true>(p, m, n, r, row_amax, cur);
+        if (EPI == H3B_EPI_RESID) {
+          // K-parts of tail tiles write fp32 partials (added into C later, in part order)
+          resid_chunk<INT8>(p, stg, lane, m - lane, n, c * 32, r, part_dst, q * 32, cnext,
+                            c + 1 < c1 && n + 32 < p.N);
         } else if (m < p.M) {
           epilogue_chunk<INT8, EPI>(p, m, n, r, row_amax);
         }
@@ -407,6 +468,7 @@ constexpr int HALF_STAGE = 128 * KBYTES;  // 16 KB: 128 rows of A or B
 constexpr int STAGES2 = 6;
 constexpr int NUM_BARS2 = 2 * STAGES2 + 5;
 constexpr int SMEM2_BYTES = 1024 + STAGES2 * 2 * HALF_STAGE + NUM_BARS2 * 8 + 16;
+static_assert(SMEM2_BYTES + STG_BYTES <= 232448 && SMEM_BYTES + STG_BYTES <= 232448, "shared memory per CTA");
 constexpr uint32_t PEER_BIT_CLEAR = 0xFEFFFFFFu;  // shared::cluster address of the same offset in rank 0
 
 __device__ __forceinline__ uint32_t cluster_rank() {
@@ -466,7 +528,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES2 * HALF_STAGE;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES2 * HALF_STAGE);
+  float* stg_all = reinterpret_cast<float*>(sB + STAGES2 * HALF_STAGE);  // residual staging (RESID only)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES2 * HALF_STAGE + (EPI == H3B_EPI_RESID ? STG_BYTES : 0));
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NUM_BARS2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -603,9 +666,14 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int m = mb * BM2 + trow;
       float row_amax = 0.f;
       const int c0 = ch * (BN / 64), c1 = (ch + 1) * (BN / 64);
-      const bool pipe = EPI == H3B_EPI_RESID && part < 0 && m < p.M && nb * BN + c0 * 32 < p.N;
+      float* const stg = stg_all + (warp - 2) * STG_FLOATS;
+      float* const part_dst =
+          EPI == H3B_EPI_RESID && part >= 0
+              ? p.partial + (static_cast<size_t>(t - p.full_tiles) * p.split + part) * (BM2 * BN)
+              : nullptr;
       float4 cnext[8];
-      if (pipe) load_resid8(p, m, nb * BN + c0 * 32, cnext);
+      if (EPI == H3B_EPI_RESID && !part_dst && nb * BN + c0 * 32 < p.N)
+        load_resid_rows(p, m - lane, nb * BN + c0 * 32, lane, cnext);
 #pragma unroll 1
       for (int c = c0; c < c1; ++c) {
         const int n = nb * BN + c * 32;
@@ -613,28 +681,9 @@ __global__ void __launch_bounds__(THREADS, 1)
         uint32_t r[32];
         tmem_ld32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN + c * 32, r);
         tmem_ld_wait();
-        if (EPI == H3B_EPI_RESID && part >= 0) {
-          float4* dst = reinterpret_cast<float4*>(
-              p.partial + (static_cast<size_t>(t - p.full_tiles) * p.split + part) * (BM2 * BN) + trow * BN + c * 32);
-          if (INT8) {
-            float v[32];
-            const float sa = m < p.M ? p.sa[m] : 0.f;
-#pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = static_cast<float>(static_cast<int>(r[i])) * sa * __ldg(p.sb + n + i);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-          } else {
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-              dst[i] = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
-                                   __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
-          }
-        } else if (pipe) {
-          float4 cur[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) cur[i] = cnext[i];
-          if (c + 1 < c1 && n + 32 < p.N) load_resid8(p, m, n + 32, cnext);
-          epilogue_chunk<INT8, EPI, true>(p, m, n, r, row_amax, cur);
+        if (EPI == H3B_EPI_RESID) {
+          resid_chunk<INT8>(p, stg, lane, m - lane, n, c * 32, r, part_dst, trow - lane, cnext,
+                            c + 1 < c1 && n + 32 < p.N);
         } else if (m < p.M) {
           epilogue_chunk<INT8, EPI>(p, m, n, r, row_amax);
         }
@@ -712,7 +761,7 @@ cudaError_t launch_gemm(const Ctx& c, const void* A, const void* B, int ab_int8,
       !encode_tmap_2d(&tb, dt, eb, B, args.K, args.N, static_cast<uint64_t>(args.K) * eb, KBYTES / eb,
                       pair ? 128 : BN))
     return cudaErrorInvalidValue;
-  const int smem = pair ? SMEM2_BYTES : SMEM_BYTES;
+  const int smem = (pair ? SMEM2_BYTES : SMEM_BYTES) + (epi == H3B_EPI_RESID ? STG_BYTES : 0);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const int num_m = (args.M + TM - 1) / TM, num_n = (args.N + BN - 1) / BN;
