@@ -464,10 +464,17 @@ __global__ void __launch_bounds__(BN) k_splitk_add(float* __restrict__ C, const 
 // ranks' barriers (multicast commit); rank 1's epilogue releases the
 // accumulator on rank 0's barrier.  No TMA load uses multicast.
 constexpr int BM2 = 256;
-constexpr int HALF_STAGE = 128 * KBYTES;  // 16 KB: 128 rows of A or B
-constexpr int STAGES2 = 6;
+constexpr int HALF_STAGE = 128 * KBYTES;  // 16 KB: 128 rows of A or B, one 128-byte K atom
+constexpr int ATOMS_RING = 6;              // K atoms of A (and of B) in the ring
+// K atoms per pipeline stage.  Two (128 bf16 / 256 int8 elements: eight MMAs
+// per barrier wait and commit) leave the issuing thread slack to absorb the
+// ALU-heavy GELU and RoPE epilogue warps that share its SM sub-partition; the
+// residual GEMMs keep one atom per stage (finer release: more bytes in flight
+// for their streamed A operand).
+__host__ __device__ constexpr int pair_atoms(int epi) { return epi == H3B_EPI_RESID ? 1 : 2; }
+constexpr int STAGES2 = ATOMS_RING;  // barrier slots (the most stages any epilogue uses)
 constexpr int NUM_BARS2 = 2 * STAGES2 + 5;
-constexpr int SMEM2_BYTES = 1024 + STAGES2 * 2 * HALF_STAGE + NUM_BARS2 * 8 + 16;
+constexpr int SMEM2_BYTES = 1024 + ATOMS_RING * 2 * HALF_STAGE + NUM_BARS2 * 8 + 16;
 static_assert(SMEM2_BYTES + STG_BYTES <= 232448 && SMEM_BYTES + STG_BYTES <= 232448, "shared memory per CTA");
 constexpr uint32_t PEER_BIT_CLEAR = 0xFEFFFFFFu;  // shared::cluster address of the same offset in rank 0
 
@@ -527,9 +534,10 @@ __global__ void __launch_bounds__(THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
-  uint8_t* sB = smem + STAGES2 * HALF_STAGE;
-  float* stg_all = reinterpret_cast<float*>(sB + STAGES2 * HALF_STAGE);  // residual staging (RESID only)
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES2 * HALF_STAGE + (EPI == H3B_EPI_RESID ? STG_BYTES : 0));
+  constexpr int AT = pair_atoms(EPI), NST = ATOMS_RING / AT, STAGE2 = AT * HALF_STAGE;
+  uint8_t* sB = smem + ATOMS_RING * HALF_STAGE;
+  float* stg_all = reinterpret_cast<float*>(sB + ATOMS_RING * HALF_STAGE);  // residual staging (RESID only)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + ATOMS_RING * HALF_STAGE + (EPI == H3B_EPI_RESID ? STG_BYTES : 0));
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NUM_BARS2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -573,7 +581,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int num_m = (p.M + BM2 - 1) / BM2, num_n = (p.N + BN - 1) / BN, num_tiles = num_m * num_n;
   const int num_units = p.split > 1 ? p.full_tiles + (num_tiles - p.full_tiles) * p.split : num_tiles;
   constexpr int KE = INT8 ? 128 : 64;
-  const int num_kb = p.K / KE;
+  constexpr int KS = AT * KE;         // K elements per stage
+  const int num_kb = (p.K + KS - 1) / KS;  // stages; the last may hold one atom (K is a multiple of KE)
 
   if (warp == 0) {
     if (lane == 0) {
@@ -590,14 +599,17 @@ __global__ void __launch_bounds__(THREADS, 1)
             break;
           }
           const uint32_t fb = full0 + 8 * stage;
-          if (leader) mbar_arrive_expect_tx(fb, 4 * HALF_STAGE);  // both ranks' A and B halves
-          tma_load_2d_pair(smem_u32(sA + stage * HALF_STAGE), &tmA, fb & PEER_BIT_CLEAR, kb * KE,
-                           mb * BM2 + 128 * rank);
-          tma_load_2d_pair(smem_u32(sB + stage * HALF_STAGE), &tmB, fb & PEER_BIT_CLEAR, kb * KE,
-                           nb * BN + 128 * rank);
+          const int na = AT == 1 ? 1 : min(AT, (p.K - kb * KS) / KE);
+          if (leader) mbar_arrive_expect_tx(fb, 4 * HALF_STAGE * na);  // both ranks' A and B halves
+          for (int a = 0; a < na; ++a) {
+            tma_load_2d_pair(smem_u32(sA + stage * STAGE2 + a * HALF_STAGE), &tmA, fb & PEER_BIT_CLEAR,
+                             kb * KS + a * KE, mb * BM2 + 128 * rank);
+            tma_load_2d_pair(smem_u32(sB + stage * STAGE2 + a * HALF_STAGE), &tmB, fb & PEER_BIT_CLEAR,
+                             kb * KS + a * KE, nb * BN + 128 * rank);
+          }
           issued |= 1u << stage;
           issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
-          if (++stage == STAGES2) {
+          if (++stage == NST) {
             stage = 0;
             phase ^= 1;
           }
@@ -605,7 +617,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (!ok) break;
       }
       if (leader)  // rank 0's stage barriers count both ranks' bytes
-        for (int s = 0; s < STAGES2; ++s)
+        for (int s = 0; s < NST; ++s)
           if ((issued >> s) & 1) mbar_drain(full0 + 8 * s, (issued_par >> s) & 1);
     }
   } else if (warp == 1) {
@@ -626,17 +638,21 @@ __global__ void __launch_bounds__(THREADS, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t a0 = smem_u32(sA + stage * HALF_STAGE), b0 = smem_u32(sB + stage * HALF_STAGE);
+          const uint32_t a0 = smem_u32(sA + stage * STAGE2), b0 = smem_u32(sB + stage * STAGE2);
+          const int nk = AT == 1 ? KBYTES / 32 : min(AT, (p.K - kb * KS) / KE) * (KBYTES / 32);
 #pragma unroll
-          for (int k = 0; k < KBYTES / 32; ++k) {
-            const uint64_t ad = desc_sw128_k(a0 + 32 * k), bd = desc_sw128_k(b0 + 32 * k);
-            if (INT8)
-              mma2_i8(d_tmem, ad, bd, idesc, (kb > kb0) || k != 0);
-            else
-              mma2_bf16(d_tmem, ad, bd, idesc, (kb > kb0) || k != 0);
+          for (int k = 0; k < AT * (KBYTES / 32); ++k) {
+            if (AT == 1 || k < nk) {
+              const uint32_t off = (k / (KBYTES / 32)) * HALF_STAGE + 32 * (k % (KBYTES / 32));
+              const uint64_t ad = desc_sw128_k(a0 + off), bd = desc_sw128_k(b0 + off);
+              if (INT8)
+                mma2_i8(d_tmem, ad, bd, idesc, (kb > kb0) || k != 0);
+              else
+                mma2_bf16(d_tmem, ad, bd, idesc, (kb > kb0) || k != 0);
+            }
           }
           commit2_both(empty0 + 8 * stage);  // frees the stage in both ranks
-          if (++stage == STAGES2) {
+          if (++stage == NST) {
             stage = 0;
             phase ^= 1;
           }
@@ -793,7 +809,9 @@ cudaError_t launch_gemm(const Ctx& c, const void* A, const void* B, int ab_int8,
   args.split = 1;
   args.full_tiles = tiles;
   args.partial = nullptr;
-  const int num_kb = args.K / (KBYTES / eb);
+  // K steps (stages) of the kernel that runs: two atoms per stage for pairs
+  const int ke = (pair ? pair_atoms(epi) : 1) * (KBYTES / eb);
+  const int num_kb = (args.K + ke - 1) / ke;
   const int rem = tiles % grid;
   if (epi == H3B_EPI_RESID && scratch && tiles > grid && rem > 0 && 3 * rem <= grid) {
     int split = grid / rem;

@@ -312,12 +312,14 @@ def test_exp2_poly_error_bound(cuda_dev):
     assert np64(h3b.exp2_poly(torch.tensor([-300.0, -126.0], device=cuda_dev))).max() < 2.0 ** -125
 
 
+@pytest.mark.parametrize("ktail", [False, True])
 @pytest.mark.parametrize("int8", [False, True])
-def test_gemm_resid_split_tail(cuda_dev, int8):
-    """A residual GEMM with a nearly empty last wave (600 tiles on 148 SMs)
-    splits its tail tiles along K; with and without scratch it matches the
-    oracle, and two split runs agree bit for bit."""
-    M, N, K = 6400, 3072, 1024
+def test_gemm_resid_split_tail(cuda_dev, int8, ktail):
+    """A residual GEMM with a nearly empty last wave (300 pair tiles) splits its
+    tail tiles along K; with and without scratch it matches the oracle, and two
+    split runs agree bit for bit.  ktail: K ends on a half stage."""
+    M, N = 6400, 3072
+    K = (1152 if int8 else 1088) if ktail else 1024
     if int8:
         A, B = wlmod.int8_tensor((M, K), 31, cuda_dev), wlmod.int8_tensor((N, K), 32, cuda_dev)
         sa = wlmod.uniform_tensor((M,), 33, cuda_dev, 0.001, 0.003)
@@ -364,7 +366,8 @@ def test_attention_key_split_tail(cuda_dev, S, H, D):
 
 
 # shapes whose 256x256 tiles fill a wave of CTA pairs -> the 2-SM (cta_group::2) kernel
-PAIR_SHAPES = [(2048, 2560, 1024), (2100, 2592, 512), (6528, 3072, 256)]
+# the last two end K on a half stage (one 128-byte atom of the two a pair stage holds)
+PAIR_SHAPES = [(2048, 2560, 1024), (2100, 2592, 512), (6528, 3072, 256), (2048, 2560, 192), (2100, 2592, 64)]
 
 
 @pytest.mark.parametrize("M,N,K", PAIR_SHAPES)
@@ -382,7 +385,7 @@ def test_gemm_pair_bf16(cuda_dev, M, N, K):
 
 @pytest.mark.parametrize("M,N,K", PAIR_SHAPES)
 def test_gemm_pair_int8_i32_bitexact(cuda_dev, M, N, K):
-    K = max(K, 128)
+    K = K if K % 128 == 0 else 2 * K  # int8 K steps are 128 wide: 192 -> 384 (1.5 stages), 64 -> 128
     A = wlmod.int8_tensor((M, K), 43, cuda_dev)
     B = wlmod.int8_tensor((N, K), 44, cuda_dev)
     C = torch.zeros((M, N), dtype=torch.int32, device=cuda_dev)
