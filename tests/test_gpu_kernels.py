@@ -123,7 +123,10 @@ def test_rmsnorm_int8(cuda_dev, rows, d):
 
 
 # ----------------------------------------------------------------------------- quantisation
-@pytest.mark.parametrize("rows,k", [(1, 8), (33, 256), (300, 5120), (17, 20480), (5, 32768)])
+# one warp per row for 1024 <= k <= 6144 (ragged lanes at 1032, the widest at
+# 6144), one CTA per row outside that range (6152 just above it)
+@pytest.mark.parametrize("rows,k", [(1, 8), (33, 256), (300, 5120), (17, 20480), (5, 32768), (37, 1024), (9, 1032),
+                                    (41, 6144), (6, 6152)])
 def test_quantize_weights_bitexact(cuda_dev, rows, k):
     w = (wlmod.normal_tensor((rows, k), 9, cuda_dev) * 0.02).to(torch.bfloat16)
     w[0, :] = 0  # zero row -> s = 0, q = 0
@@ -134,8 +137,11 @@ def test_quantize_weights_bitexact(cuda_dev, rows, k):
     assert np.array_equal(q.cpu().numpy(), qr)
 
 
-def test_quantize_rows_absmax_bitexact(cuda_dev):
-    a = (wlmod.normal_tensor((77, 1024), 10, cuda_dev) * 3).to(torch.bfloat16)
+# one CTA per row for k a multiple of 16 up to 32768 (1..8 groups of 16 per
+# thread, ragged at 12304); the 2-D grid path for k a multiple of 8 only
+@pytest.mark.parametrize("rows,k", [(77, 1024), (13, 12288), (5, 20480), (3, 32768), (4, 12304), (6, 1000)])
+def test_quantize_rows_absmax_bitexact(cuda_dev, rows, k):
+    a = (wlmod.normal_tensor((rows, k), 10, cuda_dev) * 3).to(torch.bfloat16)
     amax = a.float().abs().amax(dim=1).contiguous()
     q, s = h3b.quantize_rows_absmax(a, amax)
     torch.cuda.synchronize()
