@@ -92,7 +92,8 @@ def sample_rows(S, n_video, k=48, seed=0):
 @pytest.mark.parametrize("name,layer,merged", [("block_d3072_s6400", 0, False),
                                                ("stack8_d5120_s6528", 0, False),
                                                ("stack8_d5120_s6528", 7, False),
-                                               ("loop45_d5120_s6528", 20, True)])
+                                               ("loop45_d5120_s6528", 20, True),
+                                               ("preview40_d5120_s2784", 39, False)])
 def test_block_full_size_sampled(cuda_dev, name, layer, merged):
     wl = wlmod.WORKLOADS[name]
     x0, got, w = run_block(wl, layer, cuda_dev, merged=merged)
@@ -199,6 +200,34 @@ def test_denoise_few_steps_layer_subset_vs_oracle(cuda_dev, steps, reuse):
     ref, nf_ref = oracle.denoise(np64(x0), [host_weights(w) for w in ws_], wl, steps, reuse)
     assert nf == nf_ref
     assert rel_l2(x, ref) <= 1e-2 and max_abs(x, ref) <= 5e-2
+
+
+@pytest.mark.slow
+def test_loop45_full_size_equals_composition(cuda_dev):
+    """The benched loop itself (45 blocks at d = 5120, S = 6528, tokens merged
+    over blocks 15..29, 20 steps, whole-velocity reuse 2) equals, bit for bit,
+    its definition written with the separately verified entry points: on a
+    fresh step the velocity is the stack output of the current x, and every
+    step is the Euler update over the sigma grid 1 - i/N."""
+    wl = wlmod.WORKLOADS["loop45_d5120_s6528"]
+    dm = h3b.dims_of(wl)
+    blocks = [h3b.Block.from_dict(wlmod.block_weights(wl, l, cuda_dev)) for l in range(wl.n_blocks)]
+    ws = h3b.workspace(dm, h3b.BF16, True)
+    x0 = wlmod.initial_tokens(wl, cuda_dev)
+    x = x0.clone()
+    v = torch.empty_like(x)
+    nf = h3b.denoise(dm, blocks, x, v, ws, wl.steps, wl.reuse, wl.merge_first, wl.merge_last)
+    y = x0.clone()
+    sig = oracle.sigmas(wl.steps)
+    vel = None
+    for i in range(wl.steps):
+        if oracle.is_fresh(i, wl.steps, wl.reuse):
+            vel = h3b.stack_forward(dm, blocks, y.clone(), ws, wl.merge_first, wl.merge_last)
+        h3b.flow_step(y, vel, float(sig[i]), float(sig[i + 1]))
+    torch.cuda.synchronize()
+    assert h3b.device_error() == 0
+    assert nf == len(oracle.fresh_steps(wl.steps, wl.reuse)) == 11
+    assert torch.isfinite(x).all() and torch.equal(x, y)
 
 
 def test_denoise_fresh_counts(cuda_dev):
