@@ -40,7 +40,7 @@ __all__ = [
     "READINGS", "PINS", "MOD_FIELDS", "block_forward_cond", "stack_forward_cond", "denoise_cond",
     "linear", "rmsnorm", "gelu", "rope_sections", "token_positions", "rope_angles", "apply_rope",
     "attention", "block_forward", "stack_forward", "token_merge", "token_unmerge",
-    "quantize_rows", "dequantize_rows", "int8_matmul", "dequant_weights", "block_forward_w8a8",
+    "quantize_rows", "quantize_rows_known_max", "dequantize_rows", "int8_matmul", "dequant_weights", "block_forward_w8a8",
     "sigmas", "is_fresh", "fresh_steps", "flow_step", "denoise",
     "token_unmerge_delta", "stack_forward_ex", "denoise_core",
 ]
@@ -92,6 +92,8 @@ PINS = {
                      "permutation equivariance without RoPE; row sampling = full rows",
     "token_merge/unmerge": "explicit (f, r, c) loops; unmerge(merge(x)) = x on pair-constant x",
     "quantize_rows": "hand-computed codes incl. half-even ties; zero row",
+    "quantize_rows_known_max": "hand-computed codes with a given max below the row's (clamping), zero max; "
+                               "equals quantize_rows at the row's own max",
     "int8_matmul": "pure-Python integer dot products",
     "sigmas/fresh/denoise": "fresh counts 20/11/8 at 20 steps (control table); v = 0 identity; "
                             "single-step closed form",
@@ -354,7 +356,15 @@ def quantize_rows(a):
     s = 0 and q = 0.  Used for weights (per output channel) and for
     activations (per token)."""
     a32 = np.asarray(a, dtype=np.float32)
-    s = (np.max(np.abs(a32), axis=1) / np.float32(127.0)).astype(np.float32)
+    return quantize_rows_known_max(a32, np.max(np.abs(a32), axis=1))
+
+
+def quantize_rows_known_max(a, row_max):
+    """The same rule with each row's maximum given (the FC2 input takes it from
+    the FC1 epilogue): s = row_max/127 (fp32); values beyond row_max clamp to
+    +-127; row_max = 0 gives s = 0 and q = 0."""
+    a32 = np.asarray(a, dtype=np.float32)
+    s = (np.asarray(row_max, dtype=np.float32) / np.float32(127.0)).astype(np.float32)
     q = np.zeros(a32.shape, dtype=np.float32)
     nz = s > 0
     q[nz] = np.rint(a32[nz] / s[nz, None])

@@ -149,6 +149,22 @@ def test_quantize_rows_absmax_bitexact(cuda_dev, rows, k):
     assert np.array_equal(s.cpu().numpy(), sr) and np.array_equal(q.cpu().numpy(), qr)
 
 
+def test_quantize_rows_absmax_below_true_max_bitexact(cuda_dev):
+    """A caller-given row maximum smaller than the row's true maximum (half,
+    a quarter) and a zero maximum: values beyond it clamp to +-127, the rest
+    round as usual, bit for bit with the oracle's known-max rule."""
+    rows, k = 24, 2048
+    a = (wlmod.normal_tensor((rows, k), 12, cuda_dev) * 2).to(torch.bfloat16)
+    true_max = a.float().abs().amax(dim=1)
+    frac = torch.tensor([1.0, 0.5, 0.25, 0.0] * (rows // 4), device=cuda_dev)
+    amax = (true_max * frac).contiguous()
+    q, s = h3b.quantize_rows_absmax(a, amax)
+    torch.cuda.synchronize()
+    qr, sr = oracle.quantize_rows_known_max(a.float().cpu().numpy(), amax.cpu().numpy())
+    assert np.array_equal(s.cpu().numpy(), sr) and np.array_equal(q.cpu().numpy(), qr)
+    assert (np.abs(qr[1::4]) == 127).sum() > 0 and (qr[3::4] == 0).all()  # clamping and zero rows really occurred
+
+
 # ----------------------------------------------------------------------------- GEMM
 GEMM_SHAPES = [(1, 256, 64), (300, 768, 512), (129, 288, 1024), (1000, 1536, 3072), (6528, 512, 128)]
 

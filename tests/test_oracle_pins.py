@@ -652,3 +652,17 @@ def test_denoise_cond_rows_refilled_each_evaluation():
     assert nf == 4 and np.allclose(got, x, rtol=1e-14)
     with pytest.raises(ValueError):
         oracle.denoise_cond(x0, [0, 0], dm, 4, reuse=2, core_first=0, core_last=0, block_fn=fc)
+
+
+def test_quantize_known_max_clamps_beyond_the_given_max():
+    """Known-max int8 rule by hand: with row max 2, s = 2/127; 0.5/s = 31.75
+    rounds to 32, 2/s = 127, 3/s = 190.5 and -8/s = -508 clamp to +-127; a zero
+    max gives s = 0 and zero codes; with the row's own max it is quantize_rows."""
+    q, s = oracle.quantize_rows_known_max(np.array([[0.5, 2.0, 3.0, -8.0], [1.0, -1.0, 0.5, 0.25]]),
+                                          np.array([2.0, 0.0]))
+    assert s[0] == np.float32(np.float32(2.0) / np.float32(127.0)) and s[1] == 0
+    assert q.tolist() == [[32, 127, 127, -127], [0, 0, 0, 0]]
+    a = np.random.default_rng(3).normal(size=(5, 64)).astype(np.float32)
+    q1, s1 = oracle.quantize_rows(a)
+    q2, s2 = oracle.quantize_rows_known_max(a, np.abs(a).max(axis=1))
+    assert np.array_equal(q1, q2) and np.array_equal(s1, s2)
