@@ -405,22 +405,37 @@ __global__ void __launch_bounds__(THREADS, 1)
         base[256 * D + 256 + prow] = l;
       } else if (__all_sync(0xffffffffu, ok)) {
         tc_fence_after();
-        const int grow = q0 + t * BQ + row;
         const float inv = 1.f / l;
+        // Every MMA of the CTA has completed here (o_final follows the last S
+        // MMA of both tiles), so the Q tiles are idle: each softmax warp stages
+        // its 32 rows x D of bf16 output there (16-byte units XOR-swizzled by
+        // row: conflict-free both ways) and then writes whole row segments,
+        // 256/D rows per warp store instead of one 16-byte piece of 32 rows.
+        constexpr int UNITS = D / 8;  // 16-byte units per output row
+        uint8_t* stg = sQ + warp * (32 * D * 2);
 #pragma unroll 1
         for (int cc = 0; cc < D / 32; ++cc) {
           uint32_t o[32];
           tmem_ld32(oc + cc * 32, o);
           tmem_ld_wait();
-          if (grow < S) {
-            uint32_t w[16];
+          uint32_t w[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-              w[i] = cvt_bf16x2(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
-            uint4* dst = reinterpret_cast<uint4*>(a.out + static_cast<size_t>(grow) * d_model + h * D + cc * 32);
+          for (int i = 0; i < 16; ++i)
+            w[i] = cvt_bf16x2(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
-          }
+          for (int i = 0; i < 4; ++i)
+            *reinterpret_cast<uint4*>(stg + lane * (D * 2) + (((cc * 4 + i) ^ (lane % UNITS)) << 4)) =
+                make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+        }
+        __syncwarp();
+        constexpr int RPI = 32 / UNITS;  // rows per warp store
+        const int rbase = q0 + t * BQ + q * 32, u = lane % UNITS;
+#pragma unroll
+        for (int k = 0; k < 32 / RPI; ++k) {
+          const int r = k * RPI + lane / UNITS;
+          if (rbase + r < S)
+            *reinterpret_cast<uint4*>(a.out + static_cast<size_t>(rbase + r) * d_model + h * D + u * 8) =
+                *reinterpret_cast<const uint4*>(stg + r * (D * 2) + ((u ^ (r % UNITS)) << 4));
         }
       }
     }
