@@ -100,13 +100,18 @@ PINS = {
     "token_unmerge_delta": "explicit (f, r, c) loops; equals plain unmerge when x_pre is pair-constant; "
                            "identity when the merged blocks change nothing",
     "denoise_core": "core_reuse = 1 equals the plain loop; a core that adds a constant gives the closed form; "
-                    "hand-computed 3-step case",
+                    "hand-computed 3-step case; hand-computed loops with the reduction window strictly inside "
+                    "the core window and after it (window re-based onto its segment), plain and delta unmerge",
+    "stack_forward_ex": "hand-computed tokens with a toy block whose merged and unmerged forms differ: where the "
+                        "pre-merge tokens are taken, which merged input the delta subtracts, the window's blocks",
+    "linear": "pure-Python dot products",
     "block_forward_cond": "identity modulation without condition rows equals block_forward; zero gates give the "
                           "identity; scale = -1 makes every normed row equal to the shift (closed form without "
                           "RoPE); condition rows are permutation-equivariant among themselves (no rotation); a "
                           "class-1 zero gate leaves condition rows unchanged",
     "denoise_cond": "no condition rows and no modulation equals denoise / denoise_core; a toy block gives the "
-                    "closed form that needs the condition rows refilled every evaluation",
+                    "closed form that needs the condition rows refilled every evaluation; hand-computed loops with "
+                    "the reduction window inside / after the core window and under velocity reuse",
 }
 
 

@@ -666,3 +666,197 @@ def test_quantize_known_max_clamps_beyond_the_given_max():
     q1, s1 = oracle.quantize_rows(a)
     q2, s2 = oracle.quantize_rows_known_max(a, np.abs(a).max(axis=1))
     assert np.array_equal(q1, q2) and np.array_equal(s1, s2)
+
+
+# ----------------------------------------------------------------------------- wiring of the reduction window
+# Toy block: every row is scaled by its block's weight, and a block that runs
+# on the merged (reduced) grid also adds C.  Merged and unmerged blocks differ,
+# so the expected tokens below -- derived by hand for one 1x1x2 video grid
+# (one horizontal pair v0, v1) plus one audio row -- change if the window moves
+# by one block, if the merge or unmerge happens at the wrong place, or if the
+# delta unmerge takes the wrong pre-merge or merged tokens.
+_C = 0.3
+
+
+def _toy(x, w, d, merged):
+    return x * w + (_C if merged else 0.0)
+
+
+def _toy_cond(x, w, d, mod, n_cond, merged):
+    return _toy(x, w, d, merged)
+
+
+def test_stack_delta_unmerge_wiring_hand_computed():
+    """stack_forward_ex(unmerge_delta=True) on blocks a0 (full grid), a1, a2
+    (merged, window 1..2), a3 (full grid).  By hand, with y = a0*x the tokens
+    that enter the window, m = (y0 + y1)/2 the merged pair and
+    Y = a2*(a1*m + C) + C its output, each video token leaves the window as
+    y_c + (Y - m); the audio row leaves as a2*(a1*y_a + C) + C; block 3 scales
+    everything by a3.  The plain broadcast gives a3*Y on both video tokens."""
+    dm = dims_of(1, 1, 2, 1, 8, 1, 8)
+    a = [1.7, 0.6, 1.3, 0.8]
+    x = np.array([[0.9, -1.1], [-0.4, 2.0], [1.5, 0.25]])  # v0, v1, audio; two channels
+    seen = []
+
+    def fn(xx, w, d, merged):
+        seen.append((w, len(xx), merged))
+        return _toy(xx, w, d, merged)
+
+    got = oracle.stack_forward_ex(x, a, dm, 1, 2, unmerge_delta=True, block_fn=fn)
+    assert seen == [(a[0], 3, False), (a[1], 2, True), (a[2], 2, True), (a[3], 3, False)]
+    y = a[0] * x
+    m = (y[0] + y[1]) / 2.0
+    Y = a[2] * (a[1] * m + _C) + _C
+    Ya = a[2] * (a[1] * y[2] + _C) + _C
+    want = a[3] * np.stack([y[0] + (Y - m), y[1] + (Y - m), Ya])
+    assert np.allclose(got, want, rtol=1e-15, atol=1e-15)
+    # plain broadcast, same window
+    got_b = oracle.stack_forward_ex(x, a, dm, 1, 2, unmerge_delta=False, block_fn=_toy)
+    assert np.allclose(got_b, a[3] * np.stack([Y, Y, Ya]), rtol=1e-15, atol=1e-15)
+    # the two unmerges differ on these tokens (v0 != v1), so the test tells them apart
+    assert not np.allclose(got, got_b)
+
+
+def _eval_window_in_core(x, a, delta=None):
+    """One evaluation of the 5-block toy stack with core blocks 1..3 and the
+    reduction window 2..3 (inside the core), by hand.  Returns (velocity,
+    core update).  With delta given, the core is skipped and delta re-added."""
+    p = a[0] * x                                   # block 0, full grid
+    if delta is None:
+        q = a[1] * p                               # block 1, full grid (core)
+        m = (q[0] + q[1]) / 2.0                    # merge before block 2
+        Yv = a[3] * (a[2] * m + _C) + _C           # blocks 2, 3 on the merged grid
+        Ya = a[3] * (a[2] * q[2] + _C) + _C
+        core = np.stack([Yv, Yv, Ya])              # plain broadcast after block 3
+        delta = core - p
+    else:
+        core = p + delta
+    return a[4] * core, delta                      # block 4, full grid
+
+
+def _eval_window_after_core(x, a, delta=None):
+    """Same toy stack with core block 1 only and the reduction window 3..4
+    (after the core, in the last segment)."""
+    p = a[0] * x
+    if delta is None:
+        core = a[1] * p
+        delta = core - p
+    else:
+        core = p + delta
+    r = a[2] * core                                # block 2, full grid
+    m = (r[0] + r[1]) / 2.0
+    Yv = a[4] * (a[3] * m + _C) + _C
+    Ya = a[4] * (a[3] * r[2] + _C) + _C
+    return np.stack([Yv, Yv, Ya]), delta
+
+
+@pytest.mark.parametrize("case", ["inside_core", "after_core"])
+def test_denoise_core_reduction_window_rebased_hand_computed(case):
+    """denoise_core with the reduction window strictly inside the core window
+    (core 1..3, merge 2..3) or after it (core 1..1, merge 3..4): 3 steps, core
+    reuse 2 -> the core runs at steps 0 and 2, step 1 re-adds the cached
+    update.  The window is re-based onto the segment it lies in; an off-by-one
+    there moves the merge and changes every step below."""
+    dm = dims_of(1, 1, 2, 1, 8, 1, 8)
+    a = [0.8, 1.25, 0.7, 1.4, 0.9]
+    x0 = np.array([[1.0, -0.5], [0.2, 0.7], [-1.3, 0.4]])
+    cf, cl, mf, ml, ev = ((1, 3, 2, 3, _eval_window_in_core) if case == "inside_core"
+                          else (1, 1, 3, 4, _eval_window_after_core))
+    got, n_core = oracle.denoise_core(x0, a, dm, 3, 2, cf, cl, merge_first=mf, merge_last=ml, block_fn=_toy)
+    s = oracle.sigmas(3).astype(np.float64)
+    v0, d0 = ev(x0, a)
+    x1 = x0 + (s[1] - s[0]) * v0
+    v1, _ = ev(x1, a, delta=d0)
+    x2 = x1 + (s[2] - s[1]) * v1
+    v2, _ = ev(x2, a)
+    x3 = x2 + (s[3] - s[2]) * v2
+    assert n_core == 2
+    assert np.allclose(got, x3, rtol=1e-14, atol=1e-14)
+
+
+@pytest.mark.parametrize("case", ["inside_core", "after_core"])
+def test_denoise_cond_reduction_window_rebased_hand_computed(case):
+    """The same hand-computed loops through denoise_cond, with one condition
+    row appended (the toy block treats it like the audio row; it is refilled
+    every evaluation and left out of the Euler update), and the velocity-reuse
+    branch of denoise_cond with the window at 2..3 on the whole stack."""
+    dm = dims_of(1, 1, 2, 1, 8, 1, 8)
+    a = [0.8, 1.25, 0.7, 1.4, 0.9]
+    x0 = np.array([[1.0, -0.5], [0.2, 0.7], [-1.3, 0.4]])
+    cond = np.array([[0.6, -0.9]])
+    cf, cl, mf, ml, ev = ((1, 3, 2, 3, _eval_window_in_core) if case == "inside_core"
+                          else (1, 1, 3, 4, _eval_window_after_core))
+    got, n_fresh, n_core = oracle.denoise_cond(x0, a, dm, 3, cond_rows=cond, merge_first=mf, merge_last=ml,
+                                               core_reuse=2, core_first=cf, core_last=cl, block_fn=_toy_cond)
+    s = oracle.sigmas(3).astype(np.float64)
+    # the toy block acts row by row, so the condition row leaves the generated rows' velocity unchanged
+    v0, d0 = ev(x0, a)
+    x1 = x0 + (s[1] - s[0]) * v0
+    v1, _ = ev(x1, a, delta=d0)
+    x2 = x1 + (s[2] - s[1]) * v1
+    v2, _ = ev(x2, a)
+    x3 = x2 + (s[3] - s[2]) * v2
+    assert (n_fresh, n_core) == (3, 2)
+    assert np.allclose(got, x3, rtol=1e-14, atol=1e-14)
+
+    # velocity reuse 2 (no core window), reduction window 2..3 of the 5 blocks:
+    # fresh at steps 0 and 2, velocity reused at step 1
+    def ev_full(x):
+        p = a[1] * (a[0] * x)
+        m = (p[0] + p[1]) / 2.0
+        Yv = a[3] * (a[2] * m + _C) + _C
+        Ya = a[3] * (a[2] * p[2] + _C) + _C
+        return a[4] * np.stack([Yv, Yv, Ya])
+
+    got, n_fresh, _ = oracle.denoise_cond(x0, a, dm, 3, cond_rows=cond, reuse=2, merge_first=2, merge_last=3,
+                                          block_fn=_toy_cond)
+    v0 = ev_full(x0)
+    x1 = x0 + (s[1] - s[0]) * v0
+    x2 = x1 + (s[2] - s[1]) * v0
+    x3 = x2 + (s[3] - s[2]) * ev_full(x2)
+    assert n_fresh == 2 and np.allclose(got, x3, rtol=1e-14, atol=1e-14)
+
+
+def test_denoise_core_delta_unmerge_inside_core_hand_computed():
+    """denoise_core with the delta unmerge and the window inside the core
+    (core 1..3, merge 2..3): the core's output video tokens are
+    q_c + (Y - m) with q = a1*a0*x the tokens entering the window."""
+    dm = dims_of(1, 1, 2, 1, 8, 1, 8)
+    a = [0.8, 1.25, 0.7, 1.4, 0.9]
+    x0 = np.array([[1.0, -0.5], [0.2, 0.7], [-1.3, 0.4]])
+
+    def ev(x, delta=None):
+        p = a[0] * x
+        if delta is None:
+            q = a[1] * p
+            m = (q[0] + q[1]) / 2.0
+            Yv = a[3] * (a[2] * m + _C) + _C
+            Ya = a[3] * (a[2] * q[2] + _C) + _C
+            core = np.stack([q[0] + Yv - m, q[1] + Yv - m, Ya])
+            delta = core - p
+        else:
+            core = p + delta
+        return a[4] * core, delta
+
+    got, n_core = oracle.denoise_core(x0, a, dm, 3, 2, 1, 3, merge_first=2, merge_last=3, unmerge_delta=True,
+                                      block_fn=_toy)
+    s = oracle.sigmas(3).astype(np.float64)
+    v0, d0 = ev(x0)
+    x1 = x0 + (s[1] - s[0]) * v0
+    v1, _ = ev(x1, d0)
+    x2 = x1 + (s[2] - s[1]) * v1
+    v2, _ = ev(x2)
+    x3 = x2 + (s[3] - s[2]) * v2
+    assert n_core == 2 and np.allclose(got, x3, rtol=1e-14, atol=1e-14)
+
+
+def test_linear_vs_python_dot_products():
+    """y[m, n] = sum_k a[m, k] W[n, k] for W stored [out, in], by explicit sums."""
+    rng = random.Random(5)
+    a = [[rng.uniform(-2, 2) for _ in range(7)] for _ in range(3)]
+    w = [[rng.uniform(-2, 2) for _ in range(7)] for _ in range(4)]
+    y = oracle.linear(np.array(a), np.array(w))
+    assert y.shape == (3, 4)
+    for m in range(3):
+        for n in range(4):
+            assert abs(y[m, n] - math.fsum(a[m][k] * w[n][k] for k in range(7))) < 1e-13
