@@ -6,6 +6,7 @@
 #include <math.h>
 #include <string.h>
 
+#include <atomic>
 #include <mutex>
 #include <vector>
 
@@ -20,8 +21,11 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 
+// Per-device state, filled once under the mutex.  `ready` is published with
+// release order after num_sms and err are written, and read with acquire
+// order on the fast path, so a thread that sees ready == true also sees them.
 struct DeviceInfo {
-  bool ready = false;
+  std::atomic<bool> ready{false};
   int num_sms = 0;
   int* err = nullptr;
 };
@@ -33,9 +37,9 @@ int device_ctx(cudaStream_t stream, Ctx* c) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return H3B_ERR_DEVICE;
   DeviceInfo& di = g_dev[dev];
-  if (!di.ready) {
+  if (!di.ready.load(std::memory_order_acquire)) {
     std::lock_guard<std::mutex> lk(g_mu);
-    if (!di.ready) {
+    if (!di.ready.load(std::memory_order_relaxed)) {
       int major = 0, sms = 0;
       if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return H3B_ERR_DEVICE;
       if (major != 10) return H3B_ERR_DEVICE;
@@ -44,7 +48,7 @@ int device_ctx(cudaStream_t stream, Ctx* c) {
       if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return H3B_ERR_CUDA;
       di.num_sms = sms;
       di.err = static_cast<int*>(p);
-      di.ready = true;
+      di.ready.store(true, std::memory_order_release);
     }
   }
   c->stream = stream;

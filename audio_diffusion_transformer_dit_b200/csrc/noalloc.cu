@@ -11,6 +11,9 @@
 // In host code the array's name only stands in for it; its device address is
 // looked up once per device with cudaGetSymbolAddress (with that device
 // current) on the first call, and that address is what the kernels receive.
+// The address is cached for the life of the process: after cudaDeviceReset on
+// a device the cached address (like the library's other per-device state) is
+// stale, so the library must not be called on that device again.
 #include <mutex>
 
 #include "h3b.h"

@@ -2,14 +2,19 @@
 """Benchmark of the DiT block hot path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+    python bench.py --measure-int8-peak      # writes profiles/int8_peak.json
+    python bench.py --kernel-sweep           # memory-bound kernels alone, GB/s
 
 One step = one pass of the hot path over one batch of synthetic input.  The
-default workload is the single bf16 DiT block d=3072 (24 heads x 128, MLP
-12288) over 6x32x32 video + 256 audio tokens (S = 6400): one step is one
-h3b_block_forward (RoPE table, RMSNorm, QKV GEMM + RoPE, flash attention,
-O-proj + residual, RMSNorm, FC1 + GELU, FC2 + residual).  Other workloads:
-the 8-block d=5120 stack, the INT8 W8A8 d=5120 block over 20640 tokens and the
-45-block 20-step denoising loop with reuse 2 and token reduction.
+default workload is the 8-block bf16 stack at the 33B-class width: d = 5120
+(40 heads x 128, MLP 20480, fp32 residual stream) over 6x32x32 video + 384
+audio tokens (S = 6528); one step is one h3b_stack_forward (RoPE table, then
+per block RMSNorm, QKV GEMM + RoPE, flash attention, O-proj + residual,
+RMSNorm, FC1 + GELU, FC2 + residual).  The same run also times the INT8 W8A8
+d = 5120 block over 5x48x84 video + 480 audio tokens (S = 20640) with the same
+protocol and reports it as the "int8" sub-record.  Other workloads: the
+single d = 3072 block, the 45-block 20-step denoising loop with reuse 2 and
+token reduction, the preview loop.
 
 Timing: W untimed warm-up steps, then K steps bracketed by a barrier and
 torch.cuda.synchronize() on both sides, CUDA events on the launching stream,
@@ -20,14 +25,17 @@ exchange step, so there is no data-path collective ("scaling": "weak").
 A second pass of the same K steps records library-owned CUDA events around
 every launch for the per-kernel shares and the roofline of the dominant
 kernel ("ms_per_step_traced"; the events between launches forgo the overlap
-of neighbouring kernels, so `value` comes from the untraced pass).
+of neighbouring kernels, so `value` comes from the untraced pass).  Tensor
+peaks follow the SM clock sampled during the timed region (tensor_peak);
+fractions against the datasheet peaks are printed beside them.
 
---impl reference times the CPU oracle (numpy fp64) on the host cores on a
-bounded sample of the same workload (rank 0 only under torchrun).
+--impl reference times the CPU oracle (numpy fp64) on the host cores, one
+1/8-block token chunk per step (rank 0 only under torchrun).
 """
 from __future__ import annotations
 
 import argparse
+import ctypes
 import datetime
 import hashlib
 import json
@@ -45,13 +53,17 @@ import torch  # noqa: E402
 
 import workloads as W  # noqa: E402
 
-DEFAULT_WORKLOAD = "block_d3072_s6400"
+DEFAULT_WORKLOAD = "stack8_d5120_s6528"
+INT8_WORKLOAD = "block_int8_d5120_s20640"
 METRIC = "DiT block tokens/s"
 # default timed steps per workload: about 1-30 s of device time each
 DEFAULT_STEPS = {"block_d256_s288": 2000, "block_d3072_s6400": 300, "stack8_d5120_s6528": 30,
                  "block_int8_d5120_s20640": 60, "loop45_d5120_s6528": 2,
                  "preview40_d5120_s2784": 4}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# B200 datasheet dense peaks (bf16, int8) and the HBM figure the block is held to
+NOMINAL = {"bf16_tflops": 2250.0, "int8_tops": 4500.0, "hbm_gbs": 8000.0}
+INT8_PEAK_FILE = os.path.join(ROOT, "profiles", "int8_peak.json")
 
 
 # ----------------------------------------------------------------------------- helpers
@@ -61,6 +73,42 @@ def peaks():
         d = json.load(open(p))
         return d, "measured"
     return dict(FALLBACK_PEAKS), "fallback"
+
+
+def tensor_peak(pk, clocks, int8=False):
+    """Dense tensor peak for a kernel timed at the sampled SM clock.
+
+    Two measured points bound it: the burst figure (best single GEMM, high
+    clock) and the sustained figure (a seconds-long GEMM loop under the power
+    cap, at the median clock recorded with it).  The peak is the sustained
+    figure scaled by (median SM clock of this run / that clock), clamped to
+    [sustained, burst]: a run at full clock gets the burst peak, one at the
+    power-capped clock the sustained peak.  INT8 uses its own measured pair
+    when profiles/int8_peak.json exists, else the bf16 pair x 2 (the nominal
+    4.5 / 2.25 ratio)."""
+    src = "MEASURED_PEAKS.json (cuBLAS bf16)"
+    burst, sust = pk.get("bf16_tflops"), pk.get("bf16_tflops_sustained", pk.get("bf16_tflops"))
+    f_s = (pk.get("clocks_under_load") or {}).get("sm_mhz_median")
+    scale, nominal = 1.0, NOMINAL["bf16_tflops"]
+    if int8:
+        nominal = NOMINAL["int8_tops"]
+        if os.path.exists(INT8_PEAK_FILE):
+            q = json.load(open(INT8_PEAK_FILE))
+            burst, sust, f_s = q["int8_tops"], q["int8_tops_sustained"], q.get("sustained_sm_mhz_median")
+            src = "profiles/int8_peak.json (torch._int_mm int8)"
+        else:
+            scale = 2.0
+            src += " x 2 (nominal int8/bf16 ratio)"
+    burst, sust = burst * scale, sust * scale
+    med = (clocks or {}).get("sm_mhz")
+    if med and f_s:
+        peak = min(burst, max(sust, sust * med / f_s))
+        basis = (f"{src}: sustained {sust:.0f} x median {med:.0f} MHz / {f_s:.0f} MHz, clamped to "
+                 f"[sustained {sust:.0f}, burst {burst:.0f}]")
+    else:
+        peak = sust
+        basis = f"{src}: sustained {sust:.0f} (no clock samples)"
+    return {"peak": round(peak, 1), "basis": basis, "nominal": nominal}
 
 
 def max_over_ranks(ms: float, device) -> float:
@@ -210,14 +258,18 @@ def build_workload(wl, dev):
     return dm, blocks, x, ws
 
 
-def run_ours(args, wl):
-    from audio_diffusion_transformer_dit_b200 import h3b
-    rank, world, local = dist_env()
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
+def _barrier(world):
     if world > 1:
         import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+        dist.barrier()
+
+
+def measure(args, wl, dev, world, local):
+    """Time K steps of one workload (after W warm-ups) and return its record:
+    rate, per-kernel shares from a traced second pass, the dominant kernel's
+    roofline, the whole-step roofline and the end-to-end rate through the
+    public API with host buffers."""
+    from audio_diffusion_transformer_dit_b200 import h3b
     dm, blocks, x, ws = build_workload(wl, dev)
     loop = wl.steps > 0
     v = torch.empty_like(x) if loop else None
@@ -259,11 +311,6 @@ def run_ours(args, wl):
             h3b.block_forward(dm, blocks[0], x, ws)
         units = float(wl.seq)
 
-    def barrier():
-        if world > 1:
-            import torch.distributed as dist
-            dist.barrier()
-
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -272,7 +319,7 @@ def run_ours(args, wl):
     sampler = ClockSampler(local)
     stream = torch.cuda.current_stream()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier()
+    _barrier(world)
     torch.cuda.synchronize()
     sampler.start()
     e0.record(stream)
@@ -280,14 +327,14 @@ def run_ours(args, wl):
         step()
     e1.record(stream)
     torch.cuda.synchronize()
-    barrier()
+    _barrier(world)
     ms = max_over_ranks(e0.elapsed_time(e1), dev)
     # Per-kernel durations: the same K steps again with library-owned CUDA
     # events around every launch.  Events between launches forgo the
     # programmatic-launch overlap of neighbouring kernels, so this pass only
     # feeds the per-kernel shares and the roofline; `value` is the pass above.
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier()
+    _barrier(world)
     torch.cuda.synchronize()
     with h3b.Trace(capacity=args.steps * (4000 if loop else 16 * len(blocks) + 8)) as tr:
         t0.record(stream)
@@ -295,7 +342,7 @@ def run_ours(args, wl):
             step()
         t1.record(stream)
         torch.cuda.synchronize()
-    barrier()
+    _barrier(world)
     clocks = sampler.stop()
     ms_traced = max_over_ranks(t0.elapsed_time(t1), dev)
     assert h3b.device_error() == 0, "device error word set during the timed region"
@@ -307,6 +354,8 @@ def run_ours(args, wl):
                sorted(per.items(), key=lambda kv: -kv[1][1])}
     my_launches = sum(c for k, (c, _) in per.items() if k != "memset")
     pk, src = peaks()
+    bf16_pk = tensor_peak(pk, clocks, int8=False)
+    int8_pk = tensor_peak(pk, clocks, int8=True)
     dom = max(per.items(), key=lambda kv: kv[1][1])[0]
     amount, unit, bound = kernel_work(dom, wl, wl.dtype)
     if loop and wl.merge_first >= 0 and bound == "tensor":
@@ -317,17 +366,16 @@ def run_ours(args, wl):
     if amount is not None:
         avg_s = per[dom][1] / per[dom][0] / 1e3
         if bound == "tensor":
-            peak = pk.get("bf16_tflops_sustained", pk.get("bf16_tflops"))
-            if unit == "TOP/s":
-                peak = peak * 2.0  # int8 dense peak = bf16 measured x nominal ratio 4.5/2.25
+            tp = int8_pk if unit == "TOP/s" else bf16_pk
+            peak, basis, nominal = tp["peak"], tp["basis"], tp["nominal"]
             achieved = amount / avg_s / 1e12
         else:
-            peak = pk.get("hbm_gbs")
+            peak, basis, nominal = pk.get("hbm_gbs"), f"{src} copy bandwidth", NOMINAL["hbm_gbs"]
             achieved = amount / avg_s / 1e9
-        roof = {"kernel": dom, "bound": bound, "achieved": round(achieved, 2), "peak": peak, "unit": unit,
+        roof = {"kernel": dom, "bound": bound, "achieved": round(achieved, 2), "peak": round(peak, 1), "unit": unit,
                 "frac": round(achieved / peak, 4), "traffic": measured_traffic(dom, wl.name),
-                "peak_source": f"{src} ({'sustained bf16' if bound == 'tensor' else 'copy'})",
-                "work_per_launch": amount}
+                "peak_basis": basis, "frac_nominal": round(achieved / nominal, 4), "nominal_peak": nominal,
+                "work_per_launch": amount, "avg_launch_ms": round(avg_s * 1e3, 4)}
 
     value = whole_job_value(units, args.steps, world, ms)
     if loop:
@@ -348,32 +396,40 @@ def run_ours(args, wl):
             flops_step = per_eval * n_fresh
 
     # Whole-step roofline: every launch's algorithmic work at its own bound's
-    # measured peak, summed over the step, against the untraced step time.
-    tensor_peak = pk.get("bf16_tflops_sustained", pk.get("bf16_tflops"))
+    # peak (tensor peaks chosen for the sampled clock), summed over the step,
+    # against the untraced step time.
     if not loop:
-        t_ideal = 0.0
+        t_ideal = t_nominal = 0.0
         for k, (c, _) in per.items():
             a, u, b = kernel_work(k, wl, wl.dtype)
             if a is None:
                 continue
             if b == "tensor":
-                t_ideal += c * a / (tensor_peak * (2.0 if u == "TOP/s" else 1.0) * 1e12)
+                i8 = u == "TOP/s"
+                t_ideal += c * a / ((int8_pk if i8 else bf16_pk)["peak"] * 1e12)
+                t_nominal += c * a / ((NOMINAL["int8_tops"] if i8 else NOMINAL["bf16_tflops"]) * 1e12)
             else:
                 t_ideal += c * a / (pk.get("hbm_gbs") * 1e9)
+                t_nominal += c * a / (NOMINAL["hbm_gbs"] * 1e9)
         t_ideal /= args.steps
-        basis = "every traced launch: GEMM/attention work at the sustained bf16 peak (int8 x2), memory kernels at HBM"
+        t_nominal /= args.steps
+        basis = ("every traced launch: GEMM/attention work at the clock-chosen tensor peak "
+                 f"(bf16 {bf16_pk['peak']:.0f} TF/s, int8 {int8_pk['peak']:.0f} TOP/s), memory kernels at the "
+                 f"{src} copy bandwidth")
     else:
-        t_ideal = flops_step / (tensor_peak * 1e12)
-        basis = "GEMM + attention work of the step at the sustained bf16 peak (memory-bound kernels < 2 %)"
+        t_ideal = flops_step / (bf16_pk["peak"] * 1e12)
+        t_nominal = flops_step / (NOMINAL["bf16_tflops"] * 1e12)
+        basis = (f"GEMM + attention work of the step at the clock-chosen bf16 peak ({bf16_pk['peak']:.0f} TF/s; "
+                 "memory-bound kernels < 2 %)")
     t_step = ms / 1e3 / args.steps
     step_roofline = {"t_ideal_ms": round(t_ideal * 1e3, 4), "t_ms": round(t_step * 1e3, 4),
-                     "frac": round(t_ideal / t_step, 4), "basis": basis}
+                     "frac": round(t_ideal / t_step, 4), "frac_nominal": round(t_nominal / t_step, 4),
+                     "basis": basis}
 
     # end-to-end through the public API with the tokens in pinned host memory:
     # every step copies its input in and its result out inside the timed
     # region; HostPipeline overlaps those copies with the neighbouring steps'
     # compute on separate streams.
-    e2e = None
     if not loop:
         k2 = max(4, min(args.steps, 50))
         xin = [x.detach().cpu().pin_memory() for _ in range(2)]
@@ -383,7 +439,7 @@ def run_ours(args, wl):
             pipe.submit(xin[i % 2], xout[i % 2])
         pipe.synchronize()
         torch.cuda.synchronize()
-        barrier()
+        _barrier(world)
         torch.cuda.synchronize()
         f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         f0.record(pipe.s_in)
@@ -392,12 +448,13 @@ def run_ours(args, wl):
         f1.record(pipe.s_out)
         pipe.synchronize()
         torch.cuda.synchronize()
-        barrier()
+        _barrier(world)
         ms2 = max_over_ranks(f0.elapsed_time(f1), dev)
         nb = x.numel() * 4
         e2e = {"value": round(whole_job_value(units, k2, world, ms2), 2), "unit": unit_v, "h2d_bytes_per_step": nb,
                "d2h_bytes_per_step": nb, "steps": k2,
                "api": "h3b.HostPipeline.submit (pinned host in/out, copies overlapped with compute)"}
+        del pipe
     else:
         # one step = one whole denoising loop: x0 comes in from pinned host
         # memory and x_N goes back to it inside the timed region
@@ -405,7 +462,7 @@ def run_ours(args, wl):
         xh = x.detach().cpu().pin_memory()
         xo = torch.empty_like(xh).pin_memory()
         torch.cuda.synchronize()
-        barrier()
+        _barrier(world)
         torch.cuda.synchronize()
         f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         f0.record(stream)
@@ -415,14 +472,14 @@ def run_ours(args, wl):
             xo.copy_(x, non_blocking=True)
         f1.record(stream)
         torch.cuda.synchronize()
-        barrier()
+        _barrier(world)
         ms2 = max_over_ranks(f0.elapsed_time(f1), dev)
         nb = x.numel() * 4
         e2e = {"value": round(ms2 / 1e3 / k2 / wl.steps, 6), "unit": unit_v, "h2d_bytes_per_step": nb,
                "d2h_bytes_per_step": nb, "steps": k2,
                "api": "h3b.denoise / h3b.denoise_ex with x0 copied in from and x_N copied out to pinned host memory"}
 
-    line = {
+    rec = {
         "metric": metric, "value": round(value, 6 if loop else 2), "unit": unit_v, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 4),
         "ms_per_step_traced": round(ms_traced / args.steps, 4),
@@ -436,23 +493,41 @@ def run_ours(args, wl):
                    "l2": "no flush: per-step working set (weights + activations + workspace) > 126 MB L2"},
         "tflops": round(flops_step * args.steps * world / (ms / 1e3) / 1e12, 2),
         "roofline": roof, "step_roofline": step_roofline, "gpu_launches": my_launches, "clocks": clocks,
-        "kernels": kernels,
+        "tensor_peaks": {"bf16": bf16_pk, "int8": int8_pk}, "kernels": kernels, "e2e": e2e,
     }
     if loop:
-        line["s_per_fresh_eval"] = round(ms / 1e3 / args.steps / n_fresh, 6)
-        line["config"].update({"steps": wl.steps, "reuse": 1 if core else wl.reuse, "fresh_evals": n_fresh,
-                               "token_reduction": [wl.merge_first, wl.merge_last],
-                               "unmerge": "delta" if args.unmerge_delta else "broadcast"})
+        rec["s_per_fresh_eval"] = round(ms / 1e3 / args.steps / n_fresh, 6)
+        rec["config"].update({"steps": wl.steps, "reuse": 1 if core else wl.reuse, "fresh_evals": n_fresh,
+                              "token_reduction": [wl.merge_first, wl.merge_last],
+                              "unmerge": "delta" if args.unmerge_delta else "broadcast"})
         if core:
-            line["config"].update({"core_reuse": args.core_reuse, "core_blocks": [wl.merge_first, wl.merge_last],
-                                   "core_evals": n_core})
+            rec["config"].update({"core_reuse": args.core_reuse, "core_blocks": [wl.merge_first, wl.merge_last],
+                                  "core_evals": n_core})
         if args.cond_rows or args.modulation:
-            line["config"].update({"cond_rows": args.cond_rows, "modulation": "per step" if args.modulation else None})
-        line["ms_per_loop"] = round(ms / args.steps, 3)
-    if e2e:
-        line["e2e"] = e2e
+            rec["config"].update({"cond_rows": args.cond_rows, "modulation": "per step" if args.modulation else None})
+        rec["ms_per_loop"] = round(ms / args.steps, 3)
+    del blocks, x, ws, v
+    torch.cuda.empty_cache()
+    return rec
+
+
+def run_ours(args, wl):
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    line = measure(args, wl, dev, world, local)
+    # The INT8 W8A8 block (d = 5120 over 5x48x84 video + 480 audio tokens) is
+    # timed in the same run with the same protocol, as a sub-record.
+    if args.workload == DEFAULT_WORKLOAD and not args.no_int8 and not (args.layers or args.denoise_steps):
+        sub = measure(args, W.WORKLOADS[INT8_WORKLOAD], dev, world, local)
+        line["int8"] = {k: sub[k] for k in ("metric", "value", "unit", "ms_per_step", "ms_per_step_traced",
+                                            "dtype", "config", "tflops", "roofline", "step_roofline",
+                                            "gpu_launches", "clocks", "tensor_peaks", "kernels", "e2e")}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(wl, budget_s=args.cpu_budget)
+        line["cpu_baseline"] = cpu_baseline(wl)
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
@@ -462,34 +537,56 @@ def run_ours(args, wl):
 
 
 # ----------------------------------------------------------------------------- CPU oracle
-def _oracle_inputs(wl, layer=0, merged=False):
+def _oracle_inputs(wl, layer=0):
     w = {k: v.float().numpy() for k, v in W.block_weights(wl, layer, "cpu").items()}
-    x = W.initial_tokens(wl, "cpu", seq=wl.seq_merged if merged else wl.seq).numpy()
+    x = W.initial_tokens(wl, "cpu").numpy()
     return w, x
 
 
-def oracle_block_rate(wl, rows_a=64, rows_b=256, reps=1):
-    """Oracle block-forward time model on this host: T(R) = a + b R for R query
-    rows (keys/values always cover all S tokens); returns (a, b, seconds used)."""
-    import oracle
-    w, x = _oracle_inputs(wl)
-    if wl.dtype == W.INT8:
-        w = oracle.dequant_weights(w)
-    t_used = 0.0
-    times = {}
-    for R in (rows_a, rows_b):
-        rows = np.linspace(0, wl.seq - 1, R).astype(int)
-        best = None
-        for _ in range(reps):
-            t0 = time.perf_counter()
-            oracle.block_forward(x, w, wl, rows=rows)
-            dt = time.perf_counter() - t0
-            t_used += dt
-            best = dt if best is None else min(best, dt)
-        times[R] = best
-    b = max((times[rows_b] - times[rows_a]) / (rows_b - rows_a), 0.0)
-    a = max(times[rows_a] - b * rows_a, 0.0)
-    return a, b, t_used
+class OracleChunks:
+    """The oracle block (fp64 numpy) run one token chunk at a time.
+
+    Chunk i of n takes its tokens through every part of the block -- RMSNorm,
+    the Q, K and V projections of those tokens, RoPE, attention of its
+    queries against all S keys and values, O-projection + residual, RMSNorm,
+    GELU MLP + residual -- and writes its K and V rows into a cache that holds
+    all S tokens' keys and values (filled once at set-up).  Each chunk is thus
+    1/n of the block's arithmetic, and n consecutive chunks are exactly one
+    block's work: the time of one chunk is the time behind (S/n) tokens of
+    block throughput.  Only the oracle's own functions are called."""
+
+    def __init__(self, wl, n_chunks=8):
+        import oracle
+        self.o = oracle
+        self.wl = wl
+        w, x = _oracle_inputs(wl)
+        if wl.dtype == W.INT8:
+            w = oracle.dequant_weights(w)  # the INT8 parity reference: dequantised weights
+        self.w = {k: np.asarray(v, dtype=np.float64) for k, v in w.items()}
+        self.x = np.asarray(x, dtype=np.float64)
+        self.ang = oracle.rope_angles(wl)
+        d = wl.d
+        u = oracle.rmsnorm(self.x, self.w["g_attn"], wl.eps)
+        self.k = oracle.apply_rope(oracle.linear(u, self.w["w_qkv"][d:2 * d]), self.ang, wl.n_heads)
+        self.v = oracle.linear(u, self.w["w_qkv"][2 * d:])
+        self.bounds = np.linspace(0, wl.seq, n_chunks + 1).astype(int)
+        self.n = n_chunks
+
+    def run(self, i):
+        o, wl, w, d = self.o, self.wl, self.w, self.wl.d
+        lo, hi = self.bounds[i % self.n], self.bounds[i % self.n + 1]
+        x = self.x[lo:hi]
+        u = o.rmsnorm(x, w["g_attn"], wl.eps)
+        qkv = o.linear(u, w["w_qkv"])
+        q = o.apply_rope(qkv[:, :d], self.ang[lo:hi], wl.n_heads)
+        self.k[lo:hi] = o.apply_rope(qkv[:, d:2 * d], self.ang[lo:hi], wl.n_heads)
+        self.v[lo:hi] = qkv[:, 2 * d:]
+        x1 = x + o.linear(o.attention(q, self.k, self.v, wl.n_heads), w["w_o"])
+        g = o.gelu(o.linear(o.rmsnorm(x1, w["g_mlp"], wl.eps), w["w_fc1"]))
+        return x1 + o.linear(g, w["w_fc2"])
+
+    def tokens(self, i):
+        return int(self.bounds[i % self.n + 1] - self.bounds[i % self.n])
 
 
 def cpu_model():
@@ -510,64 +607,264 @@ def cpu_threads():
         return os.cpu_count()
 
 
-def cpu_baseline(wl, budget_s=30.0):
-    a, b, used = oracle_block_rate(wl)
-    per_block = a + b * wl.seq
-    n_blocks = wl.n_blocks
+def cpu_baseline(wl, budget_s=20.0, n_chunks=8):
+    """Block tokens/s of the oracle on this host: whole 1/n-block chunks
+    (OracleChunks) until about budget_s seconds of CPU work, at least two."""
+    oc = OracleChunks(wl, n_chunks)
+    oc.run(0)  # warm-up (BLAS threads, page-in)
+    done = toks = 0
+    t0 = time.perf_counter()
+    while done < 2 or (time.perf_counter() - t0 < budget_s and done < n_chunks):
+        oc.run(done)
+        toks += oc.tokens(done)
+        done += 1
+    dt = time.perf_counter() - t0
+    sample = (f"{done} of the {n_chunks} token chunks of one {wl.name} block (layer 0; the stack's blocks share its "
+              f"shape), each chunk through the whole block in fp64 numpy with attention against all {wl.seq} keys: "
+              f"{toks} tokens in {dt:.1f} s")
     if wl.steps > 0:
+        per_block = dt / toks * wl.seq
         n_fresh = len([i for i in range(wl.steps) if i % wl.reuse == 0 or i == wl.steps - 1])
-        seconds = per_block * n_blocks * n_fresh / wl.steps
-        return {"value": round(seconds, 3), "unit": "s/step", "cores": cpu_threads(), "cpu_model": cpu_model(),
-                "kind": "oracle",
-                "sample": f"oracle block forward on this host with 64 and 256 query rows (all {wl.seq} keys); "
-                          f"full block {per_block:.2f} s extrapolated linearly in rows, x{n_blocks} blocks "
-                          f"x{n_fresh} fresh evals / {wl.steps} steps (merged blocks counted at full S); "
-                          f"{used:.1f} s of CPU time"}
-    value = wl.seq / per_block
-    return {"value": round(value, 3), "unit": "tokens/s", "cores": cpu_threads(), "cpu_model": cpu_model(),
-            "kind": "oracle",
-            "sample": f"oracle block forward (fp64 numpy) with 64 and 256 sampled query rows, keys/values over "
-                      f"all {wl.seq} tokens; full-block time {per_block:.2f} s = fixed + per-row cost x {wl.seq} "
-                      f"rows, fitted from the two runs ({used:.1f} s of CPU time)"}
+        return {"value": round(per_block * wl.n_blocks * n_fresh / wl.steps, 3), "unit": "s/step",
+                "cores": cpu_threads(), "cpu_model": cpu_model(), "kind": "oracle",
+                "sample": sample + f"; extrapolated to {wl.n_blocks} full-length blocks x {n_fresh} fresh "
+                                   f"evaluations / {wl.steps} steps (merged blocks counted at full length)"}
+    return {"value": round(toks / dt, 3), "unit": "tokens/s", "cores": cpu_threads(), "cpu_model": cpu_model(),
+            "kind": "oracle", "sample": sample}
 
 
 def run_reference(args, wl):
+    """The oracle as the reference arm: one step = one 1/8-block token chunk of
+    the workload (OracleChunks), so eight steps are one block's arithmetic and
+    `value` = chunk tokens / chunk time (block tokens/s, the same unit as our
+    arm's).  Set-up (weights, the K/V cache) is untimed."""
     rank, world, _ = dist_env()
     if rank != 0:
         return
-    import oracle
-    w, x = _oracle_inputs(wl)
-    if wl.dtype == W.INT8:
-        w = oracle.dequant_weights(w)
-    # the fixed (keys/values) + per-row cost model, fitted during warm-up
-    R = 64
-    rows = np.linspace(0, wl.seq - 1, R).astype(int)
-    a, b, _ = oracle_block_rate(wl)
-    for _ in range(args.warmup):
-        oracle.block_forward(x, w, wl, rows=rows)
-    t0 = time.perf_counter()
-    for _ in range(args.steps):
-        oracle.block_forward(x, w, wl, rows=rows)
-    dt = (time.perf_counter() - t0) / args.steps
-    per_block = dt + b * (wl.seq - R)
-    units = wl.seq * max(1, wl.n_blocks if wl.steps == 0 else 1)
-    blocks = wl.n_blocks
     if wl.steps > 0:
-        n_fresh = len([i for i in range(wl.steps) if i % wl.reuse == 0 or i == wl.steps - 1])
-        value, unit, hib, metric = per_block * blocks * n_fresh / wl.steps, "s/step", False, "s per denoise step"
-    else:
-        value, unit, hib, metric = units / (per_block * blocks), "tokens/s", True, METRIC
-    sample = (f"each step: oracle block forward (fp64 numpy), {R} sampled query rows against all {wl.seq} "
-              f"keys/values; full block = step time + {wl.seq - R} rows x fitted per-row cost {b * 1e3:.3f} ms")
-    line = {"impl": "reference", "metric": metric, "value": round(value, 4), "unit": unit, "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 2),
-            "higher_is_better": hib, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic (same seeded inputs)", "config": {"workload": wl.name, "seq_len": wl.seq,
-                                                                 "d": wl.d, "blocks": blocks},
-            "cpu_baseline": {"value": round(value, 4), "unit": unit, "cores": cpu_threads(),
+        print(json.dumps({"impl": "reference", "unavailable": "the loop workloads are reported through their "
+                                                              "extrapolated cpu_baseline only"}), flush=True)
+        return
+    oc = OracleChunks(wl, 8)
+    for i in range(args.warmup):
+        oc.run(i)
+    toks = 0
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        oc.run(i)
+        toks += oc.tokens(i)
+    dt = time.perf_counter() - t0
+    value = toks / dt
+    sample = (f"each step: one of the 8 token chunks of a {wl.name} block (about {wl.seq // 8} tokens) through the "
+              f"whole block in fp64 numpy, attention against all {wl.seq} keys; 8 steps = one block's arithmetic; "
+              f"{toks} tokens in {dt:.1f} s")
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 2),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (same seeded inputs)",
+            "config": {"workload": wl.name, "seq_len": wl.seq, "d": wl.d, "heads": wl.n_heads,
+                       "head_dim": wl.head_dim, "ffn": wl.ffn, "blocks": wl.n_blocks,
+                       "video_grid": [wl.frames, wl.rows, wl.cols], "audio_tokens": wl.n_audio,
+                       "global_batch": 1, "parallelism": "cpu"},
+            "cpu_baseline": {"value": round(value, 4), "unit": "tokens/s", "cores": cpu_threads(),
                              "cpu_model": cpu_model(), "kind": "oracle", "sample": sample},
-            "e2e": {"value": round(value, 4), "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+            "e2e": {"value": round(value, 4), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- peak and kernel probes
+def measure_int8_peak(out_path, n=8192, burst_reps=10, sustain_s=4.0):
+    """Dense int8 tensor peak of this GPU, the way the bf16 peaks are taken:
+    torch._int_mm (cuBLAS) on n^3, best of burst_reps single launches (CUDA
+    events), then back-to-back launches for sustain_s seconds with the SM
+    clock sampled; bf16 torch.matmul on the same box for the ratio."""
+    dev = torch.device("cuda", 0)
+    g = torch.Generator(device=dev)
+    g.manual_seed(7)
+    a = torch.randint(-127, 128, (n, n), generator=g, device=dev, dtype=torch.int8)
+    b = torch.randint(-127, 128, (n, n), generator=g, device=dev, dtype=torch.int8).t()  # column-major
+    ab = torch.randn((n, n), generator=g, device=dev).to(torch.bfloat16)
+    bb = torch.randn((n, n), generator=g, device=dev).to(torch.bfloat16)
+    ops = 2.0 * n ** 3
+
+    def burst(fn):
+        for _ in range(3):
+            fn()
+        best = None
+        for _ in range(burst_reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            t = e0.elapsed_time(e1) / 1e3
+            best = t if best is None else min(best, t)
+        return ops / best / 1e12
+
+    def sustained(fn):
+        sampler = ClockSampler(0)
+        fn()
+        torch.cuda.synchronize()
+        t_est = max(1e-4, ops / (burst_i8 * 1e12))
+        reps = max(10, int(sustain_s / t_est))
+        sampler.start()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        clocks = sampler.stop()
+        return ops * reps / (e0.elapsed_time(e1) / 1e3) / 1e12, clocks, reps
+
+    i8 = lambda: torch._int_mm(a, b)  # noqa: E731
+    bf = lambda: torch.matmul(ab, bb)  # noqa: E731
+    burst_i8 = burst(i8)
+    burst_bf = burst(bf)
+    sust_i8, clk, reps = sustained(i8)
+    rec = {"int8_tops": round(burst_i8, 1), "int8_tops_sustained": round(sust_i8, 1),
+           "sustained_sm_mhz_median": clk.get("sm_mhz"), "sustained_clocks": clk,
+           "bf16_tflops_same_box": round(burst_bf, 1), "int8_over_bf16_burst": round(burst_i8 / burst_bf, 3),
+           "gpu": torch.cuda.get_device_name(dev), "torch": torch.__version__,
+           "how": (f"torch._int_mm int8 {n}^3 (A row-major, B column-major; 2*n^3 ops): best of {burst_reps} "
+                   f"(CUDA events) and {reps} back-to-back launches with nvidia-smi clock samples; "
+                   f"torch.matmul bf16 {n}^3 best of {burst_reps} on the same box"),
+           "when": datetime.datetime.now(datetime.timezone.utc).strftime("%Y-%m-%dT%H:%M:%SZ"),
+           "command": "python bench.py --measure-int8-peak"}
+    os.makedirs(os.path.dirname(out_path), exist_ok=True)
+    with open(out_path, "w") as f:
+        json.dump(rec, f, indent=1)
+        f.write("\n")
+    print(json.dumps(rec), flush=True)
+
+
+def kernel_sweep(args):
+    """Each memory-bound kernel of the path timed alone at the d = 5120
+    workload sizes (CUDA events, median of the repetitions; every input is
+    larger than L2, so no flush is needed; outputs come from torch's caching
+    allocator, which launches nothing): algorithmic bytes, time, GB/s and the
+    fraction of the measured copy bandwidth.  One JSON line per kernel."""
+    from audio_diffusion_transformer_dit_b200 import h3b
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    pk, src = peaks()
+    hbm = pk.get("hbm_gbs")
+    wl4 = W.WORKLOADS[INT8_WORKLOAD]  # 20640 tokens x 5120, MLP 20480
+    wl5 = W.WORKLOADS["loop45_d5120_s6528"]  # 6528 tokens, merge 6144 -> 3072 video tokens
+    S, d, f = wl4.seq, wl4.d, wl4.ffn
+    x = W.normal_tensor((S, d), 11, dev)
+    g = torch.ones(d, dtype=torch.float32, device=dev)
+    abf = W.normal_tensor((S, d), 12, dev, dtype=torch.bfloat16)
+    gbf = W.normal_tensor((S, f), 13, dev, dtype=torch.bfloat16)
+    amax = gbf.float().abs().amax(dim=1).contiguous()
+    dm5 = h3b.dims_of(wl5)
+    x5 = W.normal_tensor((wl5.seq, wl5.d), 14, dev)
+    xm5 = torch.empty((wl5.seq_merged, wl5.d), dtype=torch.float32, device=dev)
+    v5 = W.normal_tensor((wl5.seq, wl5.d), 15, dev)
+    cp5 = torch.empty_like(v5)
+    # outputs allocated once: every timed launch is the library call alone
+    u_bf = torch.empty((S, d), dtype=torch.bfloat16, device=dev)
+    q_d = torch.empty((S, d), dtype=torch.int8, device=dev)
+    q_f = torch.empty((S, f), dtype=torch.int8, device=dev)
+    s_r = torch.empty(S, dtype=torch.float32, device=dev)
+    lib, st = h3b.lib, h3b._stream()
+    P = lambda t: t.data_ptr()  # noqa: E731
+    cases = [
+        ("rmsnorm_bf16", lambda: lib.h3b_rmsnorm(P(x), P(g), S, d, 1e-6, P(u_bf), None, h3b.BF16, st),
+         S * d * 4 + S * d * 2, f"x fp32 [{S},{d}] -> bf16"),
+        ("rmsnorm_int8", lambda: lib.h3b_rmsnorm(P(x), P(g), S, d, 1e-6, P(q_d), P(s_r), h3b.INT8, st),
+         S * d * 4 + S * d + S * 4, f"x fp32 [{S},{d}] -> int8 + scale"),
+        ("quant_rows", lambda: lib.h3b_quantize_weights(P(abf), S, d, P(q_d), P(s_r), st),
+         S * d * 2 + S * d + S * 4, f"o bf16 [{S},{d}] -> int8 + scale"),
+        ("quant_absmax", lambda: lib.h3b_quantize_rows_absmax(P(gbf), P(amax), S, f, P(q_f), P(s_r), st),
+         S * f * 2 + S * f + S * 8, f"g bf16 [{S},{f}] + row max -> int8 + scale"),
+        ("token_merge", lambda: lib.h3b_token_merge(ctypes.byref(dm5), P(x5), P(xm5), st),
+         (wl5.seq + wl5.seq_merged) * wl5.d * 4, f"x fp32 [{wl5.seq},{wl5.d}] -> [{wl5.seq_merged},{wl5.d}]"),
+        ("token_unmerge", lambda: lib.h3b_token_unmerge(ctypes.byref(dm5), P(xm5), P(x5), st),
+         (wl5.seq + wl5.seq_merged) * wl5.d * 4, f"xm fp32 [{wl5.seq_merged},{wl5.d}] -> [{wl5.seq},{wl5.d}]"),
+        ("flow_step", lambda: lib.h3b_flow_step(P(x5), P(v5), ctypes.c_float(0.5), ctypes.c_float(0.45),
+                                                 ctypes.c_size_t(x5.numel()), None, st),
+         3 * wl5.seq * wl5.d * 4, f"x, v fp32 [{wl5.seq},{wl5.d}] -> x"),
+        ("flow_step_copy", lambda: lib.h3b_flow_step(P(x5), P(v5), ctypes.c_float(0.5), ctypes.c_float(0.45),
+                                                      ctypes.c_size_t(x5.numel()), P(cp5), st),
+         4 * wl5.seq * wl5.d * 4, f"x, v fp32 [{wl5.seq},{wl5.d}] -> x and a copy"),
+    ]
+    only = set(args.sweep_only.split(",")) if args.sweep_only else None
+    # contractions, timed alone: the INT8 and BF16 FC1 GEMMs (GELU epilogue;
+    # INT8 also writes the per-row max) and the attention of both d = 5120
+    # workloads; built only when selected (they hold ~1-3 GB)
+    tensor_cases = {
+        "gemm_fc1_int8": (INT8_WORKLOAD, "int8"), "gemm_fc1_bf16": (DEFAULT_WORKLOAD, "bf16"),
+        "attention_s6528": (DEFAULT_WORKLOAD, None), "attention_s20640": (INT8_WORKLOAD, None),
+    }
+    for name, (wname, kind) in tensor_cases.items():
+        if only is None or name not in only:
+            continue
+        wl = W.WORKLOADS[wname]
+        Sx, dx, fx = wl.seq, wl.d, wl.ffn
+        if name.startswith("gemm"):
+            if kind == "int8":
+                A = W.int8_tensor((Sx, dx), 21, dev)
+                B = W.int8_tensor((fx, dx), 22, dev)
+                sa = W.uniform_tensor((Sx,), 23, dev, 1e-3, 2e-3)
+                sb = W.uniform_tensor((fx,), 24, dev, 1e-3, 2e-3)
+            else:
+                A = W.normal_tensor((Sx, dx), 21, dev, dtype=torch.bfloat16)
+                B = W.normal_tensor((fx, dx), 22, dev, std=0.02, dtype=torch.bfloat16)
+                sa = sb = None
+            C = torch.empty((Sx, fx), dtype=torch.bfloat16, device=dev)
+            rmax = torch.zeros(Sx, dtype=torch.float32, device=dev) if kind == "int8" else None
+            fn = (lambda A=A, B=B, C=C, sa=sa, sb=sb, rmax=rmax:
+                  h3b.gemm(A, B, h3b.EPI_GELU, C, scale_a=sa, scale_b=sb, row_absmax=rmax))
+            work = 2.0 * Sx * fx * dx
+            shape = f"{kind} [{Sx},{dx}] x [{fx},{dx}]^T -> GELU bf16"
+        else:
+            qkv = W.normal_tensor((Sx, 3 * dx), 25, dev, dtype=torch.bfloat16)
+            o = torch.empty((Sx, dx), dtype=torch.bfloat16, device=dev)
+            scr = torch.empty(2 * Sx * dx, dtype=torch.float32, device=dev)
+            fn = (lambda qkv=qkv, o=o, scr=scr, wl=wl:
+                  h3b.attention(qkv, wl.n_heads, wl.head_dim, o=o, scratch=scr))
+            work = 4.0 * Sx * Sx * dx
+            shape = f"bf16 S={Sx}, {wl.n_heads} heads x {wl.head_dim}"
+        cases.append((name, fn, work, shape))
+    for name, fn, amount, shape in cases:
+        if only and name not in only:
+            continue
+        tensor = name in tensor_cases
+        for _ in range(args.sweep_warmup):
+            rc = fn()
+            assert not isinstance(rc, int) or rc == 0, f"{name}: status {rc}"
+        torch.cuda.synchronize()
+        assert h3b.device_error() == 0
+        # back-to-back launches between two events (the launch latency of one
+        # call hides behind the previous kernel), in groups; the median group
+        group = max(1, args.sweep_group)
+        times = []
+        sampler = ClockSampler(0)
+        sampler.start()
+        for _ in range(max(1, args.sweep_reps // group)):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(group):
+                fn()
+            e1.record()
+            torch.cuda.synchronize()
+            times.append(e0.elapsed_time(e1) / group)
+        clocks = sampler.stop()
+        assert h3b.device_error() == 0
+        t = statistics.median(times) / 1e3
+        rec = {"kernel": name, "shape": shape, "us_median": round(t * 1e6, 2), "us_min": round(min(times) * 1e3, 2),
+               "launches": group * len(times), "clocks": clocks}
+        if tensor:
+            tp = tensor_peak(pk, clocks, int8=name.endswith("int8"))
+            rate = amount / t / 1e12
+            rec.update({"work": amount, "unit": "TOP/s" if name.endswith("int8") else "TFLOP/s",
+                        "achieved": round(rate, 1), "peak": tp["peak"], "frac": round(rate / tp["peak"], 4),
+                        "peak_basis": tp["basis"], "frac_nominal": round(rate / tp["nominal"], 4)})
+        else:
+            rec.update({"bytes": amount, "gbs": round(amount / t / 1e9, 1), "frac": round(amount / t / 1e9 / hbm, 4),
+                        "peak_gbs": hbm, "peak_source": src})
+        print(json.dumps(rec), flush=True)
 
 
 def main():
@@ -578,6 +875,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-int8", action="store_true",
+                    help="default workload: skip the INT8 d=5120 S=20640 block sub-record")
     ap.add_argument("--core-reuse", type=int, default=0,
                     help="loop workload: core residual reuse over the reduction window (replaces velocity reuse)")
     ap.add_argument("--unmerge-delta", action="store_true", help="loop workload: delta-broadcast unmerge")
@@ -589,9 +888,22 @@ def main():
                     help="loop workload: fixed condition rows appended after the audio tokens")
     ap.add_argument("--modulation", action="store_true",
                     help="loop workload: per-step, per-block timestep modulation (shift/scale/gate)")
-    ap.add_argument("--cpu-budget", type=float, default=30.0)
+    ap.add_argument("--measure-int8-peak", action="store_true",
+                    help="measure the dense int8 tensor peak (torch._int_mm) and write profiles/int8_peak.json")
+    ap.add_argument("--kernel-sweep", action="store_true",
+                    help="time each memory-bound kernel alone at the d=5120 sizes (GB/s vs the copy bandwidth)")
+    ap.add_argument("--sweep-only", default="", help="comma-separated kernel names for --kernel-sweep")
+    ap.add_argument("--sweep-reps", type=int, default=50)
+    ap.add_argument("--sweep-warmup", type=int, default=5)
+    ap.add_argument("--sweep-group", type=int, default=10, help="back-to-back launches per timed group")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # never fewer than 3 warm-up steps
+    if args.measure_int8_peak:
+        measure_int8_peak(INT8_PEAK_FILE)
+        return
+    if args.kernel_sweep:
+        kernel_sweep(args)
+        return
     wl = W.WORKLOADS[args.workload]
     if (args.layers or args.denoise_steps or args.cond_rows or args.modulation or args.core_reuse
             or args.unmerge_delta) and wl.steps == 0:

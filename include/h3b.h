@@ -246,7 +246,10 @@ int h3b_flow_step(float* x, const float* v, float sigma_cur, float sigma_next, s
  *     S ~ 3000 tokens.
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress, with that device current); make that first call
- *     before any stream capture.
+ *     before any stream capture.  The address is kept for the life of the
+ *     process: after cudaDeviceReset on a device it is stale, and this entry
+ *     point (like the rest of the library) must not be called on that device
+ *     again.
  *   - Calls allocate nothing (no cudaMalloc/cudaFree, no allocating library
  *     routine).
  *   - Every call shares the one array per device, which keeps the previous

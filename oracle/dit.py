@@ -95,6 +95,8 @@ PINS = {
     "quantize_rows_known_max": "hand-computed codes with a given max below the row's (clamping), zero max; "
                                "equals quantize_rows at the row's own max",
     "int8_matmul": "pure-Python integer dot products",
+    "block_forward_w8a8": "pure-Python loop block with per-element fp32 quantisation and exact integer dot "
+                          "products; row sampling = full rows; close to block_forward on the dequantised weights",
     "sigmas/fresh/denoise": "fresh counts 20/11/8 at 20 steps (control table); v = 0 identity; "
                             "single-step closed form",
     "token_unmerge_delta": "explicit (f, r, c) loops; equals plain unmerge when x_pre is pair-constant; "
@@ -402,20 +404,26 @@ def _w8a8_linear(a, wq, ws):
     return acc * _f64(sa)[:, None] * _f64(ws)[None, :]
 
 
-def block_forward_w8a8(x, w, dims, merged=False, rope=True):
-    """Diagnostic block with every GEMM input fake-quantised per token as well
-    as the weights per output channel (the full W8A8 arithmetic in fp64)."""
+def block_forward_w8a8(x, w, dims, merged=False, rope=True, rows=None):
+    """Block with every GEMM input fake-quantised per token as well as the
+    weights per output channel (the full W8A8 arithmetic in fp64).  ``rows``
+    as in block_forward: x2 only at those tokens, keys and values over all
+    (per-token quantisation keeps every row independent of the others)."""
     x = _f64(x)
-    d, H = x.shape[1], dims.n_heads
+    S, d, H = x.shape[0], x.shape[1], dims.n_heads
+    rows = np.arange(S) if rows is None else np.asarray(rows)
     qw = {k: quantize_rows(w[k]) for k in ("w_qkv", "w_o", "w_fc1", "w_fc2")}
     u = rmsnorm(x, w["g_attn"], dims.eps)
-    qkv = _w8a8_linear(u, *qw["w_qkv"])
-    q, k, v = qkv[:, :d], qkv[:, d:2 * d], qkv[:, 2 * d:]
+    qa, sa = quantize_rows(u)
+    wq, ws = qw["w_qkv"]
+    k = (qa.astype(np.float64) @ wq[d:2 * d].astype(np.float64).T) * _f64(sa)[:, None] * _f64(ws[d:2 * d])[None, :]
+    v = (qa.astype(np.float64) @ wq[2 * d:].astype(np.float64).T) * _f64(sa)[:, None] * _f64(ws[2 * d:])[None, :]
+    q = (qa[rows].astype(np.float64) @ wq[:d].astype(np.float64).T) * _f64(sa[rows])[:, None] * _f64(ws[:d])[None, :]
     if rope:
         ang = rope_angles(dims, merged)
-        q, k = apply_rope(q, ang, H), apply_rope(k, ang, H)
+        q, k = apply_rope(q, ang[rows], H), apply_rope(k, ang, H)
     o = attention(q, k, v, H)
-    x1 = x + _w8a8_linear(o, *qw["w_o"])
+    x1 = x[rows] + _w8a8_linear(o, *qw["w_o"])
     g = gelu(_w8a8_linear(rmsnorm(x1, w["g_mlp"], dims.eps), *qw["w_fc1"]))
     return x1 + _w8a8_linear(g, *qw["w_fc2"])
 

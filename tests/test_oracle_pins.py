@@ -166,13 +166,26 @@ def test_attention_uniform_and_convex():
 
 
 # ----------------------------------------------------------------------------- block
-def brute_block(x, w, dm, merged=False, mod=None, n_cond=0):
+def quant_row_py(vals):
+    """Per-row symmetric int8 by the fp32 rule, element by element: s =
+    fp32(max|v|) / 127 in fp32, code = round-half-even(fp32(v) / s) (IEEE fp32
+    quotient) clamped to +-127; a zero row gives s = 0 and zero codes."""
+    a32 = [np.float32(t) for t in vals]
+    s = np.float32(max(abs(t) for t in a32) / np.float32(127.0))
+    if s == 0:
+        return [0] * len(a32), 0.0
+    return [int(min(127, max(-127, round(float(t / s))))) for t in a32], float(s)
+
+
+def brute_block(x, w, dm, merged=False, mod=None, n_cond=0, w8a8=False):
     """Pure-Python loops: RMSNorm, QKV, RoPE by explicit (f,r,c)/audio
     positions, softmax attention, output projection, RMSNorm, GELU MLP.
     With ``mod`` ([2][6][d] nested lists: shift/scale/gate for attention, then
     for the MLP; class 1 = the last n_cond rows) each normed row becomes
     u*(1+scale)+shift and each residual update is multiplied by its gate;
-    the n_cond condition rows get no rotation."""
+    the n_cond condition rows get no rotation.  With ``w8a8`` every GEMM takes
+    int8 codes of its input row and of each weight row (quant_row_py) and
+    returns float(exact integer dot product) * s_input * s_weight."""
     S, d, H, D, f = len(x), dm.d, dm.n_heads, dm.head_dim, dm.ffn
     if mod is None:
         ident = [[0.0] * d, [0.0] * d, [1.0] * d]
@@ -181,12 +194,16 @@ def brute_block(x, w, dm, merged=False, mod=None, n_cond=0):
     def cls(i):
         return 1 if i >= S - n_cond else 0
     wqkv, wo, w1, w2 = (w[k].tolist() for k in ("w_qkv", "w_o", "w_fc1", "w_fc2"))
+    wq = {id(W): [quant_row_py(r) for r in W] for W in (wqkv, wo, w1, w2)} if w8a8 else None
 
     def norm(row, g):
         r = 1.0 / math.sqrt(sum(a * a for a in row) / d + dm.eps)
         return [a * r * gg for a, gg in zip(row, g)]
 
     def mv(W, a):
+        if w8a8:
+            qa, sa = quant_row_py(a)
+            return [float(sum(qa[i] * qw[i] for i in range(len(a)))) * sa * sw for qw, sw in wq[id(W)]]
         return [sum(wr[i] * a[i] for i in range(len(a))) for wr in W]
 
     F, Hr, Wc, A = dm.frames, dm.rows, dm.cols, dm.n_audio
@@ -483,6 +500,23 @@ def test_int8_matmul_vs_python():
             assert acc[m, n] == sum(int(qa[m, k]) * int(qw[n, k]) for k in range(37))
     big_a = np.full((1, 4096), 127, np.int8)
     assert oracle.int8_matmul(big_a, -big_a)[0, 0] == -127 * 127 * 4096
+
+
+@pytest.mark.parametrize("merged", [False, True])
+def test_w8a8_block_vs_bruteforce(merged):
+    """The W8A8 block against pure-Python loops with per-element fp32
+    quantisation and exact integer dot products; row sampling = full rows."""
+    dm = dims_of(1, 2, 4, 2, 32, 2, 64)
+    rng = np.random.default_rng(16)
+    S = (4 if merged else 8) + 2
+    x = rng.normal(size=(S, 32))
+    w = rand_block(rng, 32, 64)
+    ref = brute_block(x.tolist(), w, dm, merged, w8a8=True)
+    got = oracle.block_forward_w8a8(x, w, dm, merged=merged)
+    assert np.allclose(got, ref, rtol=1e-11, atol=1e-12)
+    rows = np.array([0, 3, S - 1])
+    assert np.allclose(oracle.block_forward_w8a8(x, w, dm, merged=merged, rows=rows), got[rows], rtol=1e-13,
+                       atol=1e-13)
 
 
 def test_w8a8_block_close_to_dequant_reference():
