@@ -233,6 +233,7 @@ GemmArgs gemm_args(int M, int N, int K, void* C, const float* sa, const float* s
   a.gate_split = 0;
   a.gate_stride = 0;
   a.rope_rows = M;
+  a.group_n = 1;
   return a;
 }
 

@@ -36,15 +36,20 @@ constexpr int EPI_WARPS = 8;  // two warps per TMEM lane quarter, each half of t
 constexpr int THREADS = 64 + 32 * EPI_WARPS;
 constexpr int NUM_BARS = 2 * STAGES + 5;
 constexpr int SMEM_BYTES = 1024 + STAGES * (A_STAGE + B_STAGE) + NUM_BARS * 8 + 16;
-constexpr int GROUP_N = 8;  // N tiles per raster group (L2 reuse of A rows)
+#ifndef H3B_GEMM_STCS
+#define H3B_GEMM_STCS 0  // 1: bf16 epilogue stores marked streaming (evict first from L2)
+#endif
+#ifndef H3B_GEMM_GROUP
+#define H3B_GEMM_GROUP 0  // > 0: fixed raster group width instead of the L2-budget choice
+#endif
 
-// Tile t -> (m block, n block): groups of GROUP_N n-blocks, m-major inside a
+// Tile t -> (m block, n block): groups of group_n n-blocks, m-major inside a
 // group, so the tiles in flight share a band of B and sweep A.
-__device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int& mb, int& nb) {
-  const int per_group = num_m * GROUP_N;
+__device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int group_n, int& mb, int& nb) {
+  const int per_group = num_m * group_n;
   const int g = t / per_group;
-  const int first_n = g * GROUP_N;
-  const int gs = min(GROUP_N, num_n - first_n);
+  const int first_n = g * group_n;
+  const int gs = min(group_n, num_n - first_n);
   const int local = t - g * per_group;
   mb = local / gs;
   nb = first_n + local % gs;
@@ -247,8 +252,13 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& p, int m, int n, 
     }
   }
   uint4* c = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.C) + off);
+#if H3B_GEMM_STCS
+#pragma unroll
+  for (int i = 0; i < 4; ++i) __stcs(c + i, make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]));
+#else
 #pragma unroll
   for (int i = 0; i < 4; ++i) c[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+#endif
 }
 
 template <bool INT8, int EPI>
@@ -307,7 +317,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int u = blockIdx.x; u < num_units; u += gridDim.x) {
         int t, kb0, kb1, part, mb, nb;
         unit_range(u, p.full_tiles, p.split, num_kb, t, kb0, kb1, part);
-        tile_coords(t, num_m, num_n, mb, nb);
+        tile_coords(t, num_m, num_n, p.group_n, mb, nb);
         bool ok = true;
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(empty0 + 8 * stage, phase ^ 1, abort_flag, p.err, (EK_GEMM << 8) | 1)) {
@@ -381,7 +391,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int u = blockIdx.x; u < num_units; u += gridDim.x) {
       int t, kb0, kb1, part, mb, nb;
       unit_range(u, p.full_tiles, p.split, num_kb, t, kb0, kb1, part);
-      tile_coords(t, num_m, num_n, mb, nb);
+      tile_coords(t, num_m, num_n, p.group_n, mb, nb);
       const bool ok = mbar_wait(tfull0 + 8 * acc, acc_phase, abort_flag, p.err, (EK_GEMM << 8) | 4);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
@@ -435,12 +445,13 @@ __global__ void __launch_bounds__(THREADS, 1)
 template <int TM>
 __global__ void __launch_bounds__(BN) k_splitk_add(float* __restrict__ C, const float* __restrict__ partial, int M,
                                                    int N, int full_tiles, int split, int num_m, int num_n,
-                                                   const float* __restrict__ gate, int gate_split, int gate_stride) {
+                                                   int group_n, const float* __restrict__ gate, int gate_split,
+                                                   int gate_stride) {
   pdl_trigger();
   pdl_wait();
   const int i = blockIdx.x / TM, r = blockIdx.x % TM, col = threadIdx.x;
   int mb, nb;
-  tile_coords(full_tiles + i, num_m, num_n, mb, nb);
+  tile_coords(full_tiles + i, num_m, num_n, group_n, mb, nb);
   const int m = mb * TM + r, n = nb * BN + col;
   if (m >= M || n >= N) return;
   const float* src = partial + static_cast<size_t>(i) * split * (TM * BN) + r * BN + col;
@@ -591,7 +602,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int u = cid; u < num_units; u += nclusters) {
         int t, kb0, kb1, part, mb, nb;
         unit_range(u, p.full_tiles, p.split, num_kb, t, kb0, kb1, part);
-        tile_coords(t, num_m, num_n, mb, nb);
+        tile_coords(t, num_m, num_n, p.group_n, mb, nb);
         bool ok = true;
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(empty0 + 8 * stage, phase ^ 1, abort_flag, p.err, (EK_GEMM << 8) | 5)) {
@@ -674,7 +685,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int u = cid; u < num_units; u += nclusters) {
       int t, kb0, kb1, part, mb, nb;
       unit_range(u, p.full_tiles, p.split, num_kb, t, kb0, kb1, part);
-      tile_coords(t, num_m, num_n, mb, nb);
+      tile_coords(t, num_m, num_n, p.group_n, mb, nb);
       const bool ok = mbar_wait(tfull0 + 8 * acc, acc_phase, abort_flag, p.err, (EK_GEMM << 8) | 8);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
@@ -782,6 +793,17 @@ cudaError_t launch_gemm(const Ctx& c, const void* A, const void* B, int ab_int8,
   if (e != cudaSuccess) return e;
   const int num_m = (args.M + TM - 1) / TM, num_n = (args.N + BN - 1) / BN;
   const int tiles = num_m * num_n;
+  // Raster group width: A is read from HBM about once per group of group_n
+  // N tiles while the group's band of B stays in L2.  Measured HBM reads at
+  // d = 5120 (widths 1, 8, 16, 19, 40): 16 for B rows of at most 1.5 MB per
+  // N tile (the K = 5120 int8 GEMMs: FC1 at S = 20640 reads 652 MB at 16
+  // against 1167 MB at 8), 8 otherwise (bf16 FC1 958-969 MB at 8-16 but
+  // 1269 MB at 19; FC2 at K = 20480 1730 MB at 8, 2102 at 4, 1916 at 16).
+  {
+    int g = static_cast<double>(BN) * args.K * eb <= 1.5 * 1024 * 1024 ? 16 : 8;
+    if (H3B_GEMM_GROUP > 0) g = H3B_GEMM_GROUP;
+    args.group_n = g > num_n ? num_n : g;
+  }
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   int slots = c.num_sms;  // tiles in flight at once
@@ -831,11 +853,11 @@ cudaError_t launch_gemm(const Ctx& c, const void* A, const void* B, int ab_int8,
   if (pair)
     e = launch_pdl(c.stream, k_splitk_add<BM2>, dim3(rem * BM2), dim3(BN), 0, 1u, static_cast<float*>(args.C),
                    static_cast<const float*>(args.partial), args.M, args.N, args.full_tiles, args.split, num_m, num_n,
-                   args.gate, args.gate_split, args.gate_stride);
+                   args.group_n, args.gate, args.gate_split, args.gate_stride);
   else
     e = launch_pdl(c.stream, k_splitk_add<BM>, dim3(rem * BM), dim3(BN), 0, 1u, static_cast<float*>(args.C),
                    static_cast<const float*>(args.partial), args.M, args.N, args.full_tiles, args.split, num_m, num_n,
-                   args.gate, args.gate_split, args.gate_stride);
+                   args.group_n, args.gate, args.gate_split, args.gate_stride);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

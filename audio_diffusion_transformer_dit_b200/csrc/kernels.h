@@ -105,6 +105,8 @@ struct GemmArgs {
   const float* gate;
   int gate_split, gate_stride;
   int rope_rows;
+  // raster group width in N tiles (set by launch_gemm)
+  int group_n;
 };
 
 // A [M,K], B [N,K] K-major (bf16 or int8); C per epilogue.  scratch (may be

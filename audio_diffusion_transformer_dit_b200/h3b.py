@@ -15,14 +15,16 @@ from typing import Optional, Sequence
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libh3b.so")
+# H3B_LIBRARY names another build of the same library (e.g. one compiled with
+# different tuning macros); by default the in-tree libh3b.so is loaded.
+LIB_PATH = os.environ.get("H3B_LIBRARY") or os.path.join(_HERE, "libh3b.so")
 HEADER = os.path.join(os.path.dirname(_HERE), "include", "h3b.h")
 
 BF16, INT8 = 0, 1
 EPI_F32, EPI_BF16, EPI_QKV_ROPE, EPI_RESID, EPI_GELU, EPI_I32 = range(6)
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"libh3b.so is not built ({LIB_PATH}); run `python -m audio_diffusion_transformer_dit_b200.build`")
+    raise ImportError(f"the h3b library is not built ({LIB_PATH}); run `python -m audio_diffusion_transformer_dit_b200.build`")
 
 lib = ctypes.CDLL(LIB_PATH)
 

@@ -795,6 +795,7 @@ def kernel_sweep(args):
     # workloads; built only when selected (they hold ~1-3 GB)
     tensor_cases = {
         "gemm_fc1_int8": (INT8_WORKLOAD, "int8"), "gemm_fc1_bf16": (DEFAULT_WORKLOAD, "bf16"),
+        "gemm_fc2_bf16": (DEFAULT_WORKLOAD, "bf16"),
         "attention_s6528": (DEFAULT_WORKLOAD, None), "attention_s20640": (INT8_WORKLOAD, None),
     }
     for name, (wname, kind) in tensor_cases.items():
@@ -802,7 +803,14 @@ def kernel_sweep(args):
             continue
         wl = W.WORKLOADS[wname]
         Sx, dx, fx = wl.seq, wl.d, wl.ffn
-        if name.startswith("gemm"):
+        if name == "gemm_fc2_bf16":  # x [S, d] fp32 += g [S, f] W2 [d, f]^T
+            A = W.normal_tensor((Sx, fx), 21, dev, dtype=torch.bfloat16)
+            B = W.normal_tensor((dx, fx), 22, dev, std=0.02, dtype=torch.bfloat16)
+            C = W.normal_tensor((Sx, dx), 23, dev)
+            fn = lambda A=A, B=B, C=C: h3b.gemm(A, B, h3b.EPI_RESID, C)  # noqa: E731
+            work = 2.0 * Sx * fx * dx
+            shape = f"bf16 [{Sx},{fx}] x [{dx},{fx}]^T -> fp32 residual [{Sx},{dx}]"
+        elif name.startswith("gemm"):
             if kind == "int8":
                 A = W.int8_tensor((Sx, dx), 21, dev)
                 B = W.int8_tensor((fx, dx), 22, dev)

@@ -2,7 +2,8 @@
 
 Tolerances (per the block's stated bar): block output relative L2 <= 1e-2 and
 max-abs <= 5e-2 for BF16; relative L2 <= 2e-2 for INT8 against the oracle
-block run on the int8 round-trip of the weights.  The block update x2 - x is
+block run on the int8 round-trip of the weights, with element and per-token
+bounds derived in check_int8.  The block update x2 - x is
 also checked on its own (a stricter view: the residual dominates x2), with a
 bound derived from the bf16 roundings on the path (u, qkv, P, o, u2, GELU out:
 six roundings of 2^-9 relative each, attenuated through the GEMMs) -> 2e-2
@@ -50,9 +51,25 @@ def check_bf16(x0, got, ref):
 
 
 def check_int8(x0, got, ref):
+    """INT8 block output against the oracle block on the dequantised weights.
+
+    Relative L2 <= 2e-2 (the INT8 bound) and update relative L2 <= 6e-2.  The
+    per-token activation codes (a rounding of up to half a step, step = row
+    max / 127, at every GEMM input; bf16 roundings before each quantiser flip
+    codes too) make the error a sum of many small independent terms, so its
+    largest element grows with the output's scale and the sample size: the
+    element bound is 6 sigma of an error whose RMS is at the relative-L2 bound,
+    6 * 2e-2 * rms(ref) (measured at d = 5120, S = 20640: max-abs 0.22 against
+    0.35 allowed; 0.038 against 0.13 at d = 1024).  No token may be off by
+    more than twice the global bound, which a badly quantised token (a wrong
+    scale, a flipped sign) would break."""
     assert np.isfinite(got).all()
     assert rel_l2(got, ref) <= 2e-2
     assert rel_l2(got - x0, ref - x0) <= 6e-2
+    rms = float(np.sqrt(np.mean(np.asarray(ref, dtype=np.float64) ** 2)))
+    assert max_abs(got, ref) <= 6 * 2e-2 * rms
+    row_rel = np.linalg.norm(got - ref, axis=1) / np.maximum(np.linalg.norm(ref, axis=1), 1e-300)
+    assert row_rel.max() <= 4e-2
 
 
 @pytest.mark.parametrize("merged", [False, True])

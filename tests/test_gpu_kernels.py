@@ -96,7 +96,7 @@ def test_rope_table(cuda_dev, merged, hd):
 
 
 # ----------------------------------------------------------------------------- RMSNorm
-@pytest.mark.parametrize("rows,d", [(1, 128), (37, 256), (300, 3072), (129, 5120), (3, 8192)])
+@pytest.mark.parametrize("rows,d", [(1, 128), (37, 256), (300, 3072), (129, 5120), (3, 8192), (10000, 1024)])
 def test_rmsnorm_bf16(cuda_dev, rows, d):
     x = wlmod.normal_tensor((rows, d), 6, cuda_dev) * 2.0
     g = wlmod.uniform_tensor((d,), 7, cuda_dev, 0.5, 1.5)
@@ -107,7 +107,7 @@ def test_rmsnorm_bf16(cuda_dev, rows, d):
     assert np.all(np.abs(np64(u) - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-30)
 
 
-@pytest.mark.parametrize("rows,d", [(37, 256), (300, 5120)])
+@pytest.mark.parametrize("rows,d", [(37, 256), (300, 5120), (10000, 1024), (5, 8192)])
 def test_rmsnorm_int8(cuda_dev, rows, d):
     x = wlmod.normal_tensor((rows, d), 8, cuda_dev)
     g = torch.ones(d, device=cuda_dev)
@@ -123,10 +123,11 @@ def test_rmsnorm_int8(cuda_dev, rows, d):
 
 
 # ----------------------------------------------------------------------------- quantisation
-# one warp per row for 1024 <= k <= 6144 (ragged lanes at 1032, the widest at
-# 6144), one CTA per row outside that range (6152 just above it)
+# rows of up to 32 KB (k <= 16384) stream through shared memory, ragged at
+# 1032 and 6152, many rows per CTA at 12000 x 512; wider rows (20480, 32768)
+# take the one-CTA-per-row register kernel
 @pytest.mark.parametrize("rows,k", [(1, 8), (33, 256), (300, 5120), (17, 20480), (5, 32768), (37, 1024), (9, 1032),
-                                    (41, 6144), (6, 6152)])
+                                    (41, 6144), (6, 6152), (12000, 512), (3, 16384)])
 def test_quantize_weights_bitexact(cuda_dev, rows, k):
     w = (wlmod.normal_tensor((rows, k), 9, cuda_dev) * 0.02).to(torch.bfloat16)
     w[0, :] = 0  # zero row -> s = 0, q = 0
