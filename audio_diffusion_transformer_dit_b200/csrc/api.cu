@@ -72,7 +72,7 @@ struct Trace {
 const char* kKernelNames[KID_COUNT] = {"flow_step", "token_merge", "token_unmerge", "rope_table", "rmsnorm",
                                        "quant_rows", "quant_absmax", "gemm_qkv_rope", "gemm_o_resid",
                                        "gemm_fc1_gelu", "gemm_fc2_resid", "gemm", "attention", "memset",
-                                       "token_unmerge_delta", "copy", "gelu"};
+                                       "token_unmerge_delta", "copy", "gelu", "norm_scale"};
 
 struct TraceScope {
   TraceRec* rec = nullptr;
@@ -117,6 +117,7 @@ size_t al256(size_t x) { return (x + 255) & ~size_t(255); }
 //   overlays the rest (qkv, o and u1 are dead by then).
 struct Plan {
   size_t qkv, o, u1, oq, u2, g, gq;   // byte offsets inside the arena
+  size_t xb1, ss1, ss2, r1, r2;       // folded RMSNorm: next QKV input, partial sums, row factors (bf16)
   size_t arena, naive;                // arena bytes, bytes without aliasing
   size_t s_act, s_g, amax;            // fp32 [S] scale / max vectors (INT8)
   size_t rope, rope_m, xm;            // RoPE tables, merged-sequence buffer
@@ -182,6 +183,23 @@ Plan plan(const h3b_dims& dm, int dtype, int reduction, int keep_merged_input = 
     p.delta = off;
     off += al256(S * d * 4);
   }
+  p.xb1 = p.ss1 = p.ss2 = p.r1 = p.r2 = 0;
+  if (dtype != H3B_INT8) {
+    // bf16(x * g) for the next block's QKV GEMM (the arena is full while FC2
+    // reads the hidden activations), and the per-row partial sums of squares
+    // of both folded norms (2 per 256-column tile of d)
+    const size_t parts = 2 * ((d + 255) / 256);
+    p.xb1 = off;
+    off += al256(2 * d * S);
+    p.ss1 = off;
+    off += al256(S * parts * 4);
+    p.ss2 = off;
+    off += al256(S * parts * 4);
+    p.r1 = off;
+    off += al256(S * 4);
+    p.r2 = off;
+    off += al256(S * 4);
+  }
   p.total = off;
   return p;
 }
@@ -212,6 +230,8 @@ int check_weights(const h3b_block_weights* w, int dtype) {
     if ((expr) != cudaSuccess) return H3B_ERR_CUDA;          \
   } while (0)
 
+int norm_parts(const h3b_dims& dm) { return 2 * ((dm.d + 255) / 256); }
+
 GemmArgs gemm_args(int M, int N, int K, void* C, const float* sa, const float* sb, const float* rope,
                    const h3b_dims& dm, float* amax, int* err) {
   GemmArgs a;
@@ -234,6 +254,25 @@ GemmArgs gemm_args(int M, int N, int K, void* C, const float* sa, const float* s
   a.gate_stride = 0;
   a.rope_rows = M;
   a.group_n = 1;
+  a.xb = nullptr;
+  a.xb_gain = nullptr;
+  a.ss_out = nullptr;
+  a.ss_parts = norm_parts(dm);
+  a.row_scale = nullptr;
+  return a;
+}
+
+// Folded RMSNorm (bf16 blocks without modulation): the residual GEMM before
+// a norm writes bf16(x * g) and per-row partial sums of x^2; the GEMM after
+// it reads that copy and scales each row by 1 / sqrt(mean x^2 + eps).
+GemmArgs norm_out(GemmArgs a, __nv_bfloat16* xb, const float* gain, float* ss) {
+  a.xb = xb;
+  a.xb_gain = gain;
+  a.ss_out = ss;
+  return a;
+}
+GemmArgs norm_in(GemmArgs a, const float* r) {
+  a.row_scale = r;
   return a;
 }
 
@@ -248,8 +287,14 @@ GemmArgs gated(GemmArgs a, const float* gate, int split, int stride) {
 // filled).  mod (nullable): this block's modulation [2][6][d] fp32 -- row class
 // (generated, condition) x (shift, scale, gate of the attention half, then of
 // the MLP half).
+// Folded norms (bf16, no modulation): norm_in -- the previous block's FC2
+// left bf16(x * g_attn) in xb1 and the row sums in ss1, so RMSNorm1 is folded
+// into this block's QKV GEMM; next_gain (nullable) -- this block's FC2 leaves
+// the same for the next block, whose g_attn it is.  RMSNorm2 is folded into
+// the O-proj / FC1 pair inside every such block.
 int block_impl(const Ctx& c, const h3b_dims& dm, const h3b_block_weights& w, float* x, int merged, uint8_t* ws,
-               const Plan& p, const float* rope, const float* mod = nullptr) {
+               const Plan& p, const float* rope, const float* mod = nullptr, bool norm_in_ready = false,
+               const float* next_gain = nullptr) {
   const int Sg = seq_len(dm, merged), S = Sg + p.n_cond, d = dm.d, f = dm.ffn;
   Mod m1, m2;
   const float *gate1 = nullptr, *gate2 = nullptr;
@@ -269,24 +314,43 @@ int block_impl(const Ctx& c, const h3b_dims& dm, const h3b_block_weights& w, flo
   void* g = A + p.g;
   float* s_act = reinterpret_cast<float*>(ws + p.s_act);
   if (w.dtype == H3B_BF16) {
-    H3B_CU(KID_RMSNORM, launch_rmsnorm(c, x, w.g_attn, S, d, dm.eps, u1, nullptr, 0, m1));
+    const bool fold = !mod;  // the modulated norm is not a per-row scale
+    float* ss1 = reinterpret_cast<float*>(ws + p.ss1);
+    float* ss2 = reinterpret_cast<float*>(ws + p.ss2);
+    __nv_bfloat16* xb1 = reinterpret_cast<__nv_bfloat16*>(ws + p.xb1);
     qkv_args.C = qkv;
-    H3B_CU(KID_GEMM_QKV, launch_gemm(c, u1, w.w_qkv, 0, H3B_EPI_QKV_ROPE, qkv_args));
+    float* r1 = reinterpret_cast<float*>(ws + p.r1);
+    float* r2 = reinterpret_cast<float*>(ws + p.r2);
+    if (fold && norm_in_ready) {
+      H3B_CU(KID_NORM_SCALE, launch_norm_scale(c, ss1, S, norm_parts(dm), d, dm.eps, r1));
+      H3B_CU(KID_GEMM_QKV, launch_gemm(c, xb1, w.w_qkv, 0, H3B_EPI_QKV_ROPE, norm_in(qkv_args, r1)));
+    } else {
+      H3B_CU(KID_RMSNORM, launch_rmsnorm(c, x, w.g_attn, S, d, dm.eps, u1, nullptr, 0, m1));
+      H3B_CU(KID_GEMM_QKV, launch_gemm(c, u1, w.w_qkv, 0, H3B_EPI_QKV_ROPE, qkv_args));
+    }
     // the norm-1 arena is dead once the QKV GEMM has run: key-split attention partials
     H3B_CU(KID_ATTN, launch_attention(c, qkv, S, dm.n_heads, dm.head_dim, o, reinterpret_cast<float*>(u1),
                                       2 * static_cast<size_t>(d) * S));
-    // O-proj: the dead QKV arena holds split-K partials; FC2: the dead MLP-input arena
-    H3B_CU(KID_GEMM_O, launch_gemm(c, o, w.w_o, 0, H3B_EPI_RESID,
-                                   gated(gemm_args(S, d, d, x, nullptr, nullptr, nullptr, dm, nullptr, c.err), gate1,
-                                         Sg, 6 * d),
-                                   reinterpret_cast<float*>(A + p.qkv), p.o - p.qkv));
-    H3B_CU(KID_RMSNORM, launch_rmsnorm(c, x, w.g_mlp, S, d, dm.eps, u2, nullptr, 0, m2));
-    H3B_CU(KID_GEMM_FC1, launch_gemm(c, u2, w.w_fc1, 0, H3B_EPI_GELU,
-                                     gemm_args(S, f, d, g, nullptr, nullptr, nullptr, dm, nullptr, c.err)));
-    H3B_CU(KID_GEMM_FC2, launch_gemm(c, g, w.w_fc2, 0, H3B_EPI_RESID,
-                                     gated(gemm_args(S, d, f, x, nullptr, nullptr, nullptr, dm, nullptr, c.err),
-                                           gate2, Sg, 6 * d),
-                                     reinterpret_cast<float*>(A + p.u2), p.g - p.u2));
+    // O-proj: split-K partials in the dead QKV arena past the MLP-input slot,
+    // where the folded norm writes bf16(x1 * g_mlp) for FC1
+    GemmArgs o_args =
+        gated(gemm_args(S, d, d, x, nullptr, nullptr, nullptr, dm, nullptr, c.err), gate1, Sg, 6 * d);
+    if (fold) o_args = norm_out(o_args, reinterpret_cast<__nv_bfloat16*>(u2), w.g_mlp, ss2);
+    const size_t o_part = p.u2 + al256(2 * static_cast<size_t>(d) * S);
+    H3B_CU(KID_GEMM_O, launch_gemm(c, o, w.w_o, 0, H3B_EPI_RESID, o_args, reinterpret_cast<float*>(A + o_part),
+                                   p.o - o_part));
+    if (fold)
+      H3B_CU(KID_NORM_SCALE, launch_norm_scale(c, ss2, S, norm_parts(dm), d, dm.eps, r2));
+    else
+      H3B_CU(KID_RMSNORM, launch_rmsnorm(c, x, w.g_mlp, S, d, dm.eps, u2, nullptr, 0, m2));
+    GemmArgs fc1_args = gemm_args(S, f, d, g, nullptr, nullptr, nullptr, dm, nullptr, c.err);
+    H3B_CU(KID_GEMM_FC1, launch_gemm(c, u2, w.w_fc1, 0, H3B_EPI_GELU, fold ? norm_in(fc1_args, r2) : fc1_args));
+    // FC2: split-K partials in the dead MLP-input slot
+    GemmArgs fc2_args =
+        gated(gemm_args(S, d, f, x, nullptr, nullptr, nullptr, dm, nullptr, c.err), gate2, Sg, 6 * d);
+    if (fold && next_gain) fc2_args = norm_out(fc2_args, xb1, next_gain, ss1);
+    H3B_CU(KID_GEMM_FC2, launch_gemm(c, g, w.w_fc2, 0, H3B_EPI_RESID, fc2_args, reinterpret_cast<float*>(A + p.u2),
+                                     p.g - p.u2));
   } else {
     int8_t* oq = reinterpret_cast<int8_t*>(A + p.oq);
     int8_t* gq = reinterpret_cast<int8_t*>(A + p.gq);
@@ -336,11 +400,18 @@ int run_blocks(const Ctx& c, const h3b_dims& dm, const h3b_block_weights* blocks
   float* xm0 = on && udelta ? reinterpret_cast<float*>(ws + p.xm0) : nullptr;
   const int V = dm.frames * dm.rows * dm.cols;
   const int tail = dm.n_audio + p.n_cond;  // rows after the video rows, carried through the reduction
+  bool folded = false;  // block l-1's FC2 left block l's folded norm-1 input
   for (int l = lo; l <= hi; ++l) {
     if (on && l == mf) H3B_CU(KID_MERGE, launch_merge(c, x, xm, V, tail, dm.d, xm0));
     const bool merged = on && l >= mf && l <= ml;
+    // the chain of folded norms runs between unmodulated bf16 blocks on the
+    // same token grid (a merge or unmerge between two blocks breaks it)
+    const bool chain = !mod && l < hi && blocks[l].dtype == H3B_BF16 && blocks[l + 1].dtype == H3B_BF16 &&
+                       !(on && (l == ml || l + 1 == mf));
     H3B_TRY(block_impl(c, dm, blocks[l], merged ? xm : x, merged, ws, p, merged ? rope_m : rope,
-                       mod ? mod + static_cast<size_t>(l) * 12 * dm.d : nullptr));
+                       mod ? mod + static_cast<size_t>(l) * 12 * dm.d : nullptr, folded,
+                       chain ? blocks[l + 1].g_attn : nullptr));
+    folded = chain;
     if (on && l == ml) {
       if (udelta)
         H3B_CU(KID_UNMERGE_DELTA, launch_unmerge_delta(c, x, xm, xm0, V, tail, dm.d));

@@ -36,11 +36,8 @@ constexpr int EPI_WARPS = 8;  // two warps per TMEM lane quarter, each half of t
 constexpr int THREADS = 64 + 32 * EPI_WARPS;
 constexpr int NUM_BARS = 2 * STAGES + 5;
 constexpr int SMEM_BYTES = 1024 + STAGES * (A_STAGE + B_STAGE) + NUM_BARS * 8 + 16;
-#ifndef H3B_GEMM_STCS
-#define H3B_GEMM_STCS 0  // 1: bf16 epilogue stores marked streaming (evict first from L2)
-#endif
 #ifndef H3B_GEMM_GROUP
-#define H3B_GEMM_GROUP 0  // > 0: fixed raster group width instead of the L2-budget choice
+#define H3B_GEMM_GROUP 0  // > 0: a fixed raster group width (tuning builds) instead of the measured rule
 #endif
 
 // Tile t -> (m block, n block): groups of group_n n-blocks, m-major inside a
@@ -131,10 +128,31 @@ __device__ __forceinline__ void chunk_values(const GemmArgs& p, int m, int n, co
   }
 }
 
+// Folded RMSNorm factor of row m (1 when the GEMM has none).
+__device__ __forceinline__ float norm_row_scale(const GemmArgs& p, int m) {
+  return p.row_scale && m < p.M ? p.row_scale[m] : 1.f;
+}
+
+// Sums of squares of the rows a warp wrote (ssq[i] for row row0 + 4i + lane/8,
+// over this lane's columns) -> one partial per row and tile half.
+__device__ __forceinline__ void store_row_squares(const GemmArgs& p, int row0, int lane, int part, float (&ssq)[8]) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    float v = ssq[i];
+    v += __shfl_xor_sync(0xffffffffu, v, 1);
+    v += __shfl_xor_sync(0xffffffffu, v, 2);
+    v += __shfl_xor_sync(0xffffffffu, v, 4);
+    const int m = row0 + 4 * i + (lane >> 3);
+    if ((lane & 7) == 0 && m < p.M) p.ss_out[static_cast<size_t>(m) * p.ss_parts + part] = v;
+  }
+}
+
 // C[m, n .. n+32) += gate[class(m), n ..] * staged values (gate 1 when absent;
 // fmaf(1, v, c) rounds exactly like c + v), res = the prefetched C values.
+// With p.xb: also the bf16 copy of the new C times xb_gain, and each row's
+// sum of squares added to ssq.
 __device__ __forceinline__ void resid_rows(const GemmArgs& p, const float* stg, int row0, int n, int lane,
-                                           const float4 (&res)[8]) {
+                                           const float4 (&res)[8], float (&ssq)[8]) {
   const int col = n + 4 * (lane & 7);
   float4 g0 = make_float4(1.f, 1.f, 1.f, 1.f), g1 = g0;
   if (p.gate) {
@@ -154,6 +172,12 @@ __device__ __forceinline__ void resid_rows(const GemmArgs& p, const float* stg, 
       a.z = fmaf(g.z, v.z, a.z);
       a.w = fmaf(g.w, v.w, a.w);
       *reinterpret_cast<float4*>(C + static_cast<size_t>(m) * p.N) = a;
+      if (p.xb) {
+        const float4 gn = __ldg(reinterpret_cast<const float4*>(p.xb_gain + col));
+        *reinterpret_cast<uint2*>(p.xb + static_cast<size_t>(m) * p.N + col) =
+            make_uint2(pack_bf16x2(a.x * gn.x, a.y * gn.y), pack_bf16x2(a.z * gn.z, a.w * gn.w));
+        ssq[i] += a.x * a.x + a.y * a.y + a.z * a.z + a.w * a.w;
+      }
     }
   }
 }
@@ -170,7 +194,7 @@ __device__ __forceinline__ void partial_rows(float* part, const float* stg, int 
 template <bool INT8>
 __device__ __forceinline__ void resid_chunk(const GemmArgs& p, float* stg, int lane, int row0, int n, int ccol,
                                             const uint32_t (&r)[32], float* part, int trow0, float4 (&cnext)[8],
-                                            bool more) {
+                                            bool more, float (&ssq)[8]) {
   float v[32];
   chunk_values<INT8>(p, row0 + lane, n, r, v);
   stage_put(stg, lane, v);
@@ -182,13 +206,13 @@ __device__ __forceinline__ void resid_chunk(const GemmArgs& p, float* stg, int l
 #pragma unroll
   for (int i = 0; i < 8; ++i) cur[i] = cnext[i];
   if (more) load_resid_rows(p, row0, n + 32, lane, cnext);
-  resid_rows(p, stg, row0, n, lane, cur);
+  resid_rows(p, stg, row0, n, lane, cur, ssq);
 }
 
 // One 32-column chunk of one row (every epilogue but the residual one).
 template <bool INT8, int EPI>
 __device__ __forceinline__ void epilogue_chunk(const GemmArgs& p, int m, int n, const uint32_t (&r)[32],
-                                               float& row_amax) {
+                                               float& row_amax, float rs) {
   const size_t off = static_cast<size_t>(m) * p.N + n;
   if (EPI == H3B_EPI_I32) {
     int4* c = reinterpret_cast<int4*>(static_cast<int*>(p.C) + off);
@@ -213,6 +237,10 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& p, int m, int n, 
   } else {
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+  }
+  if (p.row_scale) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] *= rs;
   }
 
   if (EPI == H3B_EPI_F32) {
@@ -252,13 +280,8 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& p, int m, int n, 
     }
   }
   uint4* c = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.C) + off);
-#if H3B_GEMM_STCS
-#pragma unroll
-  for (int i = 0; i < 4; ++i) __stcs(c + i, make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]));
-#else
 #pragma unroll
   for (int i = 0; i < 4; ++i) c[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
-#endif
 }
 
 template <bool INT8, int EPI>
@@ -405,6 +428,8 @@ __global__ void __launch_bounds__(THREADS, 1)
               ? p.partial + (static_cast<size_t>(t - p.full_tiles) * p.split + part) * (BM * BN)
               : nullptr;
       float4 cnext[8];
+      float ssq[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      const float rs = EPI == H3B_EPI_RESID ? 1.f : norm_row_scale(p, m);
       if (EPI == H3B_EPI_RESID && !part_dst && nb * BN + c0 * 32 < p.N)
         load_resid_rows(p, m - lane, nb * BN + c0 * 32, lane, cnext);
 #pragma unroll 1
@@ -417,11 +442,12 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (EPI == H3B_EPI_RESID) {
           // K-parts of tail tiles write fp32 partials (added into C later, in part order)
           resid_chunk<INT8>(p, stg, lane, m - lane, n, c * 32, r, part_dst, q * 32, cnext,
-                            c + 1 < c1 && n + 32 < p.N);
+                            c + 1 < c1 && n + 32 < p.N, ssq);
         } else if (m < p.M) {
-          epilogue_chunk<INT8, EPI>(p, m, n, r, row_amax);
+          epilogue_chunk<INT8, EPI>(p, m, n, r, row_amax, rs);
         }
       }
+      if (EPI == H3B_EPI_RESID && p.xb && !part_dst) store_row_squares(p, m - lane, lane, 2 * nb + ch, ssq);
       if (INT8 && EPI == H3B_EPI_GELU && m < p.M)
         atomicMax(reinterpret_cast<int*>(p.row_absmax) + m, __float_as_int(row_amax));
       tc_fence_before();
@@ -442,26 +468,46 @@ __global__ void __launch_bounds__(THREADS, 1)
 
 // C[m, n] += sum over parts of the tail tiles' fp32 partials, in part order
 // (deterministic).  One CTA per (tail tile, row), one thread per column.
+// With xb set (folded RMSNorm): also the bf16 copy of C times xb_gain and the
+// row's sums of squares per 128-column tile half (the values the residual
+// epilogue writes for whole tiles).
 template <int TM>
 __global__ void __launch_bounds__(BN) k_splitk_add(float* __restrict__ C, const float* __restrict__ partial, int M,
                                                    int N, int full_tiles, int split, int num_m, int num_n,
                                                    int group_n, const float* __restrict__ gate, int gate_split,
-                                                   int gate_stride) {
+                                                   int gate_stride, __nv_bfloat16* __restrict__ xb,
+                                                   const float* __restrict__ xb_gain, float* __restrict__ ss_out,
+                                                   int ss_parts) {
   pdl_trigger();
   pdl_wait();
+  __shared__ float red[BN / 32];
   const int i = blockIdx.x / TM, r = blockIdx.x % TM, col = threadIdx.x;
   int mb, nb;
   tile_coords(full_tiles + i, num_m, num_n, group_n, mb, nb);
   const int m = mb * TM + r, n = nb * BN + col;
-  if (m >= M || n >= N) return;
-  const float* src = partial + static_cast<size_t>(i) * split * (TM * BN) + r * BN + col;
-  float acc = 0.f;
-  for (int q = 0; q < split; ++q) acc += src[static_cast<size_t>(q) * (TM * BN)];
-  if (gate)
-    C[static_cast<size_t>(m) * N + n] =
-        fmaf(gate[(m >= gate_split ? static_cast<size_t>(gate_stride) : 0) + n], acc, C[static_cast<size_t>(m) * N + n]);
-  else
-    C[static_cast<size_t>(m) * N + n] += acc;
+  if (m >= M) return;  // the whole CTA: m depends on the block only
+  float sq = 0.f;
+  if (n < N) {
+    const float* src = partial + static_cast<size_t>(i) * split * (TM * BN) + r * BN + col;
+    float acc = 0.f;
+    for (int q = 0; q < split; ++q) acc += src[static_cast<size_t>(q) * (TM * BN)];
+    float c = C[static_cast<size_t>(m) * N + n];
+    c = gate ? fmaf(gate[(m >= gate_split ? static_cast<size_t>(gate_stride) : 0) + n], acc, c) : c + acc;
+    C[static_cast<size_t>(m) * N + n] = c;
+    if (xb) {
+      xb[static_cast<size_t>(m) * N + n] = __float2bfloat16_rn(c * xb_gain[n]);
+      sq = c * c;
+    }
+  }
+  if (!xb) return;  // uniform: a kernel argument
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+  if ((col & 31) == 0) red[col >> 5] = sq;
+  __syncthreads();
+  if (col < 2) {  // warps 0-3 hold columns 0-127 of the tile, warps 4-7 columns 128-255
+    const float h = red[4 * col] + red[4 * col + 1] + red[4 * col + 2] + red[4 * col + 3];
+    ss_out[static_cast<size_t>(m) * ss_parts + 2 * nb + col] = h;
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -699,6 +745,8 @@ __global__ void __launch_bounds__(THREADS, 1)
               ? p.partial + (static_cast<size_t>(t - p.full_tiles) * p.split + part) * (BM2 * BN)
               : nullptr;
       float4 cnext[8];
+      float ssq[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      const float rs = EPI == H3B_EPI_RESID ? 1.f : norm_row_scale(p, m);
       if (EPI == H3B_EPI_RESID && !part_dst && nb * BN + c0 * 32 < p.N)
         load_resid_rows(p, m - lane, nb * BN + c0 * 32, lane, cnext);
 #pragma unroll 1
@@ -710,11 +758,12 @@ __global__ void __launch_bounds__(THREADS, 1)
         tmem_ld_wait();
         if (EPI == H3B_EPI_RESID) {
           resid_chunk<INT8>(p, stg, lane, m - lane, n, c * 32, r, part_dst, trow - lane, cnext,
-                            c + 1 < c1 && n + 32 < p.N);
+                            c + 1 < c1 && n + 32 < p.N, ssq);
         } else if (m < p.M) {
-          epilogue_chunk<INT8, EPI>(p, m, n, r, row_amax);
+          epilogue_chunk<INT8, EPI>(p, m, n, r, row_amax, rs);
         }
       }
+      if (EPI == H3B_EPI_RESID && p.xb && !part_dst) store_row_squares(p, m - lane, lane, 2 * nb + ch, ssq);
       if (INT8 && EPI == H3B_EPI_GELU && m < p.M)
         atomicMax(reinterpret_cast<int*>(p.row_absmax) + m, __float_as_int(row_amax));
       tc_fence_before();
@@ -768,7 +817,28 @@ GemmKernel pick(int epi) {
   }
 }
 
+// One thread per row: the row's partial sums of squares in order -> factor.
+__global__ void k_norm_scale(const float* __restrict__ ss, int rows, int parts, int d, float eps,
+                             float* __restrict__ r) {
+  pdl_trigger();
+  pdl_wait();
+  const int m = blockIdx.x * blockDim.x + threadIdx.x;
+  if (m >= rows) return;
+  const float* q = ss + static_cast<size_t>(m) * parts;
+  float s = 0.f;
+  for (int i = 0; i < parts; ++i) s += q[i];
+  r[m] = 1.0f / sqrtf(s / static_cast<float>(d) + eps);
+}
+
 }  // namespace
+
+cudaError_t launch_norm_scale(const Ctx& c, const float* ss, int rows, int parts, int d, float eps, float* r) {
+  if (rows == 0) return cudaSuccess;
+  const cudaError_t e = launch_pdl(c.stream, k_norm_scale, dim3((rows + 127) / 128), dim3(128), 0, 1u, ss, rows,
+                                   parts, d, eps, r);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
 
 cudaError_t launch_gemm(const Ctx& c, const void* A, const void* B, int ab_int8, int epi, const GemmArgs& args_in,
                         float* scratch, size_t scratch_bytes) {
@@ -853,11 +923,13 @@ cudaError_t launch_gemm(const Ctx& c, const void* A, const void* B, int ab_int8,
   if (pair)
     e = launch_pdl(c.stream, k_splitk_add<BM2>, dim3(rem * BM2), dim3(BN), 0, 1u, static_cast<float*>(args.C),
                    static_cast<const float*>(args.partial), args.M, args.N, args.full_tiles, args.split, num_m, num_n,
-                   args.group_n, args.gate, args.gate_split, args.gate_stride);
+                   args.group_n, args.gate, args.gate_split, args.gate_stride, args.xb, args.xb_gain, args.ss_out,
+                   args.ss_parts);
   else
     e = launch_pdl(c.stream, k_splitk_add<BM>, dim3(rem * BM), dim3(BN), 0, 1u, static_cast<float*>(args.C),
                    static_cast<const float*>(args.partial), args.M, args.N, args.full_tiles, args.split, num_m, num_n,
-                   args.group_n, args.gate, args.gate_split, args.gate_stride);
+                   args.group_n, args.gate, args.gate_split, args.gate_stride, args.xb, args.xb_gain, args.ss_out,
+                   args.ss_parts);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

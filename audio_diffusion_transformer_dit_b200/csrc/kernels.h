@@ -56,6 +56,7 @@ enum KernelId {
   KID_UNMERGE_DELTA,
   KID_COPY,
   KID_GELU,
+  KID_NORM_SCALE,
   KID_COUNT
 };
 
@@ -107,7 +108,20 @@ struct GemmArgs {
   int rope_rows;
   // raster group width in N tiles (set by launch_gemm)
   int group_n;
+  // RMSNorm folded across two GEMMs (bf16 residual stream).  Residual
+  // epilogue, when xb is set: also writes xb[m, n] = bf16(C[m, n] * xb_gain[n])
+  // and, per row and 128-column tile half, the sum of C^2 into
+  // ss_out[m * ss_parts + 2 * tile_n + half] (launch_norm_scale turns those
+  // into one factor per row).  Other epilogues, when row_scale is set: scale
+  // the accumulator of row m by row_scale[m] before RoPE / GELU.
+  __nv_bfloat16* xb;
+  const float* xb_gain;
+  float* ss_out;
+  int ss_parts;
+  const float* row_scale;
 };
+// r[m] = 1 / sqrt(sum_q ss[m * parts + q] / d + eps), q in order (deterministic).
+cudaError_t launch_norm_scale(const Ctx& c, const float* ss, int rows, int parts, int d, float eps, float* r);
 
 // A [M,K], B [N,K] K-major (bf16 or int8); C per epilogue.  scratch (may be
 // NULL) lets a residual GEMM split its last partial wave along K.

@@ -349,6 +349,18 @@ __device__ __forceinline__ uint2 quant8(const float (&f)[8], float s, float rs) 
   return make_uint2(quant4(f[0], f[1], f[2], f[3], s, rs), quant4(f[4], f[5], f[6], f[7], s, rs));
 }
 
+// max |.| of 8 bf16 on packed pairs: the sign bits cleared, then bf16x2 max
+// (exact: the max of bf16 magnitudes is one of them), widened once.
+__device__ __forceinline__ uint32_t bf16x2_absmax(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a & 0x7fff7fffu), "r"(b & 0x7fff7fffu));
+  return r;
+}
+__device__ __forceinline__ float bf16x8_absmax(const uint4& u) {
+  const uint32_t m = bf16x2_absmax(bf16x2_absmax(u.x, u.y), bf16x2_absmax(u.z, u.w));
+  return fmaxf(__uint_as_float(m << 16), __uint_as_float(m & 0xffff0000u));
+}
+
 // One CTA per row: max |row| then codes, row held in registers.
 template <int VPT>
 __global__ void __launch_bounds__(kThreads) k_quant_rows(const uint4* __restrict__ a, int k8, int8_t* __restrict__ q,
@@ -364,10 +376,7 @@ __global__ void __launch_bounds__(kThreads) k_quant_rows(const uint4* __restrict
   for (int i = 0; i < VPT; ++i) {
     const int c = threadIdx.x + i * blockDim.x;
     v[i] = c < k8 ? ar[c] : make_uint4(0, 0, 0, 0);
-    float f[8];
-    bf16x8_to_f32(v[i], f);
-#pragma unroll
-    for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(f[j]));
+    amax = fmaxf(amax, bf16x8_absmax(v[i]));
   }
   amax = block_reduce<true>(amax, red);
   const float s = amax / 127.0f, rs = 1.0f / s;
@@ -520,7 +529,14 @@ cudaError_t launch_rmsnorm(const Ctx& c, const float* x, const float* g, int row
 cudaError_t launch_quant_rows(const Ctx& c, const void* a, int rows, int k, int8_t* q, float* s) {
   if (rows == 0) return cudaSuccess;
   const int k8 = k / 8;
-  const int threads = k8 >= kThreads ? kThreads : ((k8 + 31) / 32) * 32;
+  // the most warps (8 down to 5) that give every thread the same number of
+  // 16-byte units (no idle lanes: k = 5120 takes 160 threads x 4), else 256
+  int threads = k8 >= kThreads ? kThreads : ((k8 + 31) / 32) * 32;
+  for (int w = 8; w >= 5 && k8 > kThreads; --w)
+    if (k8 % (32 * w) == 0 && k8 / (32 * w) <= 16) {
+      threads = 32 * w;
+      break;
+    }
   const int vpt = (k8 + threads - 1) / threads;
   const uint4* a4 = reinterpret_cast<const uint4*>(a);
   cudaError_t e;

@@ -236,7 +236,9 @@ def kernel_work(name, wl, dtype, merged=False):
               "rope_table": S * (wl.head_dim // 2) * 8,
               "token_merge": wl.seq * d * 4 + wl.seq_merged * d * 4,
               "token_unmerge": wl.seq * d * 4 + wl.seq_merged * d * 4,
-              "flow_step": wl.seq * d * 4 * 3}
+              "flow_step": wl.seq * d * 4 * 3,
+              # folded RMSNorm: each row's partial sums of squares (2 per 256 columns) -> one factor
+              "norm_scale": S * (2 * ((d + 255) // 256)) * 4 + S * 4}
     if name in nbytes:
         return float(nbytes[name]), "GB/s", "hbm"
     return None, None, None

@@ -152,7 +152,13 @@ def test_stack_small_vs_oracle(cuda_dev, mf, ml):
 
 
 def test_stack_equals_block_sequence(cuda_dev):
-    """h3b_stack_forward = merge + the same block calls + unmerge, bit for bit."""
+    """h3b_stack_forward = merge + the same block calls + unmerge.  Inside the
+    stack, consecutive blocks on the same token grid (blocks 1..3 in the merged
+    window) take their RMSNorm1 folded into the QKV GEMM (the previous FC2
+    leaves bf16(x * g) and the row sums of squares), where a lone block call
+    normalises first: the two differ only by where one bf16 rounding of the
+    normed operand falls (~2^-9 relative on the GEMM input), while a wrong
+    merge, unmerge, row-sum table or stale bf16 copy would be off by O(1)."""
     wl = TINY.with_(n_blocks=5, depth_scaled_init=True, seed=6)
     x0, x, _, blocks, ws = run_stack(wl, cuda_dev, 1, 3)
     dm = h3b.dims_of(wl)
@@ -166,20 +172,28 @@ def test_stack_equals_block_sequence(cuda_dev):
     h3b.token_unmerge(dm, ym, y)
     h3b.block_forward(dm, blocks[4], y, ws)
     torch.cuda.synchronize()
-    assert torch.equal(x, y)
+    assert rel_l2(x, y) <= 2e-3 and max_abs(x, y) <= 2e-2
+    assert rel_l2(x - x0, y - x0) <= 1e-2
 
 
 @pytest.mark.slow
 def test_stack8_full_size_equals_blocks(cuda_dev):
+    """The benched 8-block stack against the same blocks called one by one
+    (blocks 1..7 take the folded RMSNorm1 in the stack; see
+    test_stack_equals_block_sequence), and the stack run twice is bit-identical
+    (the folded norm sums its row partials in a fixed order)."""
     wl = wlmod.WORKLOADS["stack8_d5120_s6528"]
     x0, x, _, blocks, ws = run_stack(wl, cuda_dev)
     dm = h3b.dims_of(wl)
     y = x0.clone()
     for b in blocks:
         h3b.block_forward(dm, b, y, ws)
+    x2 = x0.clone()
+    h3b.stack_forward(dm, blocks, x2, ws)
     torch.cuda.synchronize()
-    assert torch.equal(x, y)
     assert torch.isfinite(x).all()
+    assert torch.equal(x, x2)
+    assert rel_l2(x, y) <= 2e-3 and rel_l2(x - x0, y - x0) <= 1e-2
 
 
 # ----------------------------------------------------------------------------- denoising loop
@@ -415,20 +429,33 @@ def test_modulated_block_with_condition_rows_vs_oracle(cuda_dev, int8):
     (check_int8 if int8 else check_bf16)(np64(x0), np64(x), ref)
 
 
-def test_identity_modulation_is_bitexact(cuda_dev):
-    wl = TINY.with_(n_blocks=3, depth_scaled_init=True, seed=12)
-    blocks = [h3b.Block.from_dict(wlmod.block_weights(wl, l, cuda_dev)) for l in range(3)]
+@pytest.mark.parametrize("int8", [True, False])
+def test_identity_modulation_is_bitexact(cuda_dev, int8):
+    """Zero shifts and scales with unit gates reproduce the unmodulated stack.
+    INT8 blocks normalise in a separate pass either way: bit for bit.  Without
+    modulation, bf16 blocks fold their RMSNorms into the neighbouring GEMMs
+    (the modulated norm is not a per-row scale and stays a separate pass), so
+    the two bf16 runs differ only by where one bf16 rounding of each normed
+    GEMM input falls."""
+    wl = TINY.with_(n_blocks=3, depth_scaled_init=True, seed=12, dtype=h3b.INT8 if int8 else h3b.BF16)
+    ws_ = [wlmod.block_weights(wl, l, cuda_dev) for l in range(3)]
+    blocks = [h3b.Block.quantized(w) if int8 else h3b.Block.from_dict(w) for w in ws_]
     dm = h3b.dims_of(wl)
+    dt = h3b.INT8 if int8 else h3b.BF16
     ident = torch.zeros((3, 2, 6, wl.d), device=cuda_dev)
     ident[..., 2, :] = 1.0
     ident[..., 5, :] = 1.0
     x = wlmod.initial_tokens(wl, cuda_dev)
+    x0 = x.clone()
     y = x.clone()
     o = h3b.stack_opts(0, 1, modulation=ident)
-    h3b.stack_forward_ex(dm, blocks, x, h3b.workspace_ex(dm, o), o)
-    h3b.stack_forward(dm, blocks, y, h3b.workspace(dm, h3b.BF16, True), 0, 1)
+    h3b.stack_forward_ex(dm, blocks, x, h3b.workspace_ex(dm, o, dt), o)
+    h3b.stack_forward(dm, blocks, y, h3b.workspace(dm, dt, True), 0, 1)
     torch.cuda.synchronize()
-    assert torch.equal(x, y)
+    if int8:
+        assert torch.equal(x, y)
+    else:
+        assert rel_l2(x, y) <= 2e-3 and rel_l2(x - x0, y - x0) <= 1e-2
 
 
 @pytest.mark.parametrize("delta", [False, True])
