@@ -160,6 +160,7 @@ __device__ __forceinline__ void resid_rows(const GemmArgs& p, const float* stg, 
     if (p.gate_split < p.M) g1 = __ldg(reinterpret_cast<const float4*>(p.gate + static_cast<size_t>(p.gate_stride) + col));
   }
   float* C = static_cast<float*>(p.C) + col;
+  const float4 gn = p.xb ? __ldg(reinterpret_cast<const float4*>(p.xb_gain + col)) : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const int m = row0 + 4 * i + (lane >> 3);
@@ -173,7 +174,6 @@ __device__ __forceinline__ void resid_rows(const GemmArgs& p, const float* stg, 
       a.w = fmaf(g.w, v.w, a.w);
       *reinterpret_cast<float4*>(C + static_cast<size_t>(m) * p.N) = a;
       if (p.xb) {
-        const float4 gn = __ldg(reinterpret_cast<const float4*>(p.xb_gain + col));
         *reinterpret_cast<uint2*>(p.xb + static_cast<size_t>(m) * p.N + col) =
             make_uint2(pack_bf16x2(a.x * gn.x, a.y * gn.y), pack_bf16x2(a.z * gn.z, a.w * gn.w));
         ssq[i] += a.x * a.x + a.y * a.y + a.z * a.z + a.w * a.w;
