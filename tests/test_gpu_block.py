@@ -477,6 +477,44 @@ def test_condition_stack_with_reduction_vs_oracle(cuda_dev, delta):
     check_bf16(np64(x0), np64(x), ref)
 
 
+@pytest.mark.parametrize("delta", [False, True])
+def test_condition_stack_without_modulation_vs_oracle(cuda_dev, delta):
+    """Condition rows without modulation: the RMSNorms are folded into the
+    GEMMs over every row, condition rows included (blocks 1..3 on the merged
+    grid chain their norm-1 through the previous FC2)."""
+    wl = TINY.with_(n_blocks=5, depth_scaled_init=True, seed=15)
+    C = 20
+    ws_ = [wlmod.block_weights(wl, l, cuda_dev) for l in range(5)]
+    blocks = [h3b.Block.from_dict(w) for w in ws_]
+    dm = h3b.dims_of(wl)
+    x0 = wlmod.initial_tokens(wl, cuda_dev, seq=wl.seq + C)
+    x = x0.clone()
+    o = h3b.stack_opts(1, 3, unmerge_delta=delta, n_cond=C)
+    h3b.stack_forward_ex(dm, blocks, x, h3b.workspace_ex(dm, o), o)
+    torch.cuda.synchronize()
+    assert h3b.device_error() == 0
+    ref = oracle.stack_forward_cond(np64(x0), [host_weights(w) for w in ws_], wl, None, C, 1, 3,
+                                    unmerge_delta=delta)
+    check_bf16(np64(x0), np64(x), ref)
+
+
+@pytest.mark.parametrize("n_blocks", [1, 3])
+def test_folded_norm_width_not_a_multiple_of_256(cuda_dev, n_blocks):
+    """d = 384: the residual GEMMs' last 256-column tile holds one valid half,
+    whose per-row sums of squares must count as zero in the folded norm."""
+    wl = wlmod.Workload("w384", 2, 4, 6, 8, 384, 3, 128, 1536, n_blocks, 0, 16, True)
+    ws_ = [wlmod.block_weights(wl, l, cuda_dev) for l in range(n_blocks)]
+    blocks = [h3b.Block.from_dict(w) for w in ws_]
+    dm = h3b.dims_of(wl)
+    x0 = wlmod.initial_tokens(wl, cuda_dev)
+    x = x0.clone()
+    h3b.stack_forward(dm, blocks, x, h3b.workspace(dm))
+    torch.cuda.synchronize()
+    assert h3b.device_error() == 0
+    ref = oracle.stack_forward(np64(x0), [host_weights(w) for w in ws_], wl)
+    check_bf16(np64(x0), np64(x), ref)
+
+
 @pytest.mark.parametrize("reuse,core_reuse,per_step", [(2, 1, True), (1, 3, True), (3, 1, False)])
 def test_denoise_with_condition_rows_and_modulation_vs_oracle(cuda_dev, reuse, core_reuse, per_step):
     wl = TINY.with_(n_blocks=4, depth_scaled_init=True, seed=14)
