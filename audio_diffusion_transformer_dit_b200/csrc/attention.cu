@@ -23,8 +23,9 @@
 // [-1/2, 1/2], p a degree-3 polynomial fitted to 2^f on that interval by
 // iteratively reweighted least squares on relative error (max relative
 // error 7.5e-5, below the bf16 rounding of P).  Keys past S in the last tile
-// are masked to zero probability (MUFU path only on that tile); query rows
-// past S are computed on zero-filled rows and not stored.
+// get score -inf before the row max, so one code path serves every tile and
+// their probability is exp2(-inf) = 0; query rows past S are computed on
+// zero-filled rows and not stored.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -106,24 +107,18 @@ __device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
 
 // Probabilities of keys [64h, 64h+64) of one row, in place: pair i (keys 2i,
 // 2i+1) reads r[2i], r[2i+1] and leaves its bf16 pair in r[i], a slot already
-// consumed.  Partial row sums go to acc.  LAST: keys >= valid get 0.
-template <bool LAST, int HALF>
-__device__ __forceinline__ void softmax_half(uint32_t (&r)[BKV], uint64_t c2, uint64_t nm2, int valid,
-                                             uint64_t (&acc)[4]) {
+// consumed.  Partial row sums go to acc.  Keys past S hold -inf scores here
+// (masked before the row max), so their exp2 is 0 on either pipe.
+template <int HALF>
+__device__ __forceinline__ void softmax_half(uint32_t (&r)[BKV], uint64_t c2, uint64_t nm2, uint64_t (&acc)[4]) {
 #pragma unroll
   for (int i = 32 * HALF; i < 32 * HALF + 32; ++i) {
     const uint64_t x = f2_fma(f2_pack(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])), c2, nm2);
     uint64_t p;
-    if (!LAST && (i % 8) >= 8 - POLY_OF_8) {
+    if ((i % 8) >= 8 - POLY_OF_8)
       p = ex2_poly2(x);
-    } else {
-      float p0 = ex2_mufu(f2_lo(x)), p1 = ex2_mufu(f2_hi(x));
-      if (LAST) {
-        if (2 * i >= valid) p0 = 0.f;
-        if (2 * i + 1 >= valid) p1 = 0.f;
-      }
-      p = f2_pack(p0, p1);
-    }
+    else
+      p = f2_pack(ex2_mufu(f2_lo(x)), ex2_mufu(f2_hi(x)));
     acc[i & 3] = f2_add(acc[i & 3], p);
     r[i] = cvt_bf16x2(f2_lo(p), f2_hi(p));
   }
@@ -325,17 +320,16 @@ __global__ void __launch_bounds__(THREADS, 1)
       tmem_ld32(sc + 64, *reinterpret_cast<uint32_t(*)[32]>(&r[64]));
       tmem_ld32(sc + 96, *reinterpret_cast<uint32_t(*)[32]>(&r[96]));
       tmem_ld_wait();
-      float mx0 = -INFINITY, mx1 = -INFINITY;
-      if (valid >= BKV) {
-#pragma unroll
-        for (int i = 0; i < BKV; i += 4) {
-          mx0 = max3(mx0, __uint_as_float(r[i]), __uint_as_float(r[i + 1]));
-          mx1 = max3(mx1, __uint_as_float(r[i + 2]), __uint_as_float(r[i + 3]));
-        }
-      } else {
+      if (valid < BKV) {  // last tile of a ragged S: keys past S get score -inf
 #pragma unroll
         for (int i = 0; i < BKV; ++i)
-          if (i < valid) mx0 = fmaxf(mx0, __uint_as_float(r[i]));
+          if (i >= valid) r[i] = 0xff800000u;
+      }
+      float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < BKV; i += 4) {
+        mx0 = max3(mx0, __uint_as_float(r[i]), __uint_as_float(r[i + 1]));
+        mx1 = max3(mx1, __uint_as_float(r[i + 2]), __uint_as_float(r[i + 3]));
       }
       const float m_new = fmaxf(mx0, mx1) * c;
       float alpha = 1.f;
@@ -362,19 +356,13 @@ __global__ void __launch_bounds__(THREADS, 1)
       // P of keys [0,64) -> TMEM columns [0,32), published; then keys [64,128) -> [32,64)
       const uint64_t c2 = f2_pack(c, c), nm2 = f2_pack(-m_use, -m_use);
       uint64_t acc[4] = {0, 0, 0, 0};
-      if (valid >= BKV)
-        softmax_half<false, 0>(r, c2, nm2, valid, acc);
-      else
-        softmax_half<true, 0>(r, c2, nm2, valid, acc);
+      softmax_half<0>(r, c2, nm2, acc);
       tmem_st32(sc + 0, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full + 16 * t);
-      if (valid >= BKV)
-        softmax_half<false, 1>(r, c2, nm2, valid, acc);
-      else
-        softmax_half<true, 1>(r, c2, nm2, valid, acc);
+      softmax_half<1>(r, c2, nm2, acc);
       tmem_st32(sc + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
       const uint64_t sum2 = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
       l = l * alpha + (f2_lo(sum2) + f2_hi(sum2));

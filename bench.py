@@ -793,12 +793,15 @@ def kernel_sweep(args):
     ]
     only = set(args.sweep_only.split(",")) if args.sweep_only else None
     # contractions, timed alone: the INT8 and BF16 FC1 GEMMs (GELU epilogue;
-    # INT8 also writes the per-row max) and the attention of both d = 5120
-    # workloads; built only when selected (they hold ~1-3 GB)
+    # INT8 also writes the per-row max), the FC2 and O-projection GEMMs
+    # (fp32 residual epilogue) and the attention of the d = 3072 block and
+    # both d = 5120 workloads; built only when selected (they hold ~1-3 GB)
     tensor_cases = {
         "gemm_fc1_int8": (INT8_WORKLOAD, "int8"), "gemm_fc1_bf16": (DEFAULT_WORKLOAD, "bf16"),
         "gemm_fc2_bf16": (DEFAULT_WORKLOAD, "bf16"),
-        "attention_s6528": (DEFAULT_WORKLOAD, None), "attention_s20640": (INT8_WORKLOAD, None),
+        "gemm_o_bf16_d3072": ("block_d3072_s6400", "bf16"), "gemm_o_bf16_d5120": (DEFAULT_WORKLOAD, "bf16"),
+        "attention_s6400": ("block_d3072_s6400", None), "attention_s6528": (DEFAULT_WORKLOAD, None),
+        "attention_s20640": (INT8_WORKLOAD, None),
     }
     for name, (wname, kind) in tensor_cases.items():
         if only is None or name not in only:
@@ -812,6 +815,14 @@ def kernel_sweep(args):
             fn = lambda A=A, B=B, C=C: h3b.gemm(A, B, h3b.EPI_RESID, C)  # noqa: E731
             work = 2.0 * Sx * fx * dx
             shape = f"bf16 [{Sx},{fx}] x [{dx},{fx}]^T -> fp32 residual [{Sx},{dx}]"
+        elif name.startswith("gemm_o"):  # x [S, d] fp32 += o [S, d] Wo [d, d]^T, tail split along K
+            A = W.normal_tensor((Sx, dx), 21, dev, dtype=torch.bfloat16)
+            B = W.normal_tensor((dx, dx), 22, dev, std=0.02, dtype=torch.bfloat16)
+            C = W.normal_tensor((Sx, dx), 23, dev)
+            scr = torch.empty(Sx * dx, dtype=torch.float32, device=dev)
+            fn = lambda A=A, B=B, C=C, scr=scr: h3b.gemm(A, B, h3b.EPI_RESID, C, scratch=scr)  # noqa: E731
+            work = 2.0 * Sx * dx * dx
+            shape = f"bf16 [{Sx},{dx}] x [{dx},{dx}]^T -> fp32 residual [{Sx},{dx}]"
         elif name.startswith("gemm"):
             if kind == "int8":
                 A = W.int8_tensor((Sx, dx), 21, dev)
