@@ -107,6 +107,15 @@ PINS = {
     "stack_forward_ex": "hand-computed tokens with a toy block whose merged and unmerged forms differ: where the "
                         "pre-merge tokens are taken, which merged input the delta subtracts, the window's blocks",
     "linear": "pure-Python dot products",
+    "stack_forward": "scalar toy blocks: the blocks inside the reduction window see the merged rows, the others "
+                     "the full rows, in order; identity blocks give unmerge(merge(x))",
+    "stack_forward_cond": "merge window with condition rows equals the explicit composition of pinned parts "
+                          "(block_forward_cond, token_merge, token_unmerge[_delta]); condition rows pass the merge",
+    "flow_step": "zero velocity is the identity; x + (s1 - s0) v closed form",
+    "dequantize_rows/dequant_weights": "|dequantised - input| <= s/2 per element; the W8A8 block is close to "
+                                       "block_forward on the dequantised weights",
+    "rope_sections/token_positions": "section widths D/4, 3D/8, 3D/8; hand-computed angles of a given (f, r, c), of "
+                                     "an audio token and of a merged token at column 2c'+0.5",
     "block_forward_cond": "identity modulation without condition rows equals block_forward; zero gates give the "
                           "identity; scale = -1 makes every normed row equal to the shift (closed form without "
                           "RoPE); condition rows are permutation-equivariant among themselves (no rotation); a "
