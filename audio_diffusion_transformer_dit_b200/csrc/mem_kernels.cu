@@ -393,24 +393,43 @@ __global__ void __launch_bounds__(kThreads) k_quant_rows(const uint4* __restrict
   if (threadIdx.x == 0) scale[row] = s;
 }
 
-// Known row maxima: purely elementwise.  Grid (chunks, rows); each thread
-// turns 16 bf16 (two 16-byte loads) into 16 codes (one 16-byte store).
-__global__ void k_quant_absmax(const uint4* __restrict__ a, const float* __restrict__ absmax, int k16,
-                               int8_t* __restrict__ q, float* __restrict__ scale) {
+// Known row maxima: purely elementwise.  One CTA per row; thread t takes the
+// 16-element chunks t, t + 256, ... (CPT of them), issues all their loads
+// (two 16 bytes each) before the row scale's two divisions and before it
+// converts any, and writes 16 codes per chunk in one 16-byte store.  Against
+// a grid of one 16-element chunk per thread: 269 -> 237 us for the
+// 20640 x 20480 FC2 input (0.72 -> 0.82 of the measured copy bandwidth).
+template <int CPT>
+__global__ void __launch_bounds__(kThreads) k_quant_absmax(const uint4* __restrict__ a,
+                                                           const float* __restrict__ absmax, int k16,
+                                                           int8_t* __restrict__ q, float* __restrict__ scale) {
   pdl_trigger();
   pdl_wait();
-  const int row = blockIdx.y;
-  const float s = absmax[row] / 127.0f, rs = 1.0f / s;
+  const int row = blockIdx.x;
   const uint4* ar = a + static_cast<size_t>(row) * k16 * 2;
   uint4* qr = reinterpret_cast<uint4*>(q) + static_cast<size_t>(row) * k16;
-  for (int c = blockIdx.x * blockDim.x + threadIdx.x; c < k16; c += gridDim.x * blockDim.x) {
-    float f0[8], f1[8];
-    bf16x8_to_f32(__ldcs(ar + 2 * c), f0);
-    bf16x8_to_f32(__ldcs(ar + 2 * c + 1), f1);
-    const uint2 lo = quant8(f0, s, rs), hi = quant8(f1, s, rs);
-    qr[c] = make_uint4(lo.x, lo.y, hi.x, hi.y);
+  uint4 v[2 * CPT];
+#pragma unroll
+  for (int i = 0; i < CPT; ++i) {
+    const int c = threadIdx.x + i * kThreads;
+    if (c < k16) {
+      v[2 * i] = __ldcs(ar + 2 * c);
+      v[2 * i + 1] = __ldcs(ar + 2 * c + 1);
+    }
   }
-  if (blockIdx.x == 0 && threadIdx.x == 0) scale[row] = s;
+  const float s = absmax[row] / 127.0f, rs = 1.0f / s;
+#pragma unroll
+  for (int i = 0; i < CPT; ++i) {
+    const int c = threadIdx.x + i * kThreads;
+    if (c < k16) {
+      float f0[8], f1[8];
+      bf16x8_to_f32(v[2 * i], f0);
+      bf16x8_to_f32(v[2 * i + 1], f1);
+      const uint2 lo = quant8(f0, s, rs), hi = quant8(f1, s, rs);
+      qr[c] = make_uint4(lo.x, lo.y, hi.x, hi.y);
+    }
+  }
+  if (threadIdx.x == 0) scale[row] = s;
 }
 
 // Same with 8 elements per thread (k a multiple of 8 but not of 16).
@@ -555,16 +574,28 @@ cudaError_t launch_quant_rows(const Ctx& c, const void* a, int rows, int k, int8
 cudaError_t launch_quant_absmax(const Ctx& c, const void* a, const float* absmax, int rows, int k, int8_t* q,
                                 float* s) {
   if (rows == 0 || k == 0) return cudaSuccess;
-  const int per_thread = (k % 16 == 0) ? 16 : 8;
-  const int chunks = k / per_thread;
+  const uint4* a4 = reinterpret_cast<const uint4*>(a);
+  const int k16 = k / 16, cpt = (k16 + kThreads - 1) / kThreads;
+  if (k % 16 == 0 && cpt <= 8) {  // k <= 32768: one CTA per row
+    cudaError_t e = cudaErrorInvalidValue;
+#define H3B_QA_CASE(V) \
+  case V: e = launch_pdl(c.stream, k_quant_absmax<V>, dim3(rows), dim3(kThreads), 0, 1u, a4, absmax, k16, q, s); break;
+    switch (cpt) {
+      H3B_QA_CASE(1) H3B_QA_CASE(2) H3B_QA_CASE(3) H3B_QA_CASE(4) H3B_QA_CASE(5) H3B_QA_CASE(6)
+      H3B_QA_CASE(7) H3B_QA_CASE(8)
+    }
+#undef H3B_QA_CASE
+    return e != cudaSuccess ? e : cudaGetLastError();
+  }
+  // k a multiple of 8 only, or beyond 32768: 8 elements per thread, grid (chunks, rows)
+  const int chunks = k / 8;
   const int bx = (chunks + kThreads - 1) / kThreads;
   for (int r0 = 0; r0 < rows; r0 += 65535) {  // grid.y limit
     const int nr = rows - r0 < 65535 ? rows - r0 : 65535;
     const dim3 grid(bx, nr);
-    const uint4* a4 = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(a) + static_cast<size_t>(r0) * k);
-    const cudaError_t e =
-        launch_pdl(c.stream, per_thread == 16 ? k_quant_absmax : k_quant_absmax8, grid, dim3(kThreads), 0, 1u, a4,
-                   absmax + r0, chunks, q + static_cast<size_t>(r0) * k, s + r0);
+    const uint4* ar = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(a) + static_cast<size_t>(r0) * k);
+    const cudaError_t e = launch_pdl(c.stream, k_quant_absmax8, grid, dim3(kThreads), 0, 1u, ar, absmax + r0, chunks,
+                                     q + static_cast<size_t>(r0) * k, s + r0);
     if (e != cudaSuccess) return e;
   }
   return cudaGetLastError();
