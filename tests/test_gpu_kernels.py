@@ -107,7 +107,7 @@ def test_rmsnorm_bf16(cuda_dev, rows, d):
     assert np.all(np.abs(np64(u) - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-30)
 
 
-@pytest.mark.parametrize("rows,d", [(37, 256), (300, 5120), (10000, 1024), (5, 8192)])
+@pytest.mark.parametrize("rows,d", [(37, 256), (300, 5120), (7, 4096), (7, 6144), (10000, 1024), (5, 8192)])
 def test_rmsnorm_int8(cuda_dev, rows, d):
     x = wlmod.normal_tensor((rows, d), 8, cuda_dev)
     g = torch.ones(d, device=cuda_dev)
