@@ -126,7 +126,13 @@ int h3b_block_forward(const h3b_dims* dims, const h3b_block_weights* w, float* x
  * merge_first >= 0, the sequence is merged (h3b_token_merge) before block
  * merge_first and unmerged after block merge_last (inclusive, 0-indexed)
  * [control].  ws: at least h3b_workspace_bytes(dims, dtype, merge_first >= 0).
- * All blocks must share one dtype. */
+ * All blocks must share one dtype.  Between consecutive bf16 blocks outside
+ * the reduction window's edges, RMSNorm is folded into the neighbouring
+ * GEMMs (the residual epilogue writes bf16(x * g) and per-row sums of x^2,
+ * the next GEMM scales its rows by 1/sqrt(mean x^2 + eps)) [fusion]; the
+ * result then equals a sequence of h3b_block_forward calls within rounding
+ * (the bf16 rounding falls on x * g instead of on the normalised row), not
+ * bit for bit.  INT8 stacks match the block sequence bit for bit. */
 int h3b_stack_forward(const h3b_dims* dims, const h3b_block_weights* blocks, int n_blocks,
                       int merge_first, int merge_last, float* x,
                       void* ws, size_t ws_bytes, void* stream);
@@ -147,8 +153,8 @@ int h3b_denoise(const h3b_dims* dims, const h3b_block_weights* blocks, int n_blo
  * unmerge, core residual reuse, fixed condition rows and timestep
  * modulation.  The siami.tw article's control table names the core-reuse knob
  * (--core-reuse 1/4/6, exclusive with whole-velocity reuse) but not its
- * arithmetic, its file list names "0.999 condition augmentation + fixed
- * condition rows" without a form, and no page gives an unmerge rule; the
+ * arithmetic, its file list names a 0.999 condition augmentation and fixed
+ * condition rows without a form, and no page gives an unmerge rule; the
  * forms below are the plainest readings.  Zero-initialise the struct: every
  * field's zero (with merge_first = core_first = -1) is "off".
  *   merge_first, merge_last: token-reduction window (inclusive, 0-indexed),

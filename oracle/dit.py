@@ -74,8 +74,9 @@ READINGS = {
                   "class, u = RMSNorm(x)*(1+scale)+shift before the QKV and FC1 GEMMs and x += gate*update "
                   "after the O-proj and FC2 GEMMs; class 0 = generated (video + audio) rows, class 1 = "
                   "condition rows",
-    "condition_rows": "fixed condition rows (siami.tw file list: 0.999 condition augmentation + fixed condition "
-                      "rows in native DiT): C rows appended after the audio tokens, given already augmented; "
+    "condition_rows": "fixed condition rows (the siami.tw file list names a 0.999 condition augmentation and "
+                      "fixed condition rows inside the DiT, without a form): C rows appended after the audio "
+                      "tokens, given already augmented; "
                       "they take part in every block (joint attention) with no rotary embedding, every "
                       "evaluation starts them from the given values, and the Euler update leaves them out",
 }

@@ -176,6 +176,29 @@ def test_stack_equals_block_sequence(cuda_dev):
     assert rel_l2(x - x0, y - x0) <= 1e-2
 
 
+def test_int8_stack_equals_block_sequence_bitexact(cuda_dev):
+    """INT8 blocks normalise (and quantise) in their own pass inside a stack as
+    in a lone block call, so the stack with a reduction window equals the
+    explicit merge + block calls + unmerge bit for bit."""
+    wl = TINY.with_(n_blocks=4, depth_scaled_init=True, seed=16, dtype=h3b.INT8)
+    ws_ = [wlmod.block_weights(wl, l, cuda_dev) for l in range(4)]
+    blocks = [h3b.Block.quantized(w) for w in ws_]
+    dm = h3b.dims_of(wl)
+    x = wlmod.initial_tokens(wl, cuda_dev)
+    y = x.clone()
+    ws = h3b.workspace(dm, h3b.INT8, True)
+    h3b.stack_forward(dm, blocks, x, ws, 1, 2)
+    h3b.block_forward(dm, blocks[0], y, ws)
+    ym = torch.empty((h3b.seq_len(dm, True), wl.d), device=cuda_dev)
+    h3b.token_merge(dm, y, ym)
+    for l in (1, 2):
+        h3b.block_forward(dm, blocks[l], ym, ws, merged=True)
+    h3b.token_unmerge(dm, ym, y)
+    h3b.block_forward(dm, blocks[3], y, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(x, y)
+
+
 @pytest.mark.slow
 def test_stack8_full_size_equals_blocks(cuda_dev):
     """The benched 8-block stack against the same blocks called one by one
