@@ -259,6 +259,7 @@ GemmArgs gemm_args(int M, int N, int K, void* C, const float* sa, const float* s
   a.ss_out = nullptr;
   a.ss_parts = norm_parts(dm);
   a.row_scale = nullptr;
+  a.partial_elems = 0;
   return a;
 }
 
@@ -817,6 +818,16 @@ int h3b_selftest_wait_timeout(int timeout_us, void* stream) {
   H3B_CU(KID_MEMSET, launch_selftest_wait(c, 1000ull * static_cast<unsigned long long>(timeout_us)));
   return H3B_OK;
 }
+
+int h3b_selftest_index_check(long long i, long long n, void* stream) {
+  if (n <= 0) return H3B_ERR_DIMS;
+  Ctx c;
+  H3B_TRY(device_ctx(static_cast<cudaStream_t>(stream), &c));
+  H3B_CU(KID_MEMSET, launch_selftest_index(c, i, n));
+  return H3B_OK;
+}
+
+int h3b_index_checked(void) { return H3B_CHECK; }
 
 int h3b_device_error(void* stream) {
   Ctx c;

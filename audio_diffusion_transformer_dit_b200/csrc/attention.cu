@@ -54,6 +54,7 @@ struct AttnArgs {
   int n_full;      // work items (pair, head) run whole; the rest are split along keys
   int ks;          // key-range parts per split item
   float* partial;  // split parts: O [256][D] fp32, then m [256], l [256] per part
+  size_t partial_elems;  // floats in partial (index checks)
 };
 
 template <int D>
@@ -378,19 +379,24 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc_fence_after();
         float* base = a.partial + static_cast<size_t>(slot) * slot_floats<D>();
         const int prow = t * BQ + row;
+        const long long b0 = static_cast<long long>(slot) * slot_floats<D>(), pe = static_cast<long long>(a.partial_elems);
 #pragma unroll 1
         for (int cc = 0; cc < D / 32; ++cc) {
           uint32_t o[32];
           tmem_ld32(oc + cc * 32, o);
           tmem_ld_wait();
           float4* dst = reinterpret_cast<float4*>(base + static_cast<size_t>(prow) * D + cc * 32);
+          if (idx_ok(err, b0 + static_cast<long long>(prow) * D + cc * 32, 32, pe, 31)) {
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            dst[i] = make_float4(__uint_as_float(o[4 * i]), __uint_as_float(o[4 * i + 1]),
-                                 __uint_as_float(o[4 * i + 2]), __uint_as_float(o[4 * i + 3]));
+            for (int i = 0; i < 8; ++i)
+              dst[i] = make_float4(__uint_as_float(o[4 * i]), __uint_as_float(o[4 * i + 1]),
+                                   __uint_as_float(o[4 * i + 2]), __uint_as_float(o[4 * i + 3]));
+          }
         }
-        base[256 * D + prow] = m_use;
-        base[256 * D + 256 + prow] = l;
+        if (idx_ok(err, b0 + 256 * D + prow, 257, pe, 31)) {  // m at +prow, l at +256+prow
+          base[256 * D + prow] = m_use;
+          base[256 * D + 256 + prow] = l;
+        }
       } else if (__all_sync(0xffffffffu, ok)) {
         tc_fence_after();
         const float inv = 1.f / l;
@@ -421,7 +427,8 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
         for (int k = 0; k < 32 / RPI; ++k) {
           const int r = k * RPI + lane / UNITS;
-          if (rbase + r < S)
+          if (rbase + r < S && idx_ok(err, static_cast<long long>(rbase + r) * d_model + h * D + u * 8, 8,
+                                      static_cast<long long>(S) * d_model, 30))
             *reinterpret_cast<uint4*>(a.out + static_cast<size_t>(rbase + r) * d_model + h * D + u * 8) =
                 *reinterpret_cast<const uint4*>(stg + r * (D * 2) + ((u ^ (r % UNITS)) << 4));
         }
@@ -448,6 +455,11 @@ __global__ void __launch_bounds__(D) k_attn_combine(const AttnArgs a) {
   const int item = a.n_full + ti;
   const int grow = (item % a.pairs) * 2 * BQ + r, h = item / a.pairs;
   if (grow >= a.S) return;
+  if (!idx_ok(a.err, static_cast<long long>(ti) * a.ks * slot_floats<D>(),
+              static_cast<long long>(a.ks) * slot_floats<D>(), static_cast<long long>(a.partial_elems), 32) ||
+      !idx_ok(a.err, static_cast<long long>(grow) * (a.n_heads * D) + h * D + col, 1,
+              static_cast<long long>(a.S) * a.n_heads * D, 33))
+    return;
   const float* base = a.partial + static_cast<size_t>(ti) * a.ks * slot_floats<D>();
   float M = -INFINITY;
   for (int c = 0; c < a.ks; ++c) M = fmaxf(M, base[static_cast<size_t>(c) * slot_floats<D>() + 256 * D + r]);
@@ -507,6 +519,7 @@ cudaError_t launch_attention(const Ctx& c, const void* qkv, int S, int n_heads, 
   a.n_full = items;
   a.ks = 1;
   a.partial = nullptr;
+  a.partial_elems = 0;
   // Items left after the last full wave, when they fill at most half of it,
   // are cut along the keys over the idle SMs and merged by a second kernel.
   const int tail = items % c.num_sms;
@@ -520,6 +533,7 @@ cudaError_t launch_attention(const Ctx& c, const void* qkv, int S, int n_heads, 
       a.n_full = items - tail;
       a.ks = ks;
       a.partial = scratch;
+      a.partial_elems = scratch_bytes / sizeof(float);
     }
   }
   const int grid = a.n_full + (items - a.n_full) * a.ks;

@@ -20,7 +20,37 @@ namespace h3b {
 constexpr unsigned long long WAIT_TIMEOUT_NS = 2000000000ull;  // 2 s per wait
 
 // Device error word codes: (kernel << 8) | site.
-enum ErrKernel { EK_GEMM = 1, EK_ATTN = 2, EK_SELFTEST = 3 };
+enum ErrKernel { EK_GEMM = 1, EK_ATTN = 2, EK_SELFTEST = 3, EK_INDEX = 4 };
+
+// Index checks.  Built with -DH3B_CHECK=1 (libh3b_check.so), every
+// hand-indexed global load and store first checks the element range it
+// touches, [i, i + width), against the extent of its buffer as the kernel's
+// own shape arguments define it.  Outside it, the thread records
+// (EK_INDEX << 8) | site in the device error word (the first record wins)
+// and skips the access: no trap and no fault, the context stays usable.  In
+// the default build idx_ok is the constant true and compiles away.  Sites:
+//   1-2 Euler step; 3-4 token merge; 5 unmerge; 6-7 delta unmerge; 8 RoPE
+//   table; 9 GELU; 10-12 RMSNorm; 13-14 row quantisation; 15-17 known-max
+//   quantisation; 20-25 GEMM epilogues; 26-28 split-K fix-up; 29 row factor
+//   of the folded norm; 30-31 attention epilogue; 32-33 attention combine.
+#ifndef H3B_CHECK
+#define H3B_CHECK 0
+#endif
+__device__ __forceinline__ bool idx_ok(int* err, long long i, long long width, long long n, int site) {
+#if H3B_CHECK
+  if (i < 0 || i + width > n) {
+    atomicCAS(err, 0, (EK_INDEX << 8) | site);
+    return false;
+  }
+#else
+  (void)err;
+  (void)i;
+  (void)width;
+  (void)n;
+  (void)site;
+#endif
+  return true;
+}
 
 struct Launch {
   cudaStream_t stream;

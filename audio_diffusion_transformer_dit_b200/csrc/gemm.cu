@@ -104,7 +104,10 @@ __device__ __forceinline__ void load_resid_rows(const GemmArgs& p, int row0, int
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const int m = row0 + 4 * i + (lane >> 3);
-    dst[i] = m < p.M ? *reinterpret_cast<const float4*>(C + static_cast<size_t>(m) * p.N) : make_float4(0.f, 0.f, 0.f, 0.f);
+    dst[i] = m < p.M && idx_ok(p.err, static_cast<long long>(m) * p.N + n + 4 * (lane & 7), 4,
+                               static_cast<long long>(p.M) * p.N, 20)
+                 ? *reinterpret_cast<const float4*>(C + static_cast<size_t>(m) * p.N)
+                 : make_float4(0.f, 0.f, 0.f, 0.f);
   }
 }
 
@@ -143,7 +146,9 @@ __device__ __forceinline__ void store_row_squares(const GemmArgs& p, int row0, i
     v += __shfl_xor_sync(0xffffffffu, v, 2);
     v += __shfl_xor_sync(0xffffffffu, v, 4);
     const int m = row0 + 4 * i + (lane >> 3);
-    if ((lane & 7) == 0 && m < p.M) p.ss_out[static_cast<size_t>(m) * p.ss_parts + part] = v;
+    if ((lane & 7) == 0 && m < p.M &&
+        idx_ok(p.err, static_cast<long long>(m) * p.ss_parts + part, 1, static_cast<long long>(p.M) * p.ss_parts, 22))
+      p.ss_out[static_cast<size_t>(m) * p.ss_parts + part] = v;
   }
 }
 
@@ -164,7 +169,7 @@ __device__ __forceinline__ void resid_rows(const GemmArgs& p, const float* stg, 
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const int m = row0 + 4 * i + (lane >> 3);
-    if (m < p.M) {
+    if (m < p.M && idx_ok(p.err, static_cast<long long>(m) * p.N + col, 4, static_cast<long long>(p.M) * p.N, 21)) {
       const float4 v = stage_get(stg, lane, i);
       const float4 g = m >= p.gate_split ? g1 : g0;
       float4 a = res[i];
@@ -183,11 +188,15 @@ __device__ __forceinline__ void resid_rows(const GemmArgs& p, const float* stg, 
 }
 
 // Staged chunk -> rows trow0 .. trow0+32 of a tile-shaped fp32 partial (row stride BN).
-__device__ __forceinline__ void partial_rows(float* part, const float* stg, int trow0, int ccol, int lane) {
+__device__ __forceinline__ void partial_rows(const GemmArgs& p, float* part, const float* stg, int trow0, int ccol,
+                                             int lane) {
   float* dst = part + ccol + 4 * (lane & 7);
 #pragma unroll
-  for (int i = 0; i < 8; ++i)
-    *reinterpret_cast<float4*>(dst + static_cast<size_t>(trow0 + 4 * i + (lane >> 3)) * BN) = stage_get(stg, lane, i);
+  for (int i = 0; i < 8; ++i) {
+    const long long off = static_cast<long long>(trow0 + 4 * i + (lane >> 3)) * BN;
+    if (idx_ok(p.err, (dst - p.partial) + off, 4, static_cast<long long>(p.partial_elems), 24))
+      *reinterpret_cast<float4*>(dst + off) = stage_get(stg, lane, i);
+  }
 }
 
 // One chunk of a residual tile (whole tile or K-part), all lanes of the warp.
@@ -199,7 +208,7 @@ __device__ __forceinline__ void resid_chunk(const GemmArgs& p, float* stg, int l
   chunk_values<INT8>(p, row0 + lane, n, r, v);
   stage_put(stg, lane, v);
   if (part) {
-    partial_rows(part, stg, trow0, ccol, lane);
+    partial_rows(p, part, stg, trow0, ccol, lane);
     return;
   }
   float4 cur[8];
@@ -214,6 +223,7 @@ template <bool INT8, int EPI>
 __device__ __forceinline__ void epilogue_chunk(const GemmArgs& p, int m, int n, const uint32_t (&r)[32],
                                                float& row_amax, float rs) {
   const size_t off = static_cast<size_t>(m) * p.N + n;
+  if (!idx_ok(p.err, n, 32, p.N, 23) || !idx_ok(p.err, off, 32, static_cast<long long>(p.M) * p.N, 23)) return;
   if (EPI == H3B_EPI_I32) {
     int4* c = reinterpret_cast<int4*>(static_cast<int*>(p.C) + off);
 #pragma unroll
@@ -250,8 +260,10 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& p, int m, int n, 
     return;
   }
   if (EPI == H3B_EPI_QKV_ROPE) {
-    if (n < 2 * p.d && m < p.rope_rows) {  // Q or K column block: rotate its 16 interleaved pairs
-      const int j0 = (n % p.head_dim) >> 1;
+    const int j0 = (n % p.head_dim) >> 1;
+    if (n < 2 * p.d && m < p.rope_rows &&
+        idx_ok(p.err, static_cast<long long>(m) * (p.head_dim >> 1) + j0, 16,
+               static_cast<long long>(p.rope_rows) * (p.head_dim >> 1), 23)) {  // Q or K block: rotate 16 pairs
       const float4* t4 = reinterpret_cast<const float4*>(p.rope + static_cast<size_t>(m) * (p.head_dim >> 1) + j0);
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
@@ -448,7 +460,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
       }
       if (EPI == H3B_EPI_RESID && p.xb && !part_dst) store_row_squares(p, m - lane, lane, 2 * nb + ch, ssq);
-      if (INT8 && EPI == H3B_EPI_GELU && m < p.M)
+      if (INT8 && EPI == H3B_EPI_GELU && m < p.M && idx_ok(p.err, m, 1, p.M, 25))
         atomicMax(reinterpret_cast<int*>(p.row_absmax) + m, __float_as_int(row_amax));
       tc_fence_before();
       __syncwarp();
@@ -477,7 +489,7 @@ __global__ void __launch_bounds__(BN) k_splitk_add(float* __restrict__ C, const 
                                                    int group_n, const float* __restrict__ gate, int gate_split,
                                                    int gate_stride, __nv_bfloat16* __restrict__ xb,
                                                    const float* __restrict__ xb_gain, float* __restrict__ ss_out,
-                                                   int ss_parts) {
+                                                   int ss_parts, int* err, size_t partial_elems) {
   pdl_trigger();
   pdl_wait();
   __shared__ float red[BN / 32];
@@ -487,8 +499,11 @@ __global__ void __launch_bounds__(BN) k_splitk_add(float* __restrict__ C, const 
   const int m = mb * TM + r, n = nb * BN + col;
   if (m >= M) return;  // the whole CTA: m depends on the block only
   float sq = 0.f;
-  if (n < N) {
-    const float* src = partial + static_cast<size_t>(i) * split * (TM * BN) + r * BN + col;
+  const long long src0 = static_cast<long long>(i) * split * (TM * BN) + r * BN + col;
+  if (n < N && idx_ok(err, src0, static_cast<long long>(split - 1) * (TM * BN) + 1,
+                      static_cast<long long>(partial_elems), 26) &&
+      idx_ok(err, static_cast<long long>(m) * N + n, 1, static_cast<long long>(M) * N, 27)) {
+    const float* src = partial + src0;
     float acc = 0.f;
     for (int q = 0; q < split; ++q) acc += src[static_cast<size_t>(q) * (TM * BN)];
     float c = C[static_cast<size_t>(m) * N + n];
@@ -504,7 +519,9 @@ __global__ void __launch_bounds__(BN) k_splitk_add(float* __restrict__ C, const 
   for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
   if ((col & 31) == 0) red[col >> 5] = sq;
   __syncthreads();
-  if (col < 2) {  // warps 0-3 hold columns 0-127 of the tile, warps 4-7 columns 128-255
+  if (col < 2 && idx_ok(err, static_cast<long long>(m) * ss_parts + 2 * nb + col, 1,
+                         static_cast<long long>(M) * ss_parts, 28)) {
+    // warps 0-3 hold columns 0-127 of the tile, warps 4-7 columns 128-255
     const float h = red[4 * col] + red[4 * col + 1] + red[4 * col + 2] + red[4 * col + 3];
     ss_out[static_cast<size_t>(m) * ss_parts + 2 * nb + col] = h;
   }
@@ -764,7 +781,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
       }
       if (EPI == H3B_EPI_RESID && p.xb && !part_dst) store_row_squares(p, m - lane, lane, 2 * nb + ch, ssq);
-      if (INT8 && EPI == H3B_EPI_GELU && m < p.M)
+      if (INT8 && EPI == H3B_EPI_GELU && m < p.M && idx_ok(p.err, m, 1, p.M, 25))
         atomicMax(reinterpret_cast<int*>(p.row_absmax) + m, __float_as_int(row_amax));
       tc_fence_before();
       __syncwarp();
@@ -819,11 +836,12 @@ GemmKernel pick(int epi) {
 
 // One thread per row: the row's partial sums of squares in order -> factor.
 __global__ void k_norm_scale(const float* __restrict__ ss, int rows, int parts, int d, float eps,
-                             float* __restrict__ r) {
+                             float* __restrict__ r, int* err) {
   pdl_trigger();
   pdl_wait();
   const int m = blockIdx.x * blockDim.x + threadIdx.x;
   if (m >= rows) return;
+  if (!idx_ok(err, static_cast<long long>(m) * parts, parts, static_cast<long long>(rows) * parts, 29)) return;
   const float* q = ss + static_cast<size_t>(m) * parts;
   float s = 0.f;
   for (int i = 0; i < parts; ++i) s += q[i];
@@ -835,7 +853,7 @@ __global__ void k_norm_scale(const float* __restrict__ ss, int rows, int parts, 
 cudaError_t launch_norm_scale(const Ctx& c, const float* ss, int rows, int parts, int d, float eps, float* r) {
   if (rows == 0) return cudaSuccess;
   const cudaError_t e = launch_pdl(c.stream, k_norm_scale, dim3((rows + 127) / 128), dim3(128), 0, 1u, ss, rows,
-                                   parts, d, eps, r);
+                                   parts, d, eps, r, c.err);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -901,6 +919,7 @@ cudaError_t launch_gemm(const Ctx& c, const void* A, const void* B, int ab_int8,
   args.split = 1;
   args.full_tiles = tiles;
   args.partial = nullptr;
+  args.partial_elems = 0;
   // K steps (stages) of the kernel that runs: two atoms per stage for pairs
   const int ke = (pair ? pair_atoms(epi) : 1) * (KBYTES / eb);
   const int num_kb = (args.K + ke - 1) / ke;
@@ -914,6 +933,7 @@ cudaError_t launch_gemm(const Ctx& c, const void* A, const void* B, int ab_int8,
       args.split = split;
       args.full_tiles = tiles - rem;
       args.partial = scratch;
+      args.partial_elems = scratch_bytes / sizeof(float);
     }
   }
   e = launch_pdl(c.stream, kern, dim3(pair ? 2 * grid : grid), dim3(THREADS), smem, pair ? 2u : 1u, ta, tb, args);
@@ -924,12 +944,12 @@ cudaError_t launch_gemm(const Ctx& c, const void* A, const void* B, int ab_int8,
     e = launch_pdl(c.stream, k_splitk_add<BM2>, dim3(rem * BM2), dim3(BN), 0, 1u, static_cast<float*>(args.C),
                    static_cast<const float*>(args.partial), args.M, args.N, args.full_tiles, args.split, num_m, num_n,
                    args.group_n, args.gate, args.gate_split, args.gate_stride, args.xb, args.xb_gain, args.ss_out,
-                   args.ss_parts);
+                   args.ss_parts, args.err, args.partial_elems);
   else
     e = launch_pdl(c.stream, k_splitk_add<BM>, dim3(rem * BM), dim3(BN), 0, 1u, static_cast<float*>(args.C),
                    static_cast<const float*>(args.partial), args.M, args.N, args.full_tiles, args.split, num_m, num_n,
                    args.group_n, args.gate, args.gate_split, args.gate_stride, args.xb, args.xb_gain, args.ss_out,
-                   args.ss_parts);
+                   args.ss_parts, args.err, args.partial_elems);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

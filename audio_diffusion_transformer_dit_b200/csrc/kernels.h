@@ -119,6 +119,8 @@ struct GemmArgs {
   float* ss_out;
   int ss_parts;
   const float* row_scale;
+  // floats in the split-K partial buffer (set by launch_gemm; index checks)
+  size_t partial_elems;
 };
 // r[m] = 1 / sqrt(sum_q ss[m * parts + q] / d + eps), q in order (deterministic).
 cudaError_t launch_norm_scale(const Ctx& c, const float* ss, int rows, int parts, int d, float eps, float* r);
@@ -133,6 +135,7 @@ cudaError_t launch_attention(const Ctx& c, const void* qkv, int S, int n_heads, 
                              float* scratch = nullptr, size_t scratch_bytes = 0);
 cudaError_t launch_exp2_poly(const Ctx& c, const float* x, float* y, int n);
 cudaError_t launch_selftest_wait(const Ctx& c, unsigned long long timeout_ns);
+cudaError_t launch_selftest_index(const Ctx& c, long long i, long long n);
 
 // tensor-map encoding through the driver entry point (no libcuda link)
 bool encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, int elem_bytes, const void* base, uint64_t inner,

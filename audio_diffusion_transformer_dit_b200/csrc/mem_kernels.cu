@@ -110,7 +110,7 @@ __device__ __forceinline__ uint32_t quant4(float a, float b, float c, float d, f
 
 // ------------------------------------------------------------------ Euler step
 __global__ void k_flow(float* __restrict__ x, const float* __restrict__ v, float dt, size_t n,
-                       float* __restrict__ xc) {
+                       float* __restrict__ xc, int* err) {
   pdl_trigger();
   pdl_wait();
   const size_t n4 = n >> 2;
@@ -119,6 +119,7 @@ __global__ void k_flow(float* __restrict__ x, const float* __restrict__ v, float
   const float4* v4 = reinterpret_cast<const float4*>(v);
   float4* c4 = reinterpret_cast<float4*>(xc);
   for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4; i += stride) {
+    if (!idx_ok(err, 4 * i, 4, n, 1)) continue;
     float4 a = x4[i];
     const float4 b = __ldcs(v4 + i);
     a.x = fmaf(dt, b.x, a.x);
@@ -129,6 +130,7 @@ __global__ void k_flow(float* __restrict__ x, const float* __restrict__ v, float
     if (xc) c4[i] = a;
   }
   for (size_t i = (n4 << 2) + static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += stride) {
+    if (!idx_ok(err, i, 1, n, 2)) continue;
     const float a = fmaf(dt, v[i], x[i]);
     x[i] = a;
     if (xc) xc[i] = a;
@@ -139,15 +141,18 @@ __global__ void k_flow(float* __restrict__ x, const float* __restrict__ v, float
 // Video token (f, r, 2c'+k) is row 2*((f*H + r)*(W/2) + c') + k of the full
 // sequence, so merged row i averages full rows 2i and 2i+1; audio rows follow.
 __global__ void k_merge(const float4* __restrict__ x, float4* __restrict__ xm, float4* __restrict__ xm_copy,
-                        int half_video, int n_audio, int d4) {
+                        int half_video, int n_audio, int d4, int* err) {
   pdl_trigger();
   pdl_wait();
   const size_t total = static_cast<size_t>(half_video + n_audio) * d4;
+  const long long full = (2ll * half_video + n_audio) * d4;  // float4 units of x
   const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
   for (size_t e = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < total; e += stride) {
     const size_t row = e / d4, col = e - row * d4;
+    if (!idx_ok(err, e, 1, total, 4)) continue;
     float4 o;
     if (row < static_cast<size_t>(half_video)) {
+      if (!idx_ok(err, (2 * row) * d4 + col, d4 + 1, full, 3)) continue;  // rows 2 row and 2 row + 1
       const float4 a = __ldcs(x + (2 * row) * d4 + col);
       const float4 b = __ldcs(x + (2 * row + 1) * d4 + col);
       o.x = __fmul_rn(__fadd_rn(a.x, b.x), 0.5f);
@@ -155,6 +160,7 @@ __global__ void k_merge(const float4* __restrict__ x, float4* __restrict__ xm, f
       o.z = __fmul_rn(__fadd_rn(a.z, b.z), 0.5f);
       o.w = __fmul_rn(__fadd_rn(a.w, b.w), 0.5f);
     } else {
+      if (!idx_ok(err, (row + half_video) * d4 + col, 1, full, 3)) continue;
       o = __ldcs(x + (row + half_video) * d4 + col);  // audio: full row = V + a = merged row + V/2
     }
     xm[e] = o;
@@ -162,7 +168,8 @@ __global__ void k_merge(const float4* __restrict__ x, float4* __restrict__ xm, f
   }
 }
 
-__global__ void k_unmerge(const float4* __restrict__ xm, float4* __restrict__ x, int n_video, int n_audio, int d4) {
+__global__ void k_unmerge(const float4* __restrict__ xm, float4* __restrict__ x, int n_video, int n_audio, int d4,
+                          int* err) {
   pdl_trigger();
   pdl_wait();
   const size_t total = static_cast<size_t>(n_video + n_audio) * d4;
@@ -171,6 +178,7 @@ __global__ void k_unmerge(const float4* __restrict__ xm, float4* __restrict__ x,
   for (size_t e = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < total; e += stride) {
     const size_t row = e / d4, col = e - row * d4;
     const size_t src = row < static_cast<size_t>(n_video) ? row / 2 : row - half;
+    if (!idx_ok(err, src * d4 + col, 1, (static_cast<long long>(half) + n_audio) * d4, 5)) continue;
     x[e] = xm[src * d4 + col];
   }
 }
@@ -178,7 +186,7 @@ __global__ void k_unmerge(const float4* __restrict__ xm, float4* __restrict__ x,
 // Delta-broadcast unmerge: full video row r gains ym[r/2] - xm0[r/2] (the
 // merged blocks' update); audio rows take ym.
 __global__ void k_unmerge_delta(float4* __restrict__ x, const float4* __restrict__ ym,
-                                const float4* __restrict__ xm0, int n_video, int n_audio, int d4) {
+                                const float4* __restrict__ xm0, int n_video, int n_audio, int d4, int* err) {
   pdl_trigger();
   pdl_wait();
   const size_t total = static_cast<size_t>(n_video + n_audio) * d4;
@@ -186,8 +194,10 @@ __global__ void k_unmerge_delta(float4* __restrict__ x, const float4* __restrict
   const int half = n_video / 2;
   for (size_t e = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < total; e += stride) {
     const size_t row = e / d4, col = e - row * d4;
+    const long long merged = (static_cast<long long>(half) + n_audio) * d4;
     if (row < static_cast<size_t>(n_video)) {
       const size_t src = (row / 2) * d4 + col;
+      if (!idx_ok(err, src, 1, merged, 6)) continue;
       const float4 y = ym[src], m = xm0[src];
       float4 v = x[e];
       v.x += y.x - m.x;
@@ -196,6 +206,7 @@ __global__ void k_unmerge_delta(float4* __restrict__ x, const float4* __restrict
       v.w += y.w - m.w;
       x[e] = v;
     } else {
+      if (!idx_ok(err, (row - half) * d4 + col, 1, merged, 7)) continue;
       x[e] = ym[(row - half) * d4 + col];
     }
   }
@@ -209,7 +220,7 @@ __global__ void k_unmerge_delta(float4* __restrict__ x, const float4* __restrict
 // one fp64 product and a fp64 reduction modulo 2 pi before the fp32 sincos.
 constexpr int kMaxHalfHead = 64;  // head_dim <= 128
 __global__ void k_rope_table(float2* __restrict__ table, int F, int H, int Wc, int A, int D, float theta,
-                             int merged) {
+                             int merged, int* err) {
   pdl_trigger();
   __shared__ double f_video[kMaxHalfHead], f_audio[kMaxHalfHead];
   const int half = D / 2;
@@ -247,18 +258,20 @@ __global__ void k_rope_table(float2* __restrict__ table, int F, int H, int Wc, i
     const float red = static_cast<float>(fma(-rint(ang * inv_two_pi), two_pi, ang));
     float sn, cs;
     sincosf(red, &sn, &cs);
+    if (!idx_ok(err, e, 1, total, 8)) continue;
     table[e] = make_float2(cs, sn);
   }
 }
 
 // ------------------------------------------------------------------ GELU (the FC1 epilogue's function)
-__global__ void k_gelu(const float* __restrict__ x, float* __restrict__ y, size_t n) {
+__global__ void k_gelu(const float* __restrict__ x, float* __restrict__ y, size_t n, int* err) {
   pdl_trigger();
   pdl_wait();
   // pairs through the same packed form the GEMM epilogue uses; an odd last element alone
   const size_t pairs = n / 2;
   for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < pairs;
        i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    if (!idx_ok(err, 2 * i, 2, n, 9)) continue;
     float a = x[2 * i], b = x[2 * i + 1];
     gelu_erf2(a, b);
     y[2 * i] = a;
@@ -273,11 +286,12 @@ __global__ void k_gelu(const float* __restrict__ x, float* __restrict__ y, size_
 template <int VPT, bool INT8>
 __global__ void __launch_bounds__(kThreads) k_rmsnorm(const float* __restrict__ x, const float* __restrict__ g, int d,
                                                       float eps, void* __restrict__ out, float* __restrict__ out_scale,
-                                                      const Mod mod) {
+                                                      const Mod mod, int* err) {
   pdl_trigger();
   pdl_wait();
   __shared__ float red[32];
   const int row = blockIdx.x, d4 = d >> 2;
+  const long long n4 = static_cast<long long>(gridDim.x) * d4;  // float4 units of x (and of the output rows)
   const float4* xr = reinterpret_cast<const float4*>(x + static_cast<size_t>(row) * d);
   const float4* g4 = reinterpret_cast<const float4*>(g);
   float4 v[VPT];
@@ -285,7 +299,7 @@ __global__ void __launch_bounds__(kThreads) k_rmsnorm(const float* __restrict__ 
 #pragma unroll
   for (int i = 0; i < VPT; ++i) {
     const int c = threadIdx.x + i * blockDim.x;
-    if (c < d4) {
+    if (c < d4 && idx_ok(err, static_cast<long long>(row) * d4 + c, 1, n4, 10)) {
       v[i] = xr[c];
       ss += v[i].x * v[i].x + v[i].y * v[i].y + v[i].z * v[i].z + v[i].w * v[i].w;
     } else {
@@ -319,7 +333,8 @@ __global__ void __launch_bounds__(kThreads) k_rmsnorm(const float* __restrict__ 
         uint2 p;
         p.x = pack_bf16x2(v[i].x, v[i].y);
         p.y = pack_bf16x2(v[i].z, v[i].w);
-        reinterpret_cast<uint2*>(out)[static_cast<size_t>(row) * d4 + c] = p;
+        if (idx_ok(err, static_cast<long long>(row) * d4 + c, 1, n4, 11))
+          reinterpret_cast<uint2*>(out)[static_cast<size_t>(row) * d4 + c] = p;
       }
     }
   }
@@ -329,9 +344,10 @@ __global__ void __launch_bounds__(kThreads) k_rmsnorm(const float* __restrict__ 
 #pragma unroll
     for (int i = 0; i < VPT; ++i) {
       const int c = threadIdx.x + i * blockDim.x;
-      if (c < d4) reinterpret_cast<uint32_t*>(out)[static_cast<size_t>(row) * d4 + c] = quant4(v[i].x, v[i].y, v[i].z, v[i].w, s, rs);
+      if (c < d4 && idx_ok(err, static_cast<long long>(row) * d4 + c, 1, n4, 11))
+        reinterpret_cast<uint32_t*>(out)[static_cast<size_t>(row) * d4 + c] = quant4(v[i].x, v[i].y, v[i].z, v[i].w, s, rs);
     }
-    if (threadIdx.x == 0) out_scale[row] = s;
+    if (threadIdx.x == 0 && idx_ok(err, row, 1, gridDim.x, 12)) out_scale[row] = s;
   }
 }
 
@@ -364,7 +380,7 @@ __device__ __forceinline__ float bf16x8_absmax(const uint4& u) {
 // One CTA per row: max |row| then codes, row held in registers.
 template <int VPT>
 __global__ void __launch_bounds__(kThreads) k_quant_rows(const uint4* __restrict__ a, int k8, int8_t* __restrict__ q,
-                                                         float* __restrict__ scale) {
+                                                         float* __restrict__ scale, int* err) {
   pdl_trigger();
   pdl_wait();
   __shared__ float red[32];
@@ -375,7 +391,9 @@ __global__ void __launch_bounds__(kThreads) k_quant_rows(const uint4* __restrict
 #pragma unroll
   for (int i = 0; i < VPT; ++i) {
     const int c = threadIdx.x + i * blockDim.x;
-    v[i] = c < k8 ? ar[c] : make_uint4(0, 0, 0, 0);
+    v[i] = c < k8 && idx_ok(err, static_cast<long long>(row) * k8 + c, 1, static_cast<long long>(gridDim.x) * k8, 13)
+               ? ar[c]
+               : make_uint4(0, 0, 0, 0);
     amax = fmaxf(amax, bf16x8_absmax(v[i]));
   }
   amax = block_reduce<true>(amax, red);
@@ -384,13 +402,13 @@ __global__ void __launch_bounds__(kThreads) k_quant_rows(const uint4* __restrict
 #pragma unroll
   for (int i = 0; i < VPT; ++i) {
     const int c = threadIdx.x + i * blockDim.x;
-    if (c < k8) {
+    if (c < k8 && idx_ok(err, static_cast<long long>(row) * k8 + c, 1, static_cast<long long>(gridDim.x) * k8, 14)) {
       float f[8];
       bf16x8_to_f32(v[i], f);
       qr[c] = quant8(f, s, rs);
     }
   }
-  if (threadIdx.x == 0) scale[row] = s;
+  if (threadIdx.x == 0 && idx_ok(err, row, 1, gridDim.x, 14)) scale[row] = s;
 }
 
 // Known row maxima: purely elementwise.  One CTA per row; thread t takes the
@@ -402,26 +420,28 @@ __global__ void __launch_bounds__(kThreads) k_quant_rows(const uint4* __restrict
 template <int CPT>
 __global__ void __launch_bounds__(kThreads) k_quant_absmax(const uint4* __restrict__ a,
                                                            const float* __restrict__ absmax, int k16,
-                                                           int8_t* __restrict__ q, float* __restrict__ scale) {
+                                                           int8_t* __restrict__ q, float* __restrict__ scale,
+                                                           int* err) {
   pdl_trigger();
   pdl_wait();
   const int row = blockIdx.x;
+  const long long n16 = static_cast<long long>(gridDim.x) * k16;  // 16-element chunks of a and q
   const uint4* ar = a + static_cast<size_t>(row) * k16 * 2;
   uint4* qr = reinterpret_cast<uint4*>(q) + static_cast<size_t>(row) * k16;
   uint4 v[2 * CPT];
 #pragma unroll
   for (int i = 0; i < CPT; ++i) {
     const int c = threadIdx.x + i * kThreads;
-    if (c < k16) {
+    if (c < k16 && idx_ok(err, 2 * (static_cast<long long>(row) * k16 + c), 2, 2 * n16, 15)) {
       v[2 * i] = __ldcs(ar + 2 * c);
       v[2 * i + 1] = __ldcs(ar + 2 * c + 1);
     }
   }
-  const float s = absmax[row] / 127.0f, rs = 1.0f / s;
+  const float s = idx_ok(err, row, 1, gridDim.x, 17) ? absmax[row] / 127.0f : 0.f, rs = 1.0f / s;
 #pragma unroll
   for (int i = 0; i < CPT; ++i) {
     const int c = threadIdx.x + i * kThreads;
-    if (c < k16) {
+    if (c < k16 && idx_ok(err, static_cast<long long>(row) * k16 + c, 1, n16, 16)) {
       float f0[8], f1[8];
       bf16x8_to_f32(v[2 * i], f0);
       bf16x8_to_f32(v[2 * i + 1], f1);
@@ -429,24 +449,36 @@ __global__ void __launch_bounds__(kThreads) k_quant_absmax(const uint4* __restri
       qr[c] = make_uint4(lo.x, lo.y, hi.x, hi.y);
     }
   }
-  if (threadIdx.x == 0) scale[row] = s;
+  if (threadIdx.x == 0 && idx_ok(err, row, 1, gridDim.x, 17)) scale[row] = s;
 }
 
 // Same with 8 elements per thread (k a multiple of 8 but not of 16).
 __global__ void k_quant_absmax8(const uint4* __restrict__ a, const float* __restrict__ absmax, int k8,
-                                int8_t* __restrict__ q, float* __restrict__ scale) {
+                                int8_t* __restrict__ q, float* __restrict__ scale, int* err) {
   pdl_trigger();
   pdl_wait();
   const int row = blockIdx.y;
-  const float s = absmax[row] / 127.0f, rs = 1.0f / s;
+  const long long n8 = static_cast<long long>(gridDim.y) * k8;  // 8-element chunks of a and q (this launch)
+  const float s = idx_ok(err, row, 1, gridDim.y, 17) ? absmax[row] / 127.0f : 0.f, rs = 1.0f / s;
   const uint4* ar = a + static_cast<size_t>(row) * k8;
   uint2* qr = reinterpret_cast<uint2*>(q) + static_cast<size_t>(row) * k8;
   for (int c = blockIdx.x * blockDim.x + threadIdx.x; c < k8; c += gridDim.x * blockDim.x) {
+    if (!idx_ok(err, static_cast<long long>(row) * k8 + c, 1, n8, 15)) continue;
     float f[8];
     bf16x8_to_f32(__ldcs(ar + c), f);
     qr[c] = quant8(f, s, rs);
   }
-  if (blockIdx.x == 0 && threadIdx.x == 0) scale[row] = s;
+  if (blockIdx.x == 0 && threadIdx.x == 0 && idx_ok(err, row, 1, gridDim.y, 17)) scale[row] = s;
+}
+
+// Self-test of the index checks: one thread passes index i of an extent n
+// through idx_ok as every checked access does, without touching memory.  In
+// the index-checked build an i outside [0, n) records (EK_INDEX << 8) | 99.
+__global__ void k_selftest_index(int* err, long long i, long long n) {
+  pdl_trigger();
+  pdl_wait();
+  if (idx_ok(err, i, 1, n, 99)) {
+  }
 }
 
 // Failure-path self-test: wait on an mbarrier that nothing will complete,
@@ -478,7 +510,7 @@ int grid_for(size_t work_items, int num_sms, int per_sm = 8) {
 cudaError_t launch_flow_step(const Ctx& c, float* x, const float* v, float dt, size_t n, float* x_copy) {
   if (n == 0) return cudaSuccess;
   return launch_pdl(c.stream, k_flow, dim3(grid_for((n + 3) / 4, c.num_sms)), dim3(kThreads), 0, 1u, x, v, dt, n,
-                    x_copy);
+                    x_copy, c.err);
 }
 
 cudaError_t launch_merge(const Ctx& c, const float* x, float* xm, int n_video, int n_audio, int d, float* xm_copy) {
@@ -487,7 +519,7 @@ cudaError_t launch_merge(const Ctx& c, const float* x, float* xm, int n_video, i
   if (total == 0) return cudaSuccess;
   return launch_pdl(c.stream, k_merge, dim3(grid_for(total, c.num_sms)), dim3(kThreads), 0, 1u,
                     reinterpret_cast<const float4*>(x), reinterpret_cast<float4*>(xm),
-                    reinterpret_cast<float4*>(xm_copy), n_video / 2, n_audio, d4);
+                    reinterpret_cast<float4*>(xm_copy), n_video / 2, n_audio, d4, c.err);
 }
 
 cudaError_t launch_unmerge_delta(const Ctx& c, float* x, const float* ym, const float* xm0, int n_video, int n_audio,
@@ -497,7 +529,7 @@ cudaError_t launch_unmerge_delta(const Ctx& c, float* x, const float* ym, const 
   if (total == 0) return cudaSuccess;
   return launch_pdl(c.stream, k_unmerge_delta, dim3(grid_for(total, c.num_sms)), dim3(kThreads), 0, 1u,
                     reinterpret_cast<float4*>(x), reinterpret_cast<const float4*>(ym),
-                    reinterpret_cast<const float4*>(xm0), n_video, n_audio, d4);
+                    reinterpret_cast<const float4*>(xm0), n_video, n_audio, d4, c.err);
 }
 
 cudaError_t launch_unmerge(const Ctx& c, const float* xm, float* x, int n_video, int n_audio, int d) {
@@ -505,7 +537,7 @@ cudaError_t launch_unmerge(const Ctx& c, const float* xm, float* x, int n_video,
   const size_t total = static_cast<size_t>(n_video + n_audio) * d4;
   if (total == 0) return cudaSuccess;
   return launch_pdl(c.stream, k_unmerge, dim3(grid_for(total, c.num_sms)), dim3(kThreads), 0, 1u,
-                    reinterpret_cast<const float4*>(xm), reinterpret_cast<float4*>(x), n_video, n_audio, d4);
+                    reinterpret_cast<const float4*>(xm), reinterpret_cast<float4*>(x), n_video, n_audio, d4, c.err);
 }
 
 cudaError_t launch_rope_table(const Ctx& c, const h3b_dims& dm, int merged, float* table) {
@@ -514,12 +546,12 @@ cudaError_t launch_rope_table(const Ctx& c, const h3b_dims& dm, int merged, floa
   if (total == 0) return cudaSuccess;
   return launch_pdl(c.stream, k_rope_table, dim3(grid_for(total, c.num_sms, 8)), dim3(kThreads), 0, 1u,
                     reinterpret_cast<float2*>(table), dm.frames, dm.rows, wc, dm.n_audio, dm.head_dim, dm.rope_theta,
-                    merged);
+                    merged, c.err);
 }
 
 cudaError_t launch_gelu(const Ctx& c, const float* x, float* y, size_t n) {
   if (n == 0) return cudaSuccess;
-  return launch_pdl(c.stream, k_gelu, dim3(grid_for(n, c.num_sms)), dim3(kThreads), 0, 1u, x, y, n);
+  return launch_pdl(c.stream, k_gelu, dim3(grid_for(n, c.num_sms)), dim3(kThreads), 0, 1u, x, y, n, c.err);
 }
 
 cudaError_t launch_rmsnorm(const Ctx& c, const float* x, const float* g, int rows, int d, float eps, void* out,
@@ -537,9 +569,9 @@ cudaError_t launch_rmsnorm(const Ctx& c, const float* x, const float* g, int row
 #define H3B_NORM_CASE(V)                                                                                       \
   case V:                                                                                                      \
     e = out_int8 ? launch_pdl(c.stream, k_rmsnorm<V, true>, dim3(rows), dim3(threads), 0, 1u, x, g, d, eps, out,  \
-                              out_scale, mod)                                                                  \
+                              out_scale, mod, c.err)                                                           \
                  : launch_pdl(c.stream, k_rmsnorm<V, false>, dim3(rows), dim3(threads), 0, 1u, x, g, d, eps, out, \
-                              out_scale, mod);                                                                 \
+                              out_scale, mod, c.err);                                                          \
     break;
   switch (vpt) {
     H3B_NORM_CASE(1) H3B_NORM_CASE(2) H3B_NORM_CASE(3) H3B_NORM_CASE(4)
@@ -566,7 +598,7 @@ cudaError_t launch_quant_rows(const Ctx& c, const void* a, int rows, int k, int8
   const uint4* a4 = reinterpret_cast<const uint4*>(a);
   cudaError_t e;
 #define H3B_Q_CASE(V) \
-  case V: e = launch_pdl(c.stream, k_quant_rows<V>, dim3(rows), dim3(threads), 0, 1u, a4, k8, q, s); break;
+  case V: e = launch_pdl(c.stream, k_quant_rows<V>, dim3(rows), dim3(threads), 0, 1u, a4, k8, q, s, c.err); break;
   switch (vpt) {
     H3B_Q_CASE(1) H3B_Q_CASE(2) H3B_Q_CASE(3) H3B_Q_CASE(4) H3B_Q_CASE(5) H3B_Q_CASE(6)
     H3B_Q_CASE(7) H3B_Q_CASE(8) H3B_Q_CASE(9) H3B_Q_CASE(10) H3B_Q_CASE(11) H3B_Q_CASE(12)
@@ -585,7 +617,9 @@ cudaError_t launch_quant_absmax(const Ctx& c, const void* a, const float* absmax
   if (k % 16 == 0 && cpt <= 8) {  // k <= 32768: one CTA per row
     cudaError_t e = cudaErrorInvalidValue;
 #define H3B_QA_CASE(V) \
-  case V: e = launch_pdl(c.stream, k_quant_absmax<V>, dim3(rows), dim3(kThreads), 0, 1u, a4, absmax, k16, q, s); break;
+  case V:                                                                                                          \
+    e = launch_pdl(c.stream, k_quant_absmax<V>, dim3(rows), dim3(kThreads), 0, 1u, a4, absmax, k16, q, s, c.err); \
+    break;
     switch (cpt) {
       H3B_QA_CASE(1) H3B_QA_CASE(2) H3B_QA_CASE(3) H3B_QA_CASE(4) H3B_QA_CASE(5) H3B_QA_CASE(6)
       H3B_QA_CASE(7) H3B_QA_CASE(8)
@@ -601,10 +635,14 @@ cudaError_t launch_quant_absmax(const Ctx& c, const void* a, const float* absmax
     const dim3 grid(bx, nr);
     const uint4* ar = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(a) + static_cast<size_t>(r0) * k);
     const cudaError_t e = launch_pdl(c.stream, k_quant_absmax8, grid, dim3(kThreads), 0, 1u, ar, absmax + r0, chunks,
-                                     q + static_cast<size_t>(r0) * k, s + r0);
+                                     q + static_cast<size_t>(r0) * k, s + r0, c.err);
     if (e != cudaSuccess) return e;
   }
   return cudaGetLastError();
+}
+
+cudaError_t launch_selftest_index(const Ctx& c, long long i, long long n) {
+  return launch_pdl(c.stream, k_selftest_index, dim3(1), dim3(1), 0, 1u, c.err, i, n);
 }
 
 cudaError_t launch_selftest_wait(const Ctx& c, unsigned long long timeout_ns) {

@@ -73,6 +73,8 @@ _SIGS = {
     "h3b_gelu": (_i, [_p, _p, _sz, _p]),
     "h3b_device_error": (_i, [_p]),
     "h3b_selftest_wait_timeout": (_i, [_i, _p]),
+    "h3b_selftest_index_check": (_i, [ctypes.c_longlong, ctypes.c_longlong, _p]),
+    "h3b_index_checked": (_i, []),
     "h3b_trace_start": (_i, [_i]),
     "h3b_trace_stop": (_i, [ctypes.POINTER(_i)]),
     "h3b_trace_read": (_i, [_p, _p, _i]),
@@ -414,6 +416,18 @@ def gelu(x: torch.Tensor) -> torch.Tensor:
 
 def device_error() -> int:
     return lib.h3b_device_error(_stream())
+
+
+def index_checked() -> bool:
+    """True when the loaded library is the index-checked build (libh3b_check.so)."""
+    return bool(lib.h3b_index_checked())
+
+
+def selftest_index_check(i: int, n: int) -> None:
+    """Passes index i of extent n through the kernels' index check without
+    touching memory (records (4 << 8) | 99 in the checked build when i is out
+    of range; nothing in the default build)."""
+    _check(lib.h3b_selftest_index_check(i, n, _stream()), "h3b_selftest_index_check")
 
 
 class Trace:

@@ -349,6 +349,22 @@ int h3b_gelu(const float* x, float* y, size_t n, void* stream);
  * Read the code with h3b_device_error. */
 int h3b_selftest_wait_timeout(int timeout_us, void* stream);
 
+/* Index-checked build.  libh3b_check.so is the same library compiled with
+ * -DH3B_CHECK=1: every hand-indexed global load and store first checks its
+ * element range against the extent of its buffer as the kernel's own shape
+ * arguments define it (rows x columns of a GEMM output, tokens x width of a
+ * norm, the caller's scratch bytes for split partials).  A range outside the
+ * extent records (4 << 8) | site in the device error word (the first record
+ * wins) and the access is skipped: no trap, no fault.  TMA tile loads are
+ * bounded by their tensor maps and are not checked.  h3b_index_checked
+ * returns 1 in that build and 0 in the default one.
+ * h3b_selftest_index_check(i, n) runs one thread that passes index i of
+ * extent n (n > 0) through the same check without touching memory: in the
+ * checked build an i outside [0, n) records (4 << 8) | 99; the default build
+ * records nothing. */
+int h3b_index_checked(void);
+int h3b_selftest_index_check(long long i, long long n, void* stream);
+
 /* Reads and clears the device error word of the current device
  * (synchronises the stream).  0 = no error; otherwise a code naming the
  * kernel and wait that gave up. */

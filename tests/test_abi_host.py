@@ -17,6 +17,19 @@ def test_every_header_function_is_exported():
         assert hasattr(h3b.lib, n), n
 
 
+def test_index_checked_library_exports_the_same_symbols():
+    """libh3b_check.so (built beside libh3b.so with -DH3B_CHECK=1) is a drop-in
+    for the default library: it loads without a GPU and exports every entry
+    point of include/h3b.h."""
+    import ctypes
+    import os
+    path = os.path.join(os.path.dirname(h3b.LIB_PATH), "libh3b_check.so")
+    assert os.path.exists(path), "libh3b_check.so not built"
+    lib = ctypes.CDLL(path, mode=ctypes.RTLD_LOCAL)
+    for n in h3b.header_functions():
+        assert hasattr(lib, n), n
+
+
 def test_status_strings():
     for code in range(0, -9, -1):
         assert h3b.lib.h3b_status_string(code).decode() != "unknown status"
