@@ -714,6 +714,18 @@ int h3b_token_unmerge(const h3b_dims* dims, const float* xm, float* x, void* str
   return H3B_OK;
 }
 
+int h3b_token_unmerge_delta(const h3b_dims* dims, float* x, const float* ym, const float* xm0, void* stream) {
+  H3B_TRY(check_dims(dims));
+  if (!x || !ym || !xm0) return H3B_ERR_NULL;
+  if (!aligned16(x) || !aligned16(ym) || !aligned16(xm0)) return H3B_ERR_ALIGN;
+  if (dims->cols & 1) return H3B_ERR_DIMS;
+  Ctx c;
+  H3B_TRY(device_ctx(static_cast<cudaStream_t>(stream), &c));
+  H3B_CU(KID_UNMERGE_DELTA,
+         launch_unmerge_delta(c, x, ym, xm0, dims->frames * dims->rows * dims->cols, dims->n_audio, dims->d));
+  return H3B_OK;
+}
+
 int h3b_flow_step(float* x, const float* v, float sigma_cur, float sigma_next, size_t n, float* x_copy,
                   void* stream) {
   if (n == 0) return H3B_OK;  // nothing to update; empty buffers may be NULL

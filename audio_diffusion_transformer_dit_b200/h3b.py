@@ -63,6 +63,7 @@ _SIGS = {
     "h3b_quantize_weights": (_i, [_p, _i, _i, _p, _p, _p]),
     "h3b_token_merge": (_i, [ctypes.POINTER(Dims), _p, _p, _p]),
     "h3b_token_unmerge": (_i, [ctypes.POINTER(Dims), _p, _p, _p]),
+    "h3b_token_unmerge_delta": (_i, [ctypes.POINTER(Dims), _p, _p, _p, _p]),
     "h3b_flow_step": (_i, [_p, _p, _f, _f, _sz, _p, _p]),
     "h3b_rope_table": (_i, [ctypes.POINTER(Dims), _i, _p, _p]),
     "h3b_rmsnorm": (_i, [_p, _p, _i, _i, _f, _p, _p, _i, _p]),
@@ -336,6 +337,13 @@ def token_merge(dims: Dims, x: torch.Tensor, xm: torch.Tensor) -> torch.Tensor:
 def token_unmerge(dims: Dims, xm: torch.Tensor, x: torch.Tensor) -> torch.Tensor:
     _check(lib.h3b_token_unmerge(ctypes.byref(dims), _ptr(xm, torch.float32, "xm"), _ptr(x, torch.float32, "x"),
                                  _stream()), "h3b_token_unmerge")
+    return x
+
+
+def token_unmerge_delta(dims: Dims, x: torch.Tensor, ym: torch.Tensor, xm0: torch.Tensor) -> torch.Tensor:
+    """x (the pre-merge tokens) += the merged blocks' update ym - xm0, broadcast to both columns of each pair."""
+    _check(lib.h3b_token_unmerge_delta(ctypes.byref(dims), _ptr(x, torch.float32, "x"), _ptr(ym, torch.float32, "ym"),
+                                       _ptr(xm0, torch.float32, "xm0"), _stream()), "h3b_token_unmerge_delta")
     return x
 
 

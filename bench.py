@@ -236,6 +236,7 @@ def kernel_work(name, wl, dtype, merged=False):
               "rope_table": S * (wl.head_dim // 2) * 8,
               "token_merge": wl.seq * d * 4 + wl.seq_merged * d * 4,
               "token_unmerge": wl.seq * d * 4 + wl.seq_merged * d * 4,
+              "token_unmerge_delta": 2 * wl.seq * d * 4 + 2 * wl.seq_merged * d * 4,
               "flow_step": wl.seq * d * 4 * 3,
               # folded RMSNorm: each row's partial sums of squares (2 per 256 columns) -> one factor
               "norm_scale": S * (2 * ((d + 255) // 256)) * 4 + S * 4}
@@ -764,6 +765,7 @@ def kernel_sweep(args):
     xm5 = torch.empty((wl5.seq_merged, wl5.d), dtype=torch.float32, device=dev)
     v5 = W.normal_tensor((wl5.seq, wl5.d), 15, dev)
     cp5 = torch.empty_like(v5)
+    ym5 = W.normal_tensor((wl5.seq_merged, wl5.d), 16, dev)
     # outputs allocated once: every timed launch is the library call alone
     u_bf = torch.empty((S, d), dtype=torch.bfloat16, device=dev)
     q_d = torch.empty((S, d), dtype=torch.int8, device=dev)
@@ -784,6 +786,9 @@ def kernel_sweep(args):
          (wl5.seq + wl5.seq_merged) * wl5.d * 4, f"x fp32 [{wl5.seq},{wl5.d}] -> [{wl5.seq_merged},{wl5.d}]"),
         ("token_unmerge", lambda: lib.h3b_token_unmerge(ctypes.byref(dm5), P(xm5), P(x5), st),
          (wl5.seq + wl5.seq_merged) * wl5.d * 4, f"xm fp32 [{wl5.seq_merged},{wl5.d}] -> [{wl5.seq},{wl5.d}]"),
+        ("token_unmerge_delta", lambda: lib.h3b_token_unmerge_delta(ctypes.byref(dm5), P(x5), P(ym5), P(xm5), st),
+         2 * (wl5.seq + wl5.seq_merged) * wl5.d * 4,
+         f"x fp32 [{wl5.seq},{wl5.d}] += (ym - xm0) [{wl5.seq_merged},{wl5.d}] broadcast"),
         ("flow_step", lambda: lib.h3b_flow_step(P(x5), P(v5), ctypes.c_float(0.5), ctypes.c_float(0.45),
                                                  ctypes.c_size_t(x5.numel()), None, st),
          3 * wl5.seq * wl5.d * 4, f"x, v fp32 [{wl5.seq},{wl5.d}] -> x"),

@@ -231,6 +231,15 @@ int h3b_token_merge(const h3b_dims* dims, const float* x, float* xm, void* strea
  * copied.  xm: fp32 [S', d]; x: fp32 [S, d]. */
 int h3b_token_unmerge(const h3b_dims* dims, const float* xm, float* x, void* stream);
 
+/* Delta-broadcast unmerge, the unit form of h3b_stack_opts.unmerge_delta
+ * [control]: x holds the pre-merge tokens [S, d] fp32 and is updated in
+ * place, video row (f*H+r)*W + c += ym[m] - xm0[m] with
+ * m = (f*H+r)*(W/2) + c/2 (one fp32 subtraction, then one fp32 addition);
+ * the audio rows take ym's rows after the merged video rows.  ym: what the
+ * merged blocks returned, xm0: what entered them, both fp32 [S', d] with
+ * S' = h3b_seq_len(dims, 1).  W must be even. */
+int h3b_token_unmerge_delta(const h3b_dims* dims, float* x, const float* ym, const float* xm0, void* stream);
+
 /* Euler update x[i] <- x[i] + (sigma_next - sigma_cur) * v[i] for i < n
  * (fp32, fused multiply-add); when x_copy is not NULL the updated value is
  * also written to x_copy[i] (the next fresh evaluation's input) [control].

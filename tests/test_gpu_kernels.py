@@ -58,6 +58,27 @@ def test_merge_unmerge_bitexact(cuda_dev, geom):
     assert np.array_equal(back.cpu().numpy(), oracle.token_unmerge(ref, wl).astype(np.float32))
 
 
+@pytest.mark.parametrize("geom", [(5, 48, 84, 480, 128), (2, 3, 4, 5, 256)])
+def test_unmerge_delta_bitexact(cuda_dev, geom):
+    """x_pre + (ym - xm0) broadcast: on values that are multiples of 2^-10
+    below 2^8 in magnitude the fp32 subtraction and addition are exact, so the
+    kernel equals the fp64 oracle bit for bit; audio rows are copied from ym."""
+    F, H, W, A, d = geom
+    wl = wlmod.Workload("g", F, H, W, A, d, d // 128, 128, 4 * d, 1, 0, 0, False)
+    dm = h3b.dims_of(wl)
+    S, Sm = F * H * W + A, F * H * W // 2 + A
+
+    def grid(shape, seed):
+        return torch.round(wlmod.normal_tensor(shape, seed, cuda_dev) * 1024.0 * 8.0) / 1024.0
+
+    x = grid((S, d), 70)
+    ym, xm0 = grid((Sm, d), 71), grid((Sm, d), 72)
+    ref = oracle.token_unmerge_delta(np64(x), np64(ym), np64(xm0), wl)
+    h3b.token_unmerge_delta(dm, x, ym, xm0)
+    torch.cuda.synchronize()
+    assert np.array_equal(x.cpu().numpy(), ref.astype(np.float32))
+
+
 def test_merge_rejects_odd_width(cuda_dev):
     wl = wlmod.Workload("g", 2, 3, 5, 1, 128, 1, 128, 512, 1, 0, 0, False)
     x = torch.zeros((31, 128), device=cuda_dev)
