@@ -15,8 +15,8 @@ from typing import Optional, Sequence
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-# H3B_LIBRARY names another build of the same library (e.g. one compiled with
-# different tuning macros); by default the in-tree libh3b.so is loaded.
+# H3B_LIBRARY names another build of the same library (e.g. libh3b_check.so,
+# the index-checked build next to it); by default the in-tree libh3b.so is loaded.
 LIB_PATH = os.environ.get("H3B_LIBRARY") or os.path.join(_HERE, "libh3b.so")
 HEADER = os.path.join(os.path.dirname(_HERE), "include", "h3b.h")
 
