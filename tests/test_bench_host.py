@@ -49,3 +49,30 @@ def test_oracle_chunks_int8_reference_uses_dequantised_weights():
     out = np.concatenate([oc.run(i) for i in range(4)], axis=0)
     w, x = bench._oracle_inputs(wl)
     assert np.allclose(out, oracle.block_forward(x, oracle.dequant_weights(w), wl), rtol=1e-12, atol=1e-12)
+
+
+def test_measured_traffic_only_for_the_source_it_was_taken_on(monkeypatch, tmp_path):
+    """The roofline's `traffic` comes from a committed ncu figure only while
+    the kernel's source still hashes to the digest recorded with it; after any
+    change to that source the bench reports null rather than a stale number."""
+    src = tmp_path / "k.cu"
+    src.write_text("kernel v1")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "KERNEL_SOURCES", {"attention": ["k.cu"], "gemm": ["k.cu"], "mem": ["k.cu"]})
+    (tmp_path / "profiles").mkdir()
+    rec = {"attention@wl": {"bytes_per_launch": 123, "src": bench.src_digest(["k.cu"])}}
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(rec))
+    assert bench.measured_traffic("attention", "wl") == 123
+    assert bench.measured_traffic("attention", "other_workload") is None
+    src.write_text("kernel v2")
+    assert bench.measured_traffic("attention", "wl") is None
+
+
+def test_committed_traffic_matches_the_current_sources():
+    """Every committed traffic figure was taken on the kernel sources as they
+    are in this tree (the bench line would otherwise report null)."""
+    rec = json.load(open(bench.os.path.join(bench.ROOT, "profiles", "traffic.json")))
+    assert rec
+    for key in rec:
+        kernel, wl = key.split("@")
+        assert bench.measured_traffic(kernel, wl) == rec[key]["bytes_per_launch"], key
