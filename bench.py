@@ -741,6 +741,100 @@ def measure_int8_peak(out_path, n=8192, burst_reps=10, sustain_s=4.0):
     print(json.dumps(rec), flush=True)
 
 
+def library_compare(args):
+    """This library's GEMMs and attention against the vendor libraries on the
+    d = 5120 shapes, timed back to back on one GPU in alternating rounds
+    (CUDA events, median): the four linear layers with a plain bf16 output
+    against torch.matmul (cuBLAS, same operand layouts, no K split here), and
+    bidirectional attention against torch's scaled_dot_product_attention with
+    the cuDNN and flash backends, on strided views of the same qkv buffer.
+    The implementations of a case run in interleaved blocks whose order
+    alternates, so both see the same clock history under the power cap; the
+    figure is the median over the blocks.  A comparison only: nothing on the
+    product path calls these libraries.  One JSON line per case."""
+    import torch.nn.functional as F
+    from torch.nn.attention import SDPBackend, sdpa_kernel
+    from audio_diffusion_transformer_dit_b200 import h3b
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+
+    def interleaved(fns, blocks=8, group=5):
+        for fn in fns.values():
+            for _ in range(3):
+                fn()
+        torch.cuda.synchronize()
+        ts = {k: [] for k in fns}
+        for b in range(blocks):
+            for k in (list(fns) if b % 2 == 0 else list(fns)[::-1]):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                for _ in range(group):
+                    fns[k]()
+                e1.record()
+                torch.cuda.synchronize()
+                ts[k].append(e0.elapsed_time(e1) / group)
+        return {k: statistics.median(v) for k, v in ts.items()}
+
+    wl = W.WORKLOADS["stack8_d5120_s6528"]
+    S, d, f = wl.seq, wl.d, wl.ffn
+    gemms = {"qkv": (S, 3 * d, d), "o_proj": (S, d, d), "fc1": (S, f, d), "fc2": (S, d, f)}
+    attn = [(S, wl.n_heads), (6400, 24), (W.WORKLOADS[INT8_WORKLOAD].seq, wl.n_heads)]
+    only = set(args.sweep_only.split(",")) if args.sweep_only else None
+    for name, (M, N, K) in gemms.items():
+        if only and name not in only:
+            continue
+        A = W.normal_tensor((M, K), 1, dev, dtype=torch.bfloat16)
+        B = W.normal_tensor((N, K), 2, dev, 0.02, dtype=torch.bfloat16)
+        C = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        clk = ClockSampler(0)
+        clk.start()
+        t = interleaved({"ours": lambda: h3b.gemm(A, B, h3b.EPI_BF16, C),
+                         "cublas": lambda: torch.matmul(A, B.t(), out=C)})
+        clocks = clk.stop()
+        fl = 2.0 * M * N * K
+        print(json.dumps({"compare": "gemm_bf16", "case": name, "shape_mnk": [M, N, K], "clocks": clocks,
+                          **{f"{k}_ms": round(v, 4) for k, v in t.items()},
+                          **{f"{k}_tflops": round(fl / v / 1e9, 1) for k, v in t.items()},
+                          "ours_over_cublas_speed": round(t["cublas"] / t["ours"], 3)}), flush=True)
+        del A, B, C
+    for Sa, H in attn:
+        name = f"attention_s{Sa}_h{H}"
+        if only and name not in only:
+            continue
+        D = wl.head_dim
+        qkv = W.normal_tensor((Sa, 3 * H * D), 25, dev, dtype=torch.bfloat16)
+        scr = torch.empty(2 * Sa * H * D, dtype=torch.float32, device=dev)
+        out = torch.empty((Sa, H * D), dtype=torch.bfloat16, device=dev)
+        q, k, v = (qkv[:, i * H * D:(i + 1) * H * D].view(Sa, H, D).transpose(0, 1).unsqueeze(0) for i in range(3))
+        fl = 4.0 * Sa * Sa * H * D
+
+        def sdpa(be):
+            def run():
+                with sdpa_kernel(be):
+                    return F.scaled_dot_product_attention(q, k, v)
+            return run
+        fns = {"ours": lambda: h3b.attention(qkv, H, D, o=out, scratch=scr)}
+        rec = {"compare": "attention", "case": name}
+        for bname, be in (("cudnn", SDPBackend.CUDNN_ATTENTION), ("flash", SDPBackend.FLASH_ATTENTION)):
+            try:
+                r = sdpa(be)()[0].transpose(0, 1).reshape(Sa, H * D)
+                fns["ours"]()
+                torch.cuda.synchronize()
+                rec[f"{bname}_max_abs_diff"] = float((r.float() - out.float()).abs().max())
+                fns[bname] = sdpa(be)
+            except RuntimeError as e:  # backend not available for this shape or build
+                rec[f"{bname}_error"] = str(e).splitlines()[0][:160]
+        clk = ClockSampler(0)
+        clk.start()
+        t = interleaved(fns, group=2 if Sa > 10000 else 5)
+        rec["clocks"] = clk.stop()
+        rec.update({f"{k}_ms": round(v, 4) for k, v in t.items()})
+        rec.update({f"{k}_tflops": round(fl / v / 1e9, 1) for k, v in t.items()})
+        rec.update({f"ours_over_{k}_speed": round(v / t["ours"], 3) for k, v in t.items() if k != "ours"})
+        print(json.dumps(rec), flush=True)
+        del qkv, scr, out, q, k, v
+
+
 def kernel_sweep(args):
     """Each memory-bound kernel of the path timed alone at the d = 5120
     workload sizes (CUDA events, median of the repetitions; every input is
@@ -922,8 +1016,13 @@ def main():
     ap.add_argument("--sweep-reps", type=int, default=50)
     ap.add_argument("--sweep-warmup", type=int, default=5)
     ap.add_argument("--sweep-group", type=int, default=10, help="back-to-back launches per timed group")
+    ap.add_argument("--library-compare", action="store_true",
+                    help="time the GEMMs and attention against cuBLAS / cuDNN on the d=5120 shapes (comparison only)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # never fewer than 3 warm-up steps
+    if args.library_compare:
+        library_compare(args)
+        return
     if args.measure_int8_peak:
         measure_int8_peak(INT8_PEAK_FILE)
         return
