@@ -6,7 +6,7 @@ binding is loaded on first use of any of the names below; without the built
 library that raises ImportError -- there is no CPU fallback.  Build with
 ``python -m audio_diffusion_transformer_dit_b200.build``.
 """
-_EXPORTS = ("BF16", "INT8", "Block", "Dims", "H3bError", "HostPipeline", "StackOpts", "Trace", "attention",
+_EXPORTS = ("BF16", "INT8", "Block", "Dims", "Graph", "H3bError", "HostPipeline", "StackOpts", "Trace", "attention",
             "block_forward", "denoise", "denoise_ex", "device_error", "dims_of", "flow_step", "gelu", "gemm",
             "quantize_weights", "rmsnorm", "rope_table", "seq_len", "stack_forward", "stack_forward_ex",
             "stack_opts", "token_merge", "token_unmerge", "workspace", "workspace_bytes", "workspace_ex")

@@ -438,6 +438,24 @@ def selftest_index_check(i: int, n: int) -> None:
     _check(lib.h3b_selftest_index_check(i, n, _stream()), "h3b_selftest_index_check")
 
 
+class Graph:
+    """Library calls captured once into a CUDA graph and replayed with one
+    host call per replay: the same kernels (with their programmatic-launch
+    edges), arguments and buffers.  ``fn`` issues the calls on the current
+    stream; every tensor it touches must stay alive and in place while the
+    graph exists, and the library must have run once on this device before
+    the capture (its first call sets up per-device state).  Tracing
+    (``Trace``) does not see replayed launches."""
+
+    def __init__(self, fn):
+        self.g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.g):
+            fn()
+
+    def replay(self):
+        self.g.replay()
+
+
 class Trace:
     """Per-launch CUDA-event tracing of every kernel the library launches."""
 

@@ -318,6 +318,16 @@ def measure(args, wl, dev, world, local):
         step()
     torch.cuda.synchronize()
     assert h3b.device_error() == 0, "device error word set during warm-up"
+    eager_step = step
+    if args.graph:
+        # the whole step captured once; the timed pass replays it (the traced
+        # pass below stays eager: replayed launches carry no trace events)
+        graph = h3b.Graph(eager_step)
+        step = graph.replay
+        for _ in range(args.warmup):
+            step()
+        torch.cuda.synchronize()
+        assert h3b.device_error() == 0, "device error word set during graph warm-up"
 
     sampler = ClockSampler(local)
     stream = torch.cuda.current_stream()
@@ -342,7 +352,7 @@ def measure(args, wl, dev, world, local):
     with h3b.Trace(capacity=args.steps * (4000 if loop else 16 * len(blocks) + 8)) as tr:
         t0.record(stream)
         for _ in range(args.steps):
-            step()
+            eager_step()
         t1.record(stream)
         torch.cuda.synchronize()
     _barrier(world)
@@ -493,6 +503,7 @@ def measure(args, wl, dev, world, local):
                    "head_dim": wl.head_dim, "ffn": wl.ffn, "blocks": len(blocks),
                    "video_grid": [wl.frames, wl.rows, wl.cols], "audio_tokens": wl.n_audio,
                    "global_batch": 1, "parallelism": f"replicas x{world}",
+                   "launch": "one CUDA graph replay per step" if args.graph else "eager (programmatic dependent launch)",
                    "l2": "no flush: per-step working set (weights + activations + workspace) > 126 MB L2"},
         "tflops": round(flops_step * args.steps * world / (ms / 1e3) / 1e12, 2),
         "roofline": roof, "step_roofline": step_roofline, "gpu_launches": my_launches, "clocks": clocks,
@@ -1016,6 +1027,8 @@ def main():
     ap.add_argument("--sweep-reps", type=int, default=50)
     ap.add_argument("--sweep-warmup", type=int, default=5)
     ap.add_argument("--sweep-group", type=int, default=10, help="back-to-back launches per timed group")
+    ap.add_argument("--graph", action="store_true",
+                    help="capture the step into a CUDA graph once and time its replays")
     ap.add_argument("--library-compare", action="store_true",
                     help="time the GEMMs and attention against cuBLAS / cuDNN on the d=5120 shapes (comparison only)")
     args = ap.parse_args()
