@@ -672,9 +672,10 @@ int h3b_denoise_ex(const h3b_dims* dims, const h3b_block_weights* blocks, int n_
 }
 
 int h3b_quantize_weights(const void* w, int rows, int k, int8_t* q, float* scale, void* stream) {
-  if (!w || !q || !scale) return H3B_ERR_NULL;
+  if (rows != 0 && (!w || !q || !scale)) return H3B_ERR_NULL;
   if (!aligned16(w) || !aligned16(q) || !aligned16(scale)) return H3B_ERR_ALIGN;
   if (rows < 0 || k <= 0 || k % 8 != 0 || k > 32768) return H3B_ERR_DIMS;
+  if (rows == 0) return H3B_OK;
   Ctx c;
   H3B_TRY(device_ctx(static_cast<cudaStream_t>(stream), &c));
   H3B_CU(KID_QUANT_ROWS, launch_quant_rows(c, w, rows, k, q, scale));
@@ -683,9 +684,10 @@ int h3b_quantize_weights(const void* w, int rows, int k, int8_t* q, float* scale
 
 int h3b_quantize_rows_absmax(const void* a, const float* absmax, int rows, int k, int8_t* q, float* scale,
                              void* stream) {
-  if (!a || !absmax || !q || !scale) return H3B_ERR_NULL;
+  if (rows != 0 && (!a || !absmax || !q || !scale)) return H3B_ERR_NULL;
   if (!aligned16(a) || !aligned16(q) || !aligned16(scale) || !aligned16(absmax)) return H3B_ERR_ALIGN;
   if (rows < 0 || k <= 0 || k % 8 != 0) return H3B_ERR_DIMS;
+  if (rows == 0) return H3B_OK;
   Ctx c;
   H3B_TRY(device_ctx(static_cast<cudaStream_t>(stream), &c));
   H3B_CU(KID_QUANT_ABSMAX, launch_quant_absmax(c, a, absmax, rows, k, q, scale));
@@ -750,10 +752,11 @@ int h3b_rope_table(const h3b_dims* dims, int merged, float* table, void* stream)
 
 int h3b_rmsnorm(const float* x, const float* g, int rows, int d, float eps, void* out, float* out_scale,
                 int out_dtype, void* stream) {
-  if (!x || !g || !out || (out_dtype == H3B_INT8 && !out_scale)) return H3B_ERR_NULL;
+  if (rows != 0 && (!x || !g || !out || (out_dtype == H3B_INT8 && !out_scale))) return H3B_ERR_NULL;
   if (!aligned16(x) || !aligned16(g) || !aligned16(out)) return H3B_ERR_ALIGN;
   if (out_dtype != H3B_BF16 && out_dtype != H3B_INT8) return H3B_ERR_DTYPE;
   if (rows < 0 || d <= 0 || d % 4 != 0 || d > 8192 || !(eps >= 0.f)) return H3B_ERR_DIMS;
+  if (rows == 0) return H3B_OK;
   Ctx c;
   H3B_TRY(device_ctx(static_cast<cudaStream_t>(stream), &c));
   H3B_CU(KID_RMSNORM, launch_rmsnorm(c, x, g, rows, d, eps, out, out_scale, out_dtype == H3B_INT8));
@@ -763,7 +766,8 @@ int h3b_rmsnorm(const float* x, const float* g, int rows, int d, float eps, void
 int h3b_gemm(const void* A, const void* B, int M, int N, int K, int ab_dtype, int epilogue, void* C,
              const float* scale_a, const float* scale_b, const float* rope_table, const h3b_dims* dims,
              float* row_absmax, void* scratch, size_t scratch_bytes, void* stream) {
-  if (!A || !B || !C) return H3B_ERR_NULL;
+  if (M != 0 && (!A || !C)) return H3B_ERR_NULL;
+  if (!B) return H3B_ERR_NULL;
   if (!aligned16(A) || !aligned16(B) || !aligned16(C)) return H3B_ERR_ALIGN;
   if (ab_dtype != H3B_BF16 && ab_dtype != H3B_INT8) return H3B_ERR_DTYPE;
   if (epilogue < H3B_EPI_F32 || epilogue > H3B_EPI_I32) return H3B_ERR_DTYPE;
@@ -782,6 +786,7 @@ int h3b_gemm(const void* A, const void* B, int M, int N, int K, int ab_dtype, in
     dm = *dims;
   }
   if (epilogue == H3B_EPI_GELU && ab_dtype == H3B_INT8 && !row_absmax) return H3B_ERR_NULL;
+  if (M == 0) return H3B_OK;
   Ctx c;
   H3B_TRY(device_ctx(static_cast<cudaStream_t>(stream), &c));
   if (scratch && !aligned16(scratch)) return H3B_ERR_ALIGN;
@@ -793,9 +798,10 @@ int h3b_gemm(const void* A, const void* B, int M, int N, int K, int ab_dtype, in
 
 int h3b_attention(const void* qkv, int S, int n_heads, int head_dim, void* o, void* scratch, size_t scratch_bytes,
                   void* stream) {
-  if (!qkv || !o) return H3B_ERR_NULL;
+  if (S != 0 && (!qkv || !o)) return H3B_ERR_NULL;
   if (!aligned16(qkv) || !aligned16(o) || (scratch && !aligned16(scratch))) return H3B_ERR_ALIGN;
   if (S < 0 || n_heads <= 0 || (head_dim != 64 && head_dim != 128)) return H3B_ERR_DIMS;
+  if (S == 0) return H3B_OK;
   Ctx c;
   H3B_TRY(device_ctx(static_cast<cudaStream_t>(stream), &c));
   H3B_CU(KID_ATTN, launch_attention(c, qkv, S, n_heads, head_dim, o, static_cast<float*>(scratch),

@@ -219,7 +219,8 @@ int h3b_denoise_ex(const h3b_dims* dims, const h3b_block_weights* blocks, int n_
  * clamped to [-127, 127]; an all-zero row gives s = 0, q = 0.
  * w: bf16 [rows, k]; q: int8 [rows, k]; scale: fp32 [rows].  Used once per
  * weight matrix (per output channel) and, inside the block, per token on
- * activations.  k must be a multiple of 8. */
+ * activations.  k must be a multiple of 8.  rows == 0 launches nothing (the
+ * pointers may then be NULL; k is still checked). */
 int h3b_quantize_weights(const void* w, int rows, int k, int8_t* q, float* scale, void* stream);
 
 /* Token reduction [fusion], [control]: xm[(f*H+r)*(W/2)+c'] =
@@ -289,7 +290,8 @@ int h3b_rope_table(const h3b_dims* dims, int merged, float* table, void* stream)
 /* RMSNorm of x fp32 [rows, d]: u = x * rsqrt(mean(x^2) + eps) * g.
  * out_dtype H3B_BF16: out is bf16 [rows, d], out_scale unused.
  * out_dtype H3B_INT8: out is int8 [rows, d] quantised per row (rule of
- * h3b_quantize_weights applied to the fp32 u) with scales in out_scale. */
+ * h3b_quantize_weights applied to the fp32 u) with scales in out_scale.
+ * rows == 0 launches nothing (the pointers may then be NULL). */
 int h3b_rmsnorm(const float* x, const float* g, int rows, int d, float eps,
                 void* out, float* out_scale, int out_dtype, void* stream);
 
@@ -312,14 +314,17 @@ int h3b_rmsnorm(const float* x, const float* g, int rows, int d, float eps,
  * long): with H3B_EPI_RESID, when the last wave of output tiles would leave
  * most SMs idle, those tail tiles are split along K over the idle SMs; their
  * fp32 partials go to scratch (up to 148 tiles x 128 KB) and are added into C
- * in a fixed order by a second kernel (deterministic).  NULL disables it. */
+ * in a fixed order by a second kernel (deterministic).  NULL disables it.
+ * M == 0 launches nothing (A and C may then be NULL; the other arguments are
+ * still checked). */
 int h3b_gemm(const void* A, const void* B, int M, int N, int K, int ab_dtype, int epilogue,
              void* C, const float* scale_a, const float* scale_b, const float* rope_table,
              const h3b_dims* dims, float* row_absmax, void* scratch, size_t scratch_bytes,
              void* stream);
 
 /* Quantise bf16 rows with a known max |row| (e.g. from H3B_EPI_GELU):
- * s[r] = absmax[r] / 127, q = rint(a / s) clamped, as h3b_quantize_weights. */
+ * s[r] = absmax[r] / 127, q = rint(a / s) clamped, as h3b_quantize_weights.
+ * rows == 0 launches nothing (the pointers may then be NULL). */
 int h3b_quantize_rows_absmax(const void* a, const float* absmax, int rows, int k,
                              int8_t* q, float* scale, void* stream);
 
@@ -330,11 +335,13 @@ int h3b_quantize_rows_absmax(const void* a, const float* absmax, int rows, int k
  * leave a last wave at most half full, those items are split along the keys
  * over the idle SMs; each part writes its unnormalised O, running max and sum
  * to scratch (up to 148 x 130 KB) and a second kernel merges the parts in a
- * fixed order.  NULL disables it. */
+ * fixed order.  NULL disables it.  S == 0 launches nothing (qkv and o may
+ * then be NULL). */
 int h3b_attention(const void* qkv, int S, int n_heads, int head_dim, void* o, void* scratch,
                   size_t scratch_bytes, void* stream);
 
-/* The attention kernel's FMA-pipe exp2 (used for one key pair in four):
+/* The FMA-pipe exp2 that the attention kernel can take for a share of its key
+ * pairs (a compile-time option, off by default: on B200 it slowed the kernel):
  * y = 2^n * p(x - n), n = rint(x), p a degree-3 polynomial fitted to 2^f on
  * [-1/2, 1/2] (max relative error 7.5e-5); x is clamped to >= -126.
  * x, y: fp32 [n] device buffers.  For accuracy tests of that approximation. */

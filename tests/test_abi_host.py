@@ -125,6 +125,25 @@ def test_gemm_argument_errors():
     assert g(fake, fake + 8, 128, 128, 128, 0, 0, fake, None, None, None, None, None, None, 0, None) == -2
 
 
+def test_empty_unit_calls_are_noops_before_device():
+    """rows / M / S == 0: nothing is launched and NULL buffers are accepted
+    (these return before any CUDA call, so they run without a GPU); the
+    remaining arguments are still validated."""
+    fake = 1 << 20
+    lib = h3b.lib
+    assert lib.h3b_quantize_weights(None, 0, 256, None, None, None) == 0
+    assert lib.h3b_quantize_weights(None, 0, 250, None, None, None) == -3                 # k % 8
+    assert lib.h3b_quantize_rows_absmax(None, None, 0, 1024, None, None, None) == 0
+    assert lib.h3b_rmsnorm(None, None, 0, 256, 1e-6, None, None, h3b.BF16, None) == 0
+    assert lib.h3b_rmsnorm(None, None, 0, 256, 1e-6, None, None, 7, None) == -4          # dtype
+    assert lib.h3b_gemm(None, fake, 0, 128, 128, 0, 1, None, None, None, None, None, None, None, 0, None) == 0
+    assert lib.h3b_gemm(None, fake, 0, 100, 128, 0, 1, None, None, None, None, None, None, None, 0, None) == -3
+    assert lib.h3b_gemm(None, None, 0, 128, 128, 0, 1, None, None, None, None, None, None, None, 0, None) == -1
+    assert lib.h3b_attention(None, 0, 4, 128, None, None, 0, None) == 0
+    assert lib.h3b_attention(None, 0, 4, 96, None, None, 0, None) == -3                   # head_dim
+    assert lib.h3b_flow_step(None, None, 0.5, 0.4, 0, None, None) == 0
+
+
 def test_extended_options_argument_errors():
     dm = h3b.dims_of(wlmod.WORKLOADS["block_d256_s288"])
     fake = 1 << 20

@@ -554,3 +554,24 @@ def test_attention_max_heads(cuda_dev):
     d = H * D
     ref = oracle.attention(q[:, :d], q[:, d:2 * d], q[:, 2 * d:], H)
     assert rel_l2(o, ref) < 1e-2 and max_abs(o, ref) < 3e-2
+
+
+def test_empty_inputs_launch_nothing(cuda_dev):
+    """Zero rows / tokens through the binding: empty results, no launch, no
+    device error."""
+    d, k = 256, 1024
+    g = torch.ones(d, device=cuda_dev)
+    with h3b.Trace() as tr:
+        u = h3b.rmsnorm(torch.empty((0, d), device=cuda_dev), g, 1e-6)
+        q, s = h3b.rmsnorm(torch.empty((0, d), device=cuda_dev), g, 1e-6, int8=True)
+        qw, sw = h3b.quantize_weights(torch.empty((0, k), dtype=torch.bfloat16, device=cuda_dev))
+        qa, sa = h3b.quantize_rows_absmax(torch.empty((0, k), dtype=torch.bfloat16, device=cuda_dev),
+                                          torch.empty(0, device=cuda_dev))
+        B = torch.ones((128, k), dtype=torch.bfloat16, device=cuda_dev)
+        c = h3b.gemm(torch.empty((0, k), dtype=torch.bfloat16, device=cuda_dev), B, h3b.EPI_BF16,
+                     torch.empty((0, 128), dtype=torch.bfloat16, device=cuda_dev))
+        o = h3b.attention(torch.empty((0, 3 * 2 * 128), dtype=torch.bfloat16, device=cuda_dev), 2, 128)
+        torch.cuda.synchronize()
+    assert tr.records == []
+    assert [t.shape[0] for t in (u, q, s, qw, sw, qa, sa, c, o)] == [0] * 9
+    assert h3b.device_error() == 0
