@@ -37,6 +37,8 @@ constexpr int BQ = 128, BKV = 128, THREADS = 384, KS = 3, VS = 2;
 // Register split (setmaxnreg): launch 384 x 168 = 64512; softmax warpgroups
 // 2 x 128 x 216 = 55296 plus control warpgroup 128 x 56 = 7168 -> 62464.
 constexpr int REG_SOFTMAX = 216, REG_CONTROL = 56;
+constexpr int SOFTMAX_THREADS = 256;
+constexpr int REG_SPLIT = SOFTMAX_THREADS * REG_SOFTMAX + (THREADS - SOFTMAX_THREADS) * REG_CONTROL;
 constexpr float RESCALE_LOG2 = 8.0f;
 constexpr int POLY_OF_8 = 0;   // key pairs (of every 8) that take the FMA-pipe exp2 (0: all on MUFU, measured fastest)
 // TMEM column of tile t's S/P and O regions
@@ -509,6 +511,13 @@ cudaError_t launch_attention(const Ctx& c, const void* qkv, int S, int n_heads, 
   const int smem = smem_bytes<128>();
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
+  // setmaxnreg.inc waits until the registers the block was launched with cover
+  // the split; a build whose register count could not grant it is refused here
+  // rather than left to wait.
+  cudaFuncAttributes fa;
+  e = cudaFuncGetAttributes(&fa, kern);
+  if (e != cudaSuccess) return e;
+  if (fa.numRegs * THREADS < REG_SPLIT) return cudaErrorInvalidConfiguration;
   AttnArgs a;
   a.S = S;
   a.n_heads = n_heads;
