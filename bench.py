@@ -60,7 +60,11 @@ METRIC = "DiT block tokens/s"
 DEFAULT_STEPS = {"block_d256_s288": 2000, "block_d3072_s6400": 300, "stack8_d5120_s6528": 30,
                  "block_int8_d5120_s20640": 60, "loop45_d5120_s6528": 2,
                  "preview40_d5120_s2784": 4}
-FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# used only when MEASURED_PEAKS.json is absent: an earlier measurement on B200s of
+# this kind (copy bandwidth; cuBLAS bf16 burst, and sustained under the 1 kW cap
+# at about 1.3 GHz)
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                  "clocks_under_load": {"sm_mhz_median": 1300.0}, "source": "fallback"}
 # B200 datasheet dense peaks (bf16, int8) and the HBM figure the block is held to
 NOMINAL = {"bf16_tflops": 2250.0, "int8_tops": 4500.0, "hbm_gbs": 8000.0}
 INT8_PEAK_FILE = os.path.join(ROOT, "profiles", "int8_peak.json")
@@ -86,7 +90,8 @@ def tensor_peak(pk, clocks, int8=False):
     power-capped clock the sustained peak.  INT8 uses its own measured pair
     when profiles/int8_peak.json exists, else the bf16 pair x 2 (the nominal
     4.5 / 2.25 ratio)."""
-    src = "MEASURED_PEAKS.json (cuBLAS bf16)"
+    src = ("fallback peaks (no MEASURED_PEAKS.json)" if pk.get("source") == "fallback"
+           else "MEASURED_PEAKS.json (cuBLAS bf16)")
     burst, sust = pk.get("bf16_tflops"), pk.get("bf16_tflops_sustained", pk.get("bf16_tflops"))
     f_s = (pk.get("clocks_under_load") or {}).get("sm_mhz_median")
     scale, nominal = 1.0, NOMINAL["bf16_tflops"]

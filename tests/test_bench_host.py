@@ -32,6 +32,18 @@ def test_tensor_peak_follows_the_sampled_clock(monkeypatch, tmp_path):
     assert bench.tensor_peak(PK, {"sm_mhz": 1250.0}, int8=True)["peak"] == 2500.0
 
 
+def test_fallback_peaks_are_labelled(monkeypatch, tmp_path):
+    """Without MEASURED_PEAKS.json the bench falls back to the earlier
+    measurement and says so in every basis it prints."""
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "INT8_PEAK_FILE", str(tmp_path / "absent.json"))
+    pk, src = bench.peaks()
+    assert src == "fallback" and pk["hbm_gbs"] == 6650.0
+    p = bench.tensor_peak(pk, {"sm_mhz": 1965.0})
+    assert p["peak"] == 1590.0 and p["basis"].startswith("fallback peaks")
+    assert "MEASURED_PEAKS.json (cuBLAS" not in bench.tensor_peak(pk, {"sm_mhz": 1300.0}, int8=True)["basis"]
+
+
 @pytest.mark.parametrize("name", ["block_d256_s288"])
 def test_oracle_chunks_are_one_block(name):
     wl = W.WORKLOADS[name]
